@@ -1,0 +1,345 @@
+"""Checks that pin the CPU oracle to facts outside itself.
+
+Each ``pin_*`` function takes the oracle module and raises AssertionError when
+the oracle disagrees with a printed value, a closed form, an invariant, a
+library routine or a brute-force evaluation.  ``test_oracle_pins.py`` runs them
+on the oracle as it is; ``test_oracle_mutations.py`` plants plausible mistakes
+in the oracle and checks that some pin fails for each.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand_case(seed, L, h, d, rk, rv, ab_std=1.0):
+    g = np.random.default_rng(seed)
+    return dict(
+        a_k=g.standard_normal((L, rk, h)) * ab_std,
+        b_k=g.standard_normal((L, rk, d)) / math.sqrt(d),
+        a_v=g.standard_normal((L, rv, h)) * ab_std,
+        b_v=g.standard_normal((L, rv, d)) / math.sqrt(d),
+        q=g.standard_normal((h, d)),
+    )
+
+
+# --------------------------------------------------------------------------- printed values
+def pin_cache_size(O):
+    """The page's printed per-token sizes: 2 h d_h = 8192 vs (R_K+R_V)(h+d_h) = 320."""
+    g = _golden("cache_size.json")
+    assert O.dense_elements_per_token(g["h"], g["d_h"]) == g["dense_elements_per_token"]
+    assert O.factor_elements_per_token(g["h"], g["d_h"], g["r_k"], g["r_v"]) == g["factor_elements_per_token"]
+    # the R=2 decode workload: 32 seqs x 32768 tokens x (2+2)(32+128) bf16 = 1.342 GB ("about 1.3 GB")
+    assert 32 * 32768 * O.factor_elements_per_token(32, 128, 2, 2) * 2 == 1_342_177_280
+
+
+# --------------------------------------------------------------------------- RoPE
+def pin_rope_closed_form(O):
+    """RoPE on unit vectors has closed forms: angle pos * base^(-2j/d_h)."""
+    # d_h = 2: theta_0 = 1, so e_0 at position p becomes (cos p, sin p)
+    for p in (0.0, 1.0, 2.5, 1000.0):
+        r = O.rope(np.array([1.0, 0.0]), p, 10000.0)
+        assert np.allclose(r, [math.cos(p), math.sin(p)], rtol=0, atol=1e-12)
+        r = O.rope(np.array([0.0, 1.0]), p, 10000.0)
+        assert np.allclose(r, [-math.sin(p), math.cos(p)], rtol=0, atol=1e-12)
+    # d_h = 4, base 100: theta_1 = 100^(-1/2) = 0.1, so pair 1 at position 10 turns by 1 rad
+    r = O.rope(np.array([0.0, 0.0, 1.0, 0.0]), 10.0, 100.0)
+    assert np.allclose(r, [0.0, 0.0, math.cos(1.0), math.sin(1.0)], rtol=0, atol=1e-12)
+    r = O.rope(np.array([1.0, 0.0, 0.0, 0.0]), 10.0, 100.0)
+    assert np.allclose(r, [math.cos(10.0), math.sin(10.0), 0.0, 0.0], rtol=0, atol=1e-12)
+    # d_h = 8, base 10000: theta_j = 10^(-j), pair 3 at position 1000 turns by 1 rad
+    x = np.zeros(8)
+    x[6] = 1.0
+    assert np.allclose(O.rope(x, 1000.0, 10000.0)[6:], [math.cos(1.0), math.sin(1.0)], atol=1e-12)
+
+
+def pin_rope_complex(O):
+    """Pairs rotate as complex numbers: (x + iy) * exp(i pos theta_j)."""
+    g = np.random.default_rng(7)
+    d = 16
+    x = g.standard_normal((5, d))
+    pos = np.array([0.0, 3.0, 17.0, 4095.0, 524287.0])
+    r = O.rope(x, pos, 10000.0)
+    j = np.arange(d // 2)
+    theta = 10000.0 ** (-(2.0 * j) / d)
+    zc = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(1j * pos[:, None] * theta[None, :])
+    assert np.allclose(r[:, 0::2], zc.real, atol=1e-12)
+    assert np.allclose(r[:, 1::2], zc.imag, atol=1e-12)
+    # rotations keep norms and position 0 is the identity
+    assert np.allclose(np.linalg.norm(r, axis=1), np.linalg.norm(x, axis=1), atol=1e-12)
+    assert np.array_equal(O.rope(x, 0.0, 10000.0), x)
+
+
+def _block_rotation(d, delta, base):
+    """T_delta as an explicit block-diagonal matrix (row-vector convention x T)."""
+    Tm = np.zeros((d, d))
+    for j in range(d // 2):
+        a = delta * base ** (-(2.0 * j) / d)
+        c, s = math.cos(a), math.sin(a)
+        # row vector (x, y) maps to (x c - y s, x s + y c)
+        Tm[2 * j, 2 * j], Tm[2 * j, 2 * j + 1] = c, s
+        Tm[2 * j + 1, 2 * j], Tm[2 * j + 1, 2 * j + 1] = -s, c
+    return Tm
+
+
+def pin_theorem_3_1(O):
+    """Theorem 3.1: Q~_t K~_s^T = Q_t T_{t-s} K_s^T with RoPE on the B factors only.
+
+    Built from factors: K_s from A_K, B_K with B_K rotated at s; Q_t from A_Q, B_Q
+    with B_Q rotated at t.  Also: scores do not change under a common shift.
+    """
+    g = np.random.default_rng(11)
+    h, d, rq, rk = 3, 8, 2, 2
+    base = 10000.0
+    a_q, b_q = g.standard_normal((rq, h)), g.standard_normal((rq, d))
+    a_k, b_k = g.standard_normal((rk, h)), g.standard_normal((rk, d))
+    q_plain = O.tensor_product(a_q, b_q)                  # [h, d]
+    k_plain = O.tensor_product(a_k, b_k)
+    for t, s in ((5, 2), (2, 5), (700, 3), (400000, 123456)):
+        q_rot = O.tensor_product(a_q, O.rope(b_q, float(t), base))
+        k_rot = O.tensor_product(a_k, O.rope(b_k, float(s), base))
+        lhs = np.einsum("ik,ik->i", q_rot, k_rot)
+        rhs = np.einsum("ik,kl,il->i", q_plain, _block_rotation(d, t - s, base), k_plain)
+        assert np.allclose(lhs, rhs, rtol=1e-9, atol=1e-9), (t, s, lhs, rhs)
+    # common shift of every position leaves decode scores (hence outputs) unchanged
+    c = _rand_case(3, 40, 4, 16, 2, 2)
+    pos = np.arange(40, dtype=np.float64)
+    o0 = O.decode_attention(c["a_k"], O.append_rope(c["b_k"], pos, base), c["a_v"], c["b_v"], c["q"], 40.0, 0.25, base)
+    for delta in (1.0, 1000.0, 400000.0):
+        o1 = O.decode_attention(c["a_k"], O.append_rope(c["b_k"], pos + delta, base), c["a_v"], c["b_v"],
+                                c["q"], 40.0 + delta, 0.25, base)
+        assert np.allclose(o0, o1, rtol=1e-9, atol=1e-11), delta
+
+
+# --------------------------------------------------------------------------- closed forms
+def pin_two_token_golden(O):
+    """Worked two-token example (tests/golden/two_token_decode.json), closed form."""
+    g = _golden("two_token_decode.json")
+    a_k, b_k = np.array(g["a_k"]), np.array(g["b_k"])
+    a_v, b_v = np.array(g["a_v"]), np.array(g["b_v"])
+    pos = np.array(g["positions"], dtype=np.float64)
+    q = np.array(g["q"])
+    o = O.decode_attention(a_k, O.append_rope(b_k, pos, g["rope_base"]), a_v, b_v, q, float(g["q_pos"]),
+                           1.0 / math.sqrt(g["d_h"]), g["rope_base"])
+    z0 = math.sqrt(2.0) * math.sin(1.0)
+    z1 = 1.0 / math.sqrt(2.0)
+    p0 = 1.0 / (1.0 + math.exp(z1 - z0))
+    assert np.allclose(o, [[p0, 3.0 * (1.0 - p0)]], rtol=0, atol=1e-13), o
+
+
+def pin_single_token(O):
+    """One cached token: softmax weight 1, so o_i = V_0[i] = (1/R_V) sum_r A_V[0,r,i] B_V[0,r,:]."""
+    c = _rand_case(5, 1, 3, 8, 2, 2)
+    o = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], c["q"], 9.0, 0.3, 10000.0)
+    v0 = np.zeros((3, 8))
+    for i in range(3):
+        for k in range(8):
+            v0[i, k] = (c["a_v"][0, 0, i] * c["b_v"][0, 0, k] + c["a_v"][0, 1, i] * c["b_v"][0, 1, k]) / 2.0
+    assert np.allclose(o, v0, rtol=0, atol=1e-13)
+
+
+def pin_zero_query_mean(O):
+    """q = 0: every score is 0, the weights are uniform and o is the mean of V."""
+    c = _rand_case(6, 9, 2, 8, 1, 2)
+    o = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], np.zeros((2, 8)), 3.0, 0.3, 10000.0)
+    v = np.einsum("sri,srk->sik", c["a_v"], c["b_v"]) / 2.0
+    assert np.allclose(o, v.mean(axis=0), rtol=0, atol=1e-13)
+
+
+def pin_duplicate_ranks(O):
+    """R copies of the same rank-1 factors equal the rank-1 result (the 1/R sits in the product)."""
+    c = _rand_case(8, 30, 4, 16, 1, 1)
+    o1 = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], c["q"], 30.0, 0.25, 10000.0)
+    for r in (2, 3):
+        rep = {k: np.repeat(c[k], r, axis=1) for k in ("a_k", "b_k", "a_v", "b_v")}
+        o2 = O.decode_attention(rep["a_k"], rep["b_k"], rep["a_v"], rep["b_v"], c["q"], 30.0, 0.25, 10000.0)
+        assert np.allclose(o1, o2, rtol=1e-12, atol=1e-14)
+
+
+def pin_factor_rescale(O):
+    """A -> cA, B -> B/c leaves the output unchanged (only the product A^T B matters)."""
+    c = _rand_case(9, 25, 3, 8, 2, 2)
+    o1 = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], c["q"], 25.0, 0.4, 10000.0)
+    o2 = O.decode_attention(c["a_k"] * 4.0, c["b_k"] / 4.0, c["a_v"] * 0.5, c["b_v"] * 2.0, c["q"], 25.0, 0.4,
+                            10000.0)
+    assert np.allclose(o1, o2, rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------- library routines
+def pin_mqa_sdpa(O):
+    """A_K = A_V = 1 with rank 1 makes every head share K and V (multi-query attention).
+
+    Compared with PyTorch's float64 scaled_dot_product_attention on the rotated
+    keys and values.
+    """
+    g = np.random.default_rng(12)
+    L, h, d = 37, 4, 16
+    b_k = g.standard_normal((L, 1, d)) / 4
+    b_v = g.standard_normal((L, 1, d))
+    q = g.standard_normal((h, d))
+    ones = np.ones((L, 1, h))
+    pos = np.arange(L, dtype=np.float64)
+    bkr = O.append_rope(b_k, pos, 500.0)
+    o = O.decode_attention(ones, bkr, ones, b_v, q, 44.0, 0.37, 500.0)
+    qr = torch.from_numpy(O.rope(q, 44.0, 500.0))[None, :, None, :]            # [1, h, 1, d]
+    kk = torch.from_numpy(bkr[:, 0, :]).expand(h, L, d)[None]
+    vv = torch.from_numpy(b_v[:, 0, :]).expand(h, L, d)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(qr, kk, vv, scale=0.37)[0, :, 0, :].numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+def pin_general_sdpa(O):
+    """For any factors, decode equals SDPA on K, V expanded per token by scalar loops."""
+    c = _rand_case(13, 21, 3, 8, 2, 1)
+    L, h, d = 21, 3, 8
+    k = np.zeros((h, L, d))
+    v = np.zeros((h, L, d))
+    for s in range(L):
+        for i in range(h):
+            for kk in range(d):
+                k[i, s, kk] = sum(c["a_k"][s, r, i] * c["b_k"][s, r, kk] for r in range(2)) / 2.0
+                v[i, s, kk] = c["a_v"][s, 0, i] * c["b_v"][s, 0, kk]
+    o = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], c["q"], 0.0, 0.5, 10000.0)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(c["q"])[:, None, :], torch.from_numpy(k), torch.from_numpy(v), scale=0.5)[:, 0, :].numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_causal_sdpa(O):
+    """Causal prefill equals SDPA with a causal mask on queries/keys expanded by loops."""
+    g = np.random.default_rng(14)
+    T, h, d, rq, rk, rv = 11, 2, 8, 3, 2, 2
+    a_q, b_q = g.standard_normal((T, rq, h)), g.standard_normal((T, rq, d))
+    a_k, b_k = g.standard_normal((T, rk, h)), g.standard_normal((T, rk, d))
+    a_v, b_v = g.standard_normal((T, rv, h)), g.standard_normal((T, rv, d))
+    pos = np.arange(T, dtype=np.float64)
+    bkr = O.append_rope(b_k, pos, 10000.0)
+    o = O.prefill_attention(a_k, bkr, a_v, b_v, a_q, b_q, pos, 0.3, 10000.0)
+    bqr = O.rope(b_q, pos[:, None], 10000.0)
+    Q = np.zeros((h, T, d)); K = np.zeros((h, T, d)); V = np.zeros((h, T, d))
+    for t in range(T):
+        for i in range(h):
+            for k in range(d):
+                Q[i, t, k] = sum(a_q[t, j, i] * bqr[t, j, k] for j in range(rq)) / rq
+                K[i, t, k] = sum(a_k[t, r, i] * bkr[t, r, k] for r in range(rk)) / rk
+                V[i, t, k] = sum(a_v[t, r, i] * b_v[t, r, k] for r in range(rv)) / rv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), torch.from_numpy(K), torch.from_numpy(V), is_causal=True, scale=0.3).numpy()
+    assert np.allclose(o, ref.transpose(1, 0, 2), rtol=1e-12, atol=1e-13)
+
+
+# --------------------------------------------------------------------------- brute force
+def _brute_rot(x, pos, base):
+    d = len(x)
+    out = [0.0] * d
+    for j in range(d // 2):
+        a = pos * base ** (-(2.0 * j) / d)
+        out[2 * j] = x[2 * j] * math.cos(a) - x[2 * j + 1] * math.sin(a)
+        out[2 * j + 1] = x[2 * j] * math.sin(a) + x[2 * j + 1] * math.cos(a)
+    return out
+
+
+def pin_brute_force_decode(O):
+    """Every step by scalar loops (math.cos/sin/exp, math.fsum) on tiny inputs."""
+    for seed, (L, h, d, rk, rv) in enumerate([(1, 1, 2, 1, 1), (3, 2, 4, 2, 1), (3, 2, 4, 1, 2), (5, 1, 6, 3, 3)]):
+        c = _rand_case(100 + seed, L, h, d, rk, rv)
+        pos = [float(3 * s + 1) for s in range(L)]
+        qpos, scale, base = 17.0, 0.7, 50.0
+        o = O.decode_attention(c["a_k"], O.append_rope(c["b_k"], np.array(pos), base), c["a_v"], c["b_v"],
+                               c["q"], qpos, scale, base)
+        for i in range(h):
+            qr = _brute_rot(list(c["q"][i]), qpos, base)
+            z = []
+            for s in range(L):
+                key = [0.0] * d
+                for r in range(rk):
+                    br = _brute_rot(list(c["b_k"][s, r]), pos[s], base)
+                    for k in range(d):
+                        key[k] += c["a_k"][s, r, i] * br[k] / rk
+                z.append(scale * math.fsum(qr[k] * key[k] for k in range(d)))
+            m = max(z)
+            w = [math.exp(x - m) for x in z]
+            tot = math.fsum(w)
+            for k in range(d):
+                ref = math.fsum(w[s] / tot * math.fsum(c["a_v"][s, r, i] * c["b_v"][s, r, k] / rv for r in range(rv))
+                                for s in range(L))
+                assert abs(o[i, k] - ref) <= 1e-12 * (1 + abs(ref)), (seed, i, k, o[i, k], ref)
+
+
+def pin_brute_force_prefill(O):
+    """Causal prefill with a previous chunk (P > 0) by scalar loops on tiny inputs."""
+    g = np.random.default_rng(21)
+    P, T, h, d, rq, rk, rv = 2, 3, 2, 4, 2, 1, 2
+    L = P + T
+    a_k, b_k = g.standard_normal((L, rk, h)), g.standard_normal((L, rk, d))
+    a_v, b_v = g.standard_normal((L, rv, h)), g.standard_normal((L, rv, d))
+    a_q, b_q = g.standard_normal((T, rq, h)), g.standard_normal((T, rq, d))
+    kpos = [float(s) for s in range(L)]
+    qpos = [float(P + t) for t in range(T)]
+    base, scale = 10000.0, 0.5
+    o = O.prefill_attention(a_k, O.append_rope(b_k, np.array(kpos), base), a_v, b_v, a_q, b_q,
+                            np.array(qpos), scale, base)
+    for t in range(T):
+        for i in range(h):
+            qv = [0.0] * d
+            for j in range(rq):
+                br = _brute_rot(list(b_q[t, j]), qpos[t], base)
+                for k in range(d):
+                    qv[k] += a_q[t, j, i] * br[k] / rq
+            z = []
+            for s in range(P + t + 1):
+                key = [0.0] * d
+                for r in range(rk):
+                    br = _brute_rot(list(b_k[s, r]), kpos[s], base)
+                    for k in range(d):
+                        key[k] += a_k[s, r, i] * br[k] / rk
+                z.append(scale * math.fsum(qv[k] * key[k] for k in range(d)))
+            m = max(z)
+            w = [math.exp(x - m) for x in z]
+            tot = math.fsum(w)
+            for k in range(d):
+                ref = math.fsum(w[s] / tot * math.fsum(a_v[s, r, i] * b_v[s, r, k] / rv for r in range(rv))
+                                for s in range(len(z)))
+                assert abs(o[t, i, k] - ref) <= 1e-12 * (1 + abs(ref)), (t, i, k)
+
+
+def pin_prefill_first_row(O):
+    """Prefill query 0 with no earlier chunk sees only slot 0: o = V_0."""
+    g = np.random.default_rng(22)
+    T, h, d = 5, 2, 8
+    a_k, b_k = g.standard_normal((T, 2, h)), g.standard_normal((T, 2, d))
+    a_v, b_v = g.standard_normal((T, 2, h)), g.standard_normal((T, 2, d))
+    a_q, b_q = g.standard_normal((T, 6, h)), g.standard_normal((T, 6, d))
+    o = O.prefill_attention(a_k, b_k, a_v, b_v, a_q, b_q, np.arange(T, dtype=np.float64), 0.3, 10000.0, rows=[0])
+    v0 = (a_v[0].T @ b_v[0]) / 2.0
+    assert np.allclose(o[0], v0, rtol=0, atol=1e-13)
+
+
+ALL_PINS = [
+    pin_cache_size,
+    pin_rope_closed_form,
+    pin_rope_complex,
+    pin_theorem_3_1,
+    pin_two_token_golden,
+    pin_single_token,
+    pin_zero_query_mean,
+    pin_duplicate_ranks,
+    pin_factor_rescale,
+    pin_mqa_sdpa,
+    pin_general_sdpa,
+    pin_prefill_causal_sdpa,
+    pin_brute_force_decode,
+    pin_brute_force_prefill,
+    pin_prefill_first_row,
+]

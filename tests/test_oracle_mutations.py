@@ -1,0 +1,87 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+A pin set that let one of these through would not be pinning the oracle.
+"""
+import numpy as np
+import pytest
+
+import oracle.tpa_oracle as O
+from tests.oracle_pins import ALL_PINS
+
+_rope = O.rope
+_tp = O.tensor_product
+_freq = O.rope_frequencies
+_decode = O.decode_attention
+_prefill_q = O.prefill_queries
+
+
+def _rope_flipped(x, pos, base):              # wrong rotation sense
+    return _rope(x, -np.asarray(pos, dtype=np.float64), base)
+
+
+def _rope_rotate_half(x, pos, base):          # pairs (j, j + d/2) instead of (2j, 2j+1)
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    perm = np.concatenate([np.arange(0, d, 2), np.arange(1, d, 2)])
+    inv = np.argsort(perm)
+    y = x[..., inv]
+    return _rope(y, pos, base)[..., perm]
+
+
+def _freq_no_two(d_h, base):                  # theta_j = base^(-j/d_h)
+    j = np.arange(d_h // 2, dtype=np.float64)
+    return np.power(np.float64(base), -j / d_h)
+
+
+def _tp_no_rank_scale(a, b):                  # dropped 1/R
+    return _tp(a, b) * np.asarray(a).shape[-2]
+
+
+def _tp_first_rank_only(a, b):                # dropped terms of the rank sum
+    a = np.asarray(a, dtype=np.float64)
+    return _tp(a[..., :1, :], np.asarray(b, dtype=np.float64)[..., :1, :])
+
+
+def _tp_transposed(a, b):                     # head/feature factor roles swapped in a square case
+    out = _tp(a, b)
+    if out.shape[-1] == out.shape[-2]:
+        return np.swapaxes(out, -1, -2)
+    return np.flip(out, axis=-2)
+
+
+def _decode_no_query_rope(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block=8192):
+    return _decode(a_k, b_k_rot, a_v, b_v, q, 0.0, scale, base, block)
+
+
+def _decode_scale_squared(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block=8192):
+    return _decode(a_k, b_k_rot, a_v, b_v, q, q_pos, scale * scale, base, block)
+
+
+def _prefill_q_no_rope(a_q, b_q, q_pos, base):
+    return _tp(a_q, b_q)
+
+
+MUTANTS = {
+    "rope_flipped": ("rope", _rope_flipped),
+    "rope_rotate_half": ("rope", _rope_rotate_half),
+    "freq_no_two": ("rope_frequencies", _freq_no_two),
+    "no_rank_scale": ("tensor_product", _tp_no_rank_scale),
+    "first_rank_only": ("tensor_product", _tp_first_rank_only),
+    "transposed_product": ("tensor_product", _tp_transposed),
+    "decode_no_query_rope": ("decode_attention", _decode_no_query_rope),
+    "decode_scale_squared": ("decode_attention", _decode_scale_squared),
+    "prefill_no_query_rope": ("prefill_queries", _prefill_q_no_rope),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_some_pin_catches(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(O)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"mutant {name} passed every pin"
