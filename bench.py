@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of TPA attention over a factorized KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--kernel auto|simt|tensor]
+
+One step of a decode workload is one generation step of the whole batch: the
+newest token's factors are written into the cache (RoPE on B_K at its
+position) and its query attends every cached token (query RoPE, factor
+scores, online softmax, rank-R value updates, split-KV log-sum-exp merge).
+The cache keeps a fixed length: the newest token is rewritten in place each
+step, so every step attends exactly sum_b L_b tokens.
+
+One step of the prefill workload writes the prompt's factors and runs the
+causal prefill over them.
+
+Rank 0 prints one JSON line.  Under torchrun every rank runs its own batch on
+its own GPU (weak scaling, no collective on the data path); the time is the
+maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cached tokens attended/sec (TPA decode) + achieved HBM GB/s vs peak, 1×B200"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# --------------------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, kernel_sources):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_sha") != source_sha(kernel_sources):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), sm_max=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hw_th=parts[6], sw_th=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hw_th", "hw_thermal_slowdown"),
+                              ("sw_th", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        loaded = [r["sm"] for r in rows if r["power"] > 200.0] or [r["sm"] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r["sm_max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "power_w_max": max(r["power"] for r in rows)}
+
+
+# --------------------------------------------------------------------------- CPU oracle runs
+def _oracle_task(args):
+    """One decode over a slice of a sequence with the float64 oracle, RoPE on B_K
+    included (runs in a spawned worker)."""
+    import oracle.tpa_oracle as O
+    a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base = args
+    f = lambda a: np.asarray(a, dtype=np.float64)
+    O.decode_attention_from_unrotated(f(a_k), f(b_k), f(a_v), f(b_v), positions, f(q), q_pos, scale, base)
+    return a_k.shape[0]
+
+
+def _decode_tasks(host, w, n_tasks, slice_tokens):
+    """Oracle tasks cycling over the workload's sequences, `slice_tokens` tokens each."""
+    B = host["a_k"].shape[0]
+    tasks = []
+    scale = 1.0 / math.sqrt(w.head_dim)
+    for t in range(n_tasks):
+        b = t % B
+        L = int(host["lengths"][b])
+        n = min(L, slice_tokens)
+        s0 = (t // B * n) % max(1, L - n + 1)
+        tasks.append((host["a_k"][b, s0:s0 + n], host["b_k"][b, s0:s0 + n], host["a_v"][b, s0:s0 + n],
+                      host["b_v"][b, s0:s0 + n], np.arange(s0, s0 + n), host["q"][b], float(host["q_pos"][b]),
+                      scale, w.rope_base))
+    return tasks
+
+
+def cpu_oracle_rate(host, w, target_s: float, workers: int):
+    """Cached tokens attended per second by the float64 oracle on `workers` host cores."""
+    slice_tokens = 4096
+    t0 = time.perf_counter()
+    n1 = _oracle_task(_decode_tasks(host, w, 1, slice_tokens)[0])
+    per_token = (time.perf_counter() - t0) / n1
+    per_task = per_token * min(slice_tokens, int(host["lengths"].max()))
+    n_tasks = max(workers, int(target_s * workers / max(per_task, 1e-6)))
+    n_tasks = (n_tasks + workers - 1) // workers * workers
+    tasks = _decode_tasks(host, w, n_tasks, slice_tokens)
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        pool.map(_oracle_task, tasks[:workers])          # import + warm
+        t0 = time.perf_counter()
+        done = sum(pool.map(_oracle_task, tasks, chunksize=1))
+        dt = time.perf_counter() - t0
+    return done / dt, dict(tokens=done, seconds=dt, tasks=len(tasks), slice_tokens=slice_tokens)
+
+
+# --------------------------------------------------------------------------- decode bench
+def decode_host_inputs(w, rank):
+    from factorized_kv_cache_b200 import synthetic as S
+    ww = w.replace(seed=w.seed + 1000 * rank) if rank else w
+    return S.decode_inputs(ww)
+
+
+def run_ours_decode(args, w, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+    from factorized_kv_cache_b200 import synthetic as S
+    from factorized_kv_cache_b200 import tpa as T
+
+    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR}[args.kernel]
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    esize = 4 if w.dtype == "f32" else 2
+    x = decode_host_inputs(w, rank)
+    B, cap = x["a_k"].shape[:2]
+    lengths = x["lengths"].numpy().astype(np.int64)
+    per_tok = (w.r_k + w.r_v) * (w.heads + w.head_dim) * esize
+    cache_bytes = B * cap * per_tok
+    copies = 1 if cache_bytes >= 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / cache_bytes)) + 1
+
+    # copy 0 from the seeded inputs through the product append path, the rest cloned
+    c0 = T.TpaCache.allocate(B, cap, w.heads, w.head_dim, w.r_k, w.r_v, dtype=dt, rope_base=w.rope_base, device=dev)
+    T.tpa_cache_append(c0, x["positions"].to(dev), x["a_k"].to(dev), x["b_k"].to(dev), x["a_v"].to(dev),
+                       x["b_v"].to(dev))
+    c0.seq_lens.copy_(x["lengths"].to(dev))
+    caches = [c0] + [T.TpaCache(c0.a_k.clone(), c0.b_k.clone(), c0.a_v.clone(), c0.b_v.clone(), c0.seq_lens.clone(),
+                                w.rope_base) for _ in range(copies - 1)]
+    # the newest token of every sequence is rewritten each step: slot L_b-1, position L_b-1
+    newest = torch.from_numpy((lengths - 1).clip(min=0).astype(np.int32))[:, None]
+    slots = newest.to(dev)
+    pos = newest.to(dev)
+    new_f = {k: x[k][torch.arange(B), torch.from_numpy((lengths - 1).clip(min=0))][:, None].contiguous().to(dev)
+             for k in ("a_k", "b_k", "a_v", "b_v")}
+    q = x["q"].to(dev)
+    q_pos = newest[:, 0].contiguous().to(dev)
+    out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32, device=dev)
+    splits = T.tpa_decode_default_splits(c0, cap, kernel)
+    ws = T.workspace(T.tpa_decode_workspace_size(c0, cap, 0, kernel), dev)
+    tokens_per_step = int(lengths.sum())
+
+    def write(c):
+        T.tpa_cache_write_slots(caches[c], slots, pos, new_f["a_k"], new_f["b_k"], new_f["a_v"], new_f["b_v"])
+
+    def decode(c):
+        T.tpa_decode_attention(caches[c], q, q_pos, out=out, max_len=cap, kernel=kernel, workspace_buf=ws)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for c in range(copies):     # eager run first (loads the module, checks arguments)
+            write(c)
+            decode(c)
+    torch.cuda.synchronize(dev)
+    gw, gd = [], []
+    for c in range(copies):
+        g1, g2 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            write(c)
+        with torch.cuda.graph(g2, stream=stream):
+            decode(c)
+        gw.append(g1)
+        gd.append(g2)
+    torch.cuda.synchronize(dev)
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set after set-up")
+
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for k in range(W):
+            gw[k % copies].replay()
+            gd[k % copies].replay()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for k in range(K):
+            c = (W + k) % copies
+            gw[c].replay()
+            ev[k][0].record(stream)
+            gd[c].replay()
+            ev[k][1].record(stream)
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of the output
+    host_in = {k: v.cpu().pin_memory() for k, v in new_f.items()}
+    host_q = x["q"].pin_memory()
+    host_idx = newest.pin_memory()
+    host_out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32).pin_memory()
+    dev_in = {k: torch.empty_like(v) for k, v in new_f.items()}
+    dev_q = torch.empty_like(q)
+    dev_idx = torch.empty_like(slots)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + host_q.numel() * host_q.element_size() + \
+        host_idx.numel() * 4
+    d2h = host_out.numel() * 4
+    e2e_steps = max(1, min(K, 2000))
+
+    def e2e_step(c):
+        with torch.cuda.stream(stream):
+            for k2, v in host_in.items():
+                dev_in[k2].copy_(v, non_blocking=True)
+            dev_q.copy_(host_q, non_blocking=True)
+            dev_idx.copy_(host_idx, non_blocking=True)
+            T.tpa_cache_write_slots(caches[c], dev_idx, dev_idx, dev_in["a_k"], dev_in["b_k"], dev_in["a_v"],
+                                    dev_in["b_v"], stream=stream)
+            T.tpa_decode_attention(caches[c], dev_q, dev_idx[:, 0], out=out, max_len=cap, kernel=kernel,
+                                   workspace_buf=ws, stream=stream)
+            host_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for k in range(min(W, 10)):
+        e2e_step(k % copies)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for k in range(e2e_steps):
+        e2e_step(k % copies)
+    e2e_s = time.perf_counter() - t0
+    if world > 1:
+        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+
+    launches_per_step = 1 + 1 + (1 if splits > 1 else 0)
+    bytes_per_decode = tokens_per_step * per_tok + B * w.heads * w.head_dim * (esize + 4)
+    mean_decode_s = statistics.mean(decode_ms) / 1e3
+    peaks, kind = measured_peaks()
+    achieved = bytes_per_decode / mean_decode_s / 1e9
+    kernel_src = ["factorized_kv_cache_b200/csrc/attention_simt.cu"] if (
+        kernel == T.TPA_KERNEL_SIMT or w.dtype == "f32") else ["factorized_kv_cache_b200/csrc/decode_tensor.cu"]
+    kernel_src = [p for p in kernel_src if os.path.exists(os.path.join(ROOT, p))]
+    res = {
+        "metric": METRIC,
+        "value": world * tokens_per_step * K / (elapsed_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": elapsed_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded Philox normals; A~N(0,1), B~N(0,1/d_h), q~N(0,1))",
+        "config": {
+            "workload": w.name, "batch": B, "seq_len": int(lengths.max()), "seq_len_min": int(lengths.min()),
+            "heads": w.heads, "head_dim": w.head_dim, "r_k": w.r_k, "r_v": w.r_v,
+            "tokens_attended_per_step": tokens_per_step, "kernel": args.kernel, "splits": splits,
+            "step": "write newest token (RoPE on B_K) + decode attention (+ LSE merge), CUDA graphs",
+            "l2": (f"inputs larger than L2: {copies} cache copies rotated ({copies * cache_bytes / 2**20:.0f} MiB "
+                   f"> 126 MiB L2)" if copies > 1 else f"inputs larger than L2 ({cache_bytes / 2**20:.0f} MiB)"),
+            "parallelism": f"dp{world} (independent batches, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(w.name, kernel_src) if kernel_src else None,
+            "peak_kind": kind, "kernel": "decode attention call (split kernel + merge)",
+            "algorithmic_bytes_per_launch": bytes_per_decode, "mean_launch_us": mean_decode_s * 1e6,
+        },
+        "e2e": {"value": world * tokens_per_step * e2e_steps / e2e_s, "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": K * launches_per_step,
+        "clocks": clk,
+    }
+    return res, x, lengths
+
+
+def _host_arrays(x, lengths):
+    host = {k: x[k].float().numpy() for k in ("a_k", "b_k", "a_v", "b_v", "q")}
+    host["lengths"] = lengths
+    host["q_pos"] = (lengths - 1).clip(min=0)
+    return host
+
+
+def add_cpu_baseline(res, x, w, lengths, target_s):
+    host = _host_arrays(x, lengths)
+    host["lengths"] = lengths
+    host["q_pos"] = (lengths - 1).clip(min=0)
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    rate, info = cpu_oracle_rate(host, w, target_s, workers)
+    res["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                           "sample": f"{info['tasks']} decode slices of <= {info['slice_tokens']} cached tokens "
+                                     f"(all {w.heads} heads) of this workload, float64 oracle, "
+                                     f"{info['seconds']:.1f} s on {workers} spawned processes"}
+
+
+def run_reference(args, w):
+    """The float64 CPU oracle as the reference arm (host cores only)."""
+    x = decode_host_inputs(w, 0)
+    lengths = x["lengths"].numpy().astype(np.int64)
+    host = _host_arrays(x, lengths)
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    K, W = args.steps, args.warmup
+    budget = 150.0 / max(1, K + W)
+    slice_tokens = 4096
+    t0 = time.perf_counter()
+    _oracle_task(_decode_tasks(host, w, 1, slice_tokens)[0])
+    per_task = time.perf_counter() - t0
+    tasks_per_step = max(1, min(workers, int(budget * workers / max(per_task, 1e-6))))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        for k in range(W):
+            pool.map(_oracle_task, _decode_tasks(host, w, tasks_per_step, slice_tokens))
+        t0 = time.perf_counter()
+        done = 0
+        for k in range(K):
+            done += sum(pool.map(_oracle_task, _decode_tasks(host, w, tasks_per_step, slice_tokens)))
+        dt = time.perf_counter() - t0
+    value = done / dt
+    sample = (f"each step: {tasks_per_step} decode slices of <= {slice_tokens} cached tokens (all heads) of "
+              f"{w.name}, float64 oracle on {workers} spawned processes")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": K,
+        "warmup": W, "ms_per_step": dt / max(1, K) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": int(x["a_k"].shape[0]), "seq_len": int(lengths.max()),
+                   "heads": w.heads, "head_dim": w.head_dim, "r_k": w.r_k, "r_v": w.r_v},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_b8_l8k")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from factorized_kv_cache_b200 import synthetic as S
+    w = S.WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    try:
+        res, x, lengths = run_ours_decode(args, w, rank, world, dev)
+        if rank == 0 and args.cpu_seconds > 0:
+            add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

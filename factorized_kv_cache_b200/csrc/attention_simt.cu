@@ -1,0 +1,301 @@
+// CUDA-core attention over the factorized cache (fp32 FMA), every supported
+// shape and both dtypes.  It serves the fp32 decode workload, the shapes the
+// tensor-core kernels do not cover, and as the CUDA-core baseline.
+//
+// Per cached token s and head i (Tensor Product Attention Is All You Need,
+// sections 关键设计 and FlashTPA; the factors are never expanded to K or V):
+//   S'[r, i] = q~_i . B~_K[s, r]                       (rank-r feature dot)
+//   z[i]     = scale * (1/R_K) sum_r A_K[s, r, i] S'[r, i]
+//   online softmax over s (running max m, sum l; base-2 exponentials)
+//   o_i     += p (1/R_V) sum_r A_V[s, r, i] B_V[s, r, :]   (rank-R_V update)
+// A CTA owns one (query, split) pair.  Eight threads share a head, each
+// holding d_h/8 features of q~ and of the accumulator; their partial dots are
+// summed with three xor-shuffles.  Token groups inside the CTA stride over
+// the split's tokens and are merged through shared memory at the end.
+#include <math.h>
+
+#include "device_common.cuh"
+#include "tpa_internal.h"
+
+namespace tpa {
+namespace {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSlices = 8;
+
+template <typename T, int SL>
+__device__ __forceinline__ void load_slice(const T* __restrict__ p, float* out) {
+  constexpr int V = Vec16<T>::N;
+  if constexpr (SL % V == 0) {
+#pragma unroll
+    for (int k = 0; k < SL; k += V) load16_f32(p + k, out + k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < SL; ++k) out[k] = to_f32(p[k]);
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads) simt_attention_kernel(const __grid_constant__ SimtArgs a) {
+  constexpr int SL = D / kSlices;
+  const int h = a.cache.heads;
+  const int rk = a.cache.r_k, rv = a.cache.r_v;
+  const int group = kSlices * h;
+  const int G = kSimtThreads / group;
+  const int tid = threadIdx.x;
+  const int g = tid / group;
+  const bool lane_on = g < G;
+  const int i = lane_on ? (tid % group) / kSlices : 0;
+  const int c = tid % kSlices;
+
+  const int qi = blockIdx.y;
+  const int b = qi / a.q_per_seq;
+  const int t = qi % a.q_per_seq;
+  const int split = blockIdx.x;
+
+  int len = a.cache.seq_lens[b];
+  int limit;
+  if (a.causal) {
+    const int P = len - a.q_per_seq;
+    if (len > a.cache.capacity || P < 0) {
+      if (tid == 0 && split == 0) atomicOr(a.err, TPA_DEVERR_PREFILL_LEN);
+      return;  // leave this query's output untouched
+    }
+    limit = P + t + 1;
+  } else {
+    if (len < 0 || len > a.cache.capacity || len > a.max_len) {
+      if (tid == 0 && split == 0) atomicOr(a.err, TPA_DEVERR_LEN_RANGE);
+      len = min(max(len, 0), min(a.cache.capacity, a.max_len));
+    }
+    limit = len;
+  }
+  const int s_begin = split * a.plan.chunk;
+  const int s_end = min(limit, s_begin + a.plan.chunk);
+
+  // q~ slice for head i, features [c*SL, c*SL+SL)
+  float qv[SL];
+  if (a.q_rotated_f32) {
+    const float* qp = static_cast<const float*>(a.q) + (static_cast<size_t>(qi) * h + i) * D + c * SL;
+#pragma unroll
+    for (int k = 0; k < SL; ++k) qv[k] = qp[k];
+  } else {
+    const T* qp = static_cast<const T*>(a.q) + (static_cast<size_t>(b) * h + i) * D + c * SL;
+    load_slice<T, SL>(qp, qv);
+    const int pos = a.q_pos[b];
+#pragma unroll
+    for (int p = 0; p < SL / 2; ++p) {
+      float cs, sn;
+      rope_cos_sin(pos, a.rope.theta[(c * SL) / 2 + p], &cs, &sn);
+      rope_pair(qv[2 * p], qv[2 * p + 1], cs, sn);
+    }
+  }
+
+  const float zs = a.scale * kLog2e / static_cast<float>(rk);
+  const float inv_rv = 1.0f / static_cast<float>(rv);
+  const size_t cap = a.cache.capacity;
+  const T* AK = static_cast<const T*>(a.cache.a_k) + static_cast<size_t>(b) * cap * rk * h;
+  const T* BK = static_cast<const T*>(a.cache.b_k) + static_cast<size_t>(b) * cap * rk * D;
+  const T* AV = static_cast<const T*>(a.cache.a_v) + static_cast<size_t>(b) * cap * rv * h;
+  const T* BV = static_cast<const T*>(a.cache.b_v) + static_cast<size_t>(b) * cap * rv * D;
+
+  float m = -INFINITY, l = 0.0f;
+  float acc[SL];
+#pragma unroll
+  for (int k = 0; k < SL; ++k) acc[k] = 0.0f;
+
+  for (int base = s_begin; base < s_end; base += G) {
+    const int s = base + g;
+    const bool valid = lane_on && s < s_end;
+    float z = 0.0f;
+    for (int r = 0; r < rk; ++r) {
+      float part = 0.0f;
+      float av = 0.0f;
+      if (valid) {
+        float kb[SL];
+        load_slice<T, SL>(BK + (static_cast<size_t>(s) * rk + r) * D + c * SL, kb);
+#pragma unroll
+        for (int k = 0; k < SL; ++k) part = fmaf(qv[k], kb[k], part);
+        av = to_f32(AK[(static_cast<size_t>(s) * rk + r) * h + i]);
+      }
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      part += __shfl_xor_sync(0xffffffffu, part, 4);
+      z = fmaf(av, part, z);
+    }
+    if (valid) {
+      z *= zs;
+      const float m_new = fmaxf(m, z);
+      const float corr = exp2f(m - m_new);
+      const float p = exp2f(z - m_new);
+      l = fmaf(l, corr, p);
+      float vv[SL];
+#pragma unroll
+      for (int k = 0; k < SL; ++k) vv[k] = 0.0f;
+      for (int r = 0; r < rv; ++r) {
+        float vb[SL];
+        load_slice<T, SL>(BV + (static_cast<size_t>(s) * rv + r) * D + c * SL, vb);
+        const float w = to_f32(AV[(static_cast<size_t>(s) * rv + r) * h + i]);
+#pragma unroll
+        for (int k = 0; k < SL; ++k) vv[k] = fmaf(w, vb[k], vv[k]);
+      }
+      const float pw = p * inv_rv;
+#pragma unroll
+      for (int k = 0; k < SL; ++k) acc[k] = fmaf(acc[k], corr, pw * vv[k]);
+      m = m_new;
+    }
+  }
+
+  // merge the token groups of this CTA
+  __shared__ float s_m[kSimtThreads / kSlices];
+  __shared__ float s_l[kSimtThreads / kSlices];
+  __shared__ float s_o[kSimtThreads / kSlices][D];
+  const int slot = g * h + i;  // < G*h <= 32
+  if (lane_on) {
+    if (c == 0) {
+      s_m[slot] = m;
+      s_l[slot] = l;
+    }
+#pragma unroll
+    for (int k = 0; k < SL; ++k) s_o[slot][c * SL + k] = acc[k];
+  }
+  __syncthreads();
+  if (!lane_on || g != 0) return;
+  float M = -INFINITY;
+  for (int gg = 0; gg < G; ++gg) M = fmaxf(M, s_m[gg * h + i]);
+  float L = 0.0f;
+  float O[SL];
+#pragma unroll
+  for (int k = 0; k < SL; ++k) O[k] = 0.0f;
+  if (M != -INFINITY) {
+    for (int gg = 0; gg < G; ++gg) {
+      const float mg = s_m[gg * h + i];
+      const float wgt = (mg == -INFINITY) ? 0.0f : exp2f(mg - M);
+      L = fmaf(s_l[gg * h + i], wgt, L);
+#pragma unroll
+      for (int k = 0; k < SL; ++k) O[k] = fmaf(s_o[gg * h + i][c * SL + k], wgt, O[k]);
+    }
+  }
+  if (a.plan.splits == 1) {
+    float* op = a.out + (static_cast<size_t>(qi) * h + i) * D + c * SL;
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int k = 0; k < SL; ++k) op[k] = O[k] * inv;
+  } else {
+    const size_t part = (static_cast<size_t>(qi) * a.plan.splits + split) * h + i;
+    if (c == 0) {
+      a.ws_ml[2 * part] = M;
+      a.ws_ml[2 * part + 1] = L;
+    }
+    float* op = a.ws_o + part * D + c * SL;
+#pragma unroll
+    for (int k = 0; k < SL; ++k) op[k] = O[k];
+  }
+}
+
+template <typename T>
+cudaError_t launch_simt_t(const SimtArgs& a, cudaStream_t stream) {
+  dim3 grid(a.plan.splits, a.cache.batch * a.q_per_seq);
+  switch (a.cache.head_dim) {
+    case 16: simt_attention_kernel<T, 16><<<grid, kSimtThreads, 0, stream>>>(a); break;
+    case 32: simt_attention_kernel<T, 32><<<grid, kSimtThreads, 0, stream>>>(a); break;
+    case 64: simt_attention_kernel<T, 64><<<grid, kSimtThreads, 0, stream>>>(a); break;
+    case 128: simt_attention_kernel<T, 128><<<grid, kSimtThreads, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+// Log-sum-exp merge: M = max_j m_j, L = sum_j l_j 2^(m_j-M),
+// o = sum_j o_j 2^(m_j-M) / L (m in base-2 units).  One CTA per (query, head).
+__global__ void merge_kernel(const __grid_constant__ MergeArgs a) {
+  // with programmatic dependent launch, wait here for the split kernel's writes
+  if (a.use_pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int q = blockIdx.x, i = blockIdx.y;
+  const size_t row = static_cast<size_t>(q) * a.splits;
+  float M = -INFINITY;
+  for (int j = 0; j < a.splits; ++j) M = fmaxf(M, a.ws_ml[2 * ((row + j) * a.heads + i)]);
+  for (int k = threadIdx.x; k < a.head_dim; k += blockDim.x) {
+    float L = 0.0f, O = 0.0f;
+    if (M != -INFINITY) {
+      for (int j = 0; j < a.splits; ++j) {
+        const size_t part = (row + j) * a.heads + i;
+        const float mj = a.ws_ml[2 * part];
+        if (mj == -INFINITY) continue;
+        const float w = exp2f(mj - M);
+        L = fmaf(a.ws_ml[2 * part + 1], w, L);
+        O = fmaf(a.ws_o[part * a.head_dim + k], w, O);
+      }
+    }
+    a.out[(static_cast<size_t>(q) * a.heads + i) * a.head_dim + k] = L > 0.0f ? O / L : 0.0f;
+  }
+}
+
+// Dense rotated prefill queries (fp32): Q[t][i] = (1/R_Q) sum_j A_Q[t,j,i] RoPE(B_Q[t,j], pos_t)
+// (section 解决思路 for the Q factorization, Theorem 3.1 for RoPE on B_Q).
+template <typename T>
+__global__ void prefill_q_kernel(const __grid_constant__ PrefillQArgs a) {
+  extern __shared__ float s_bq[];  // [r_q][head_dim]
+  const int t = blockIdx.x, b = blockIdx.y;
+  const int d = a.head_dim, h = a.heads, rq = a.r_q;
+  const size_t tok = static_cast<size_t>(b) * a.n_tokens + t;
+  const int pos = a.q_pos[tok];
+  const T* bq = static_cast<const T*>(a.b_q) + tok * rq * d;
+  for (int e = threadIdx.x; e < rq * d / 2; e += blockDim.x) {
+    const int j = e / (d / 2), p = e % (d / 2);
+    float x = to_f32(bq[j * d + 2 * p]), y = to_f32(bq[j * d + 2 * p + 1]);
+    float cs, sn;
+    rope_cos_sin(pos, a.rope.theta[p], &cs, &sn);
+    rope_pair(x, y, cs, sn);
+    s_bq[j * d + 2 * p] = x;
+    s_bq[j * d + 2 * p + 1] = y;
+  }
+  __syncthreads();
+  const T* aq = static_cast<const T*>(a.a_q) + tok * rq * h;
+  const float inv_rq = 1.0f / static_cast<float>(rq);
+  float* qo = a.q_out + tok * h * d;
+  for (int e = threadIdx.x; e < h * d; e += blockDim.x) {
+    const int i = e / d, k = e % d;
+    float acc = 0.0f;
+    for (int j = 0; j < rq; ++j) acc = fmaf(to_f32(aq[j * h + i]), s_bq[j * d + k], acc);
+    qo[e] = acc * inv_rq;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_simt_attention(const SimtArgs& a, cudaStream_t stream) {
+  if (a.cache.dtype == TPA_F32) return launch_simt_t<float>(a, stream);
+  return launch_simt_t<__nv_bfloat16>(a, stream);
+}
+
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream) {
+  dim3 grid(a.n_queries, a.heads);
+  const int threads = a.head_dim < 32 ? 32 : a.head_dim;
+  if (!a.use_pdl) {
+    merge_kernel<<<grid, threads, 0, stream>>>(a);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, merge_kernel, a);
+}
+
+cudaError_t launch_prefill_q(const PrefillQArgs& a, cudaStream_t stream) {
+  dim3 grid(a.n_tokens, a.batch);
+  const size_t smem = static_cast<size_t>(a.r_q) * a.head_dim * sizeof(float);
+  if (a.dtype == TPA_F32) {
+    prefill_q_kernel<float><<<grid, 128, smem, stream>>>(a);
+  } else {
+    prefill_q_kernel<__nv_bfloat16><<<grid, 128, smem, stream>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tpa

@@ -1,0 +1,72 @@
+// Device helpers shared by the kernels: element conversion, 16-byte vector
+// loads/stores and the RoPE angle (double-precision angle, fp32 rotation).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tpa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T>
+struct Vec16;  // 16 bytes of T
+template <>
+struct Vec16<float> {
+  static constexpr int N = 4;
+};
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+};
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Load 16 bytes (N elements of T) and widen to fp32.
+template <typename T>
+__device__ __forceinline__ void load16_f32(const T* __restrict__ p, float* out) {
+  uint4 raw = *reinterpret_cast<const uint4*>(p);
+  const T* e = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+  for (int k = 0; k < Vec16<T>::N; ++k) out[k] = to_f32(e[k]);
+}
+
+// Narrow N fp32 values to T and store 16 bytes.
+template <typename T>
+__device__ __forceinline__ void store16_from_f32(T* __restrict__ p, const float* in) {
+  uint4 raw;
+  T* e = reinterpret_cast<T*>(&raw);
+#pragma unroll
+  for (int k = 0; k < Vec16<T>::N; ++k) e[k] = from_f32<T>(in[k]);
+  *reinterpret_cast<uint4*>(p) = raw;
+}
+
+// cos/sin of pos * theta, the angle formed and evaluated in double precision
+// (positions reach 2^19, where an fp32 angle would be off by ~0.03 rad).
+__device__ __forceinline__ void rope_cos_sin(int pos, double theta, float* c, float* s) {
+  double sd, cd;
+  sincos(static_cast<double>(pos) * theta, &sd, &cd);
+  *c = static_cast<float>(cd);
+  *s = static_cast<float>(sd);
+}
+
+// Rotate the pair (x, y): (x c - y s, x s + y c), in fp32.
+__device__ __forceinline__ void rope_pair(float& x, float& y, float c, float s) {
+  const float xr = x * c - y * s;
+  const float yr = x * s + y * c;
+  x = xr;
+  y = yr;
+}
+
+}  // namespace tpa

@@ -1,0 +1,51 @@
+// Internal interface of the tensor-core kernels (decode and causal prefill).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "tpa_internal.h"
+
+namespace tpa {
+
+// ---- decode (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2})
+bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_v);
+int tensor_decode_token_granule(int r_k);  // split lengths are multiples of this
+int tensor_decode_default_splits(int batch, int max_len, int r_k, int sms);
+
+struct TensorDecodeArgs {
+  CacheView cache;
+  const void* q;
+  const int32_t* q_pos;
+  float scale;
+  int max_len;
+  SplitPlan plan;
+  float* out;
+  float* ws_ml;
+  float* ws_o;
+  RopeTable rope;
+  unsigned int* err;
+};
+cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream);
+
+// ---- causal prefill (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2}, R_Q <= 8)
+bool tensor_prefill_supported(int dtype, int heads, int head_dim, int r_k, int r_v, int r_q);
+size_t tensor_prefill_workspace_bytes(int batch, int n_tokens, int heads, int head_dim);
+
+struct TensorPrefillArgs {
+  CacheView cache;
+  int n_tokens;
+  int r_q;
+  const void* a_q;
+  const void* b_q;
+  const int32_t* q_pos;
+  float scale;
+  float* out;
+  void* workspace;
+  RopeTable rope;
+  unsigned int* err;
+  int sms;
+};
+cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t stream);
+
+}  // namespace tpa

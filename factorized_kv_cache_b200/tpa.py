@@ -1,0 +1,320 @@
+"""Python binding of libtpa (include/tpa.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Tensors are
+PyTorch CUDA tensors used as plain device buffers; every step of the attention
+path runs in the library's CUDA kernels.  There is no fallback: if
+``libtpa.so`` is missing, loading raises ``TpaError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtpa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "tpa.h")
+
+TPA_OK = 0
+TPA_F32, TPA_BF16 = 0, 1
+TPA_KERNEL_AUTO, TPA_KERNEL_SIMT, TPA_KERNEL_TENSOR = 0, 1, 2
+TPA_DEVERR_APPEND_OVERFLOW = 0x1
+TPA_DEVERR_LEN_RANGE = 0x2
+TPA_DEVERR_PREFILL_LEN = 0x4
+
+STATUS_NAMES = {
+    0: "TPA_OK", 1: "TPA_ERR_NULL", 2: "TPA_ERR_SHAPE", 3: "TPA_ERR_UNSUPPORTED",
+    4: "TPA_ERR_CAPACITY", 5: "TPA_ERR_WORKSPACE", 6: "TPA_ERR_ALIGNMENT", 7: "TPA_ERR_CUDA",
+}
+
+_DTYPES = {TPA_F32: torch.float32, TPA_BF16: torch.bfloat16}
+
+
+class TpaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class tpa_cache(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int32),
+        ("capacity", ctypes.c_int32),
+        ("heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("r_k", ctypes.c_int32),
+        ("r_v", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("rope_base", ctypes.c_double),
+        ("a_k", ctypes.c_void_p),
+        ("b_k", ctypes.c_void_p),
+        ("a_v", ctypes.c_void_p),
+        ("b_v", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libtpa.so once and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise TpaError(7, f"{path} is not built; run `python -m factorized_kv_cache_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    I32 = ctypes.c_int32
+    C = ctypes.POINTER(tpa_cache)
+    sig = {
+        "tpa_factor_elements_per_token": (ctypes.c_size_t, [I32, I32, I32, I32]),
+        "tpa_cache_append": (ctypes.c_int, [C, I32, P, P, P, P, P, P]),
+        "tpa_cache_write_slots": (ctypes.c_int, [C, I32, P, P, P, P, P, P, P]),
+        "tpa_decode_default_splits": (I32, [C, I32, I32]),
+        "tpa_decode_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
+        "tpa_decode_attention": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P, ctypes.c_size_t, P]),
+        "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
+        "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
+        "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
+        "tpa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "tpa_last_error_message": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def declared_functions(header: str = HEADER_PATH) -> list[str]:
+    """Names of the functions include/tpa.h declares."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tpa_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status: int):
+    if status != TPA_OK:
+        msg = load_library().tpa_last_error_message().decode()
+        raise TpaError(status, msg)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+@dataclass
+class TpaCache:
+    """A factorized KV cache whose planes are caller-owned CUDA tensors."""
+
+    a_k: torch.Tensor      # [B, cap, r_k, h]
+    b_k: torch.Tensor      # [B, cap, r_k, d_h], rotated at each token's position
+    a_v: torch.Tensor      # [B, cap, r_v, h]
+    b_v: torch.Tensor      # [B, cap, r_v, d_h]
+    seq_lens: torch.Tensor  # [B] int32
+    rope_base: float = 10000.0
+
+    @classmethod
+    def allocate(cls, batch, capacity, heads, head_dim, r_k, r_v, dtype=torch.bfloat16,
+                 rope_base=10000.0, device="cuda", fill=None):
+        kw = dict(dtype=dtype, device=device)
+        mk = (lambda *s: torch.full(s, fill, **kw)) if fill is not None else (lambda *s: torch.empty(s, **kw))
+        return cls(mk(batch, capacity, r_k, heads), mk(batch, capacity, r_k, head_dim),
+                   mk(batch, capacity, r_v, heads), mk(batch, capacity, r_v, head_dim),
+                   torch.zeros(batch, dtype=torch.int32, device=device), rope_base)
+
+    @property
+    def batch(self):
+        return self.a_k.shape[0]
+
+    @property
+    def capacity(self):
+        return self.a_k.shape[1]
+
+    @property
+    def heads(self):
+        return self.a_k.shape[3]
+
+    @property
+    def head_dim(self):
+        return self.b_k.shape[3]
+
+    @property
+    def r_k(self):
+        return self.a_k.shape[2]
+
+    @property
+    def r_v(self):
+        return self.a_v.shape[2]
+
+    @property
+    def dtype(self):
+        return self.a_k.dtype
+
+    def struct(self) -> tpa_cache:
+        B, cap, rk, h = self.a_k.shape
+        d = self.b_k.shape[3]
+        rv = self.a_v.shape[2]
+        dev = self.a_k.device
+        _need(self.a_k, "a_k")
+        _need(self.b_k, "b_k", self.a_k.dtype, (B, cap, rk, d), dev)
+        _need(self.a_v, "a_v", self.a_k.dtype, (B, cap, rv, h), dev)
+        _need(self.b_v, "b_v", self.a_k.dtype, (B, cap, rv, d), dev)
+        _need(self.seq_lens, "seq_lens", torch.int32, (B,), dev)
+        dt = {torch.float32: TPA_F32, torch.bfloat16: TPA_BF16}.get(self.a_k.dtype)
+        if dt is None:
+            raise TypeError(f"cache dtype {self.a_k.dtype} is not float32 or bfloat16")
+        return tpa_cache(B, cap, h, d, rk, rv, dt, 0, float(self.rope_base),
+                         self.a_k.data_ptr(), self.b_k.data_ptr(), self.a_v.data_ptr(), self.b_v.data_ptr(),
+                         self.seq_lens.data_ptr())
+
+
+def tpa_factor_elements_per_token(heads: int, head_dim: int, r_k: int, r_v: int) -> int:
+    return int(load_library().tpa_factor_elements_per_token(heads, head_dim, r_k, r_v))
+
+
+def tpa_status_string(status: int) -> str:
+    return load_library().tpa_status_string(status).decode()
+
+
+def tpa_cache_append(cache: TpaCache, positions, a_k, b_k, a_v, b_v, stream=None):
+    """Append n_new tokens per sequence (inputs [B, n_new, R, h|d_h], B_K unrotated)."""
+    lib = load_library()
+    B = cache.batch
+    n_new = positions.shape[1]
+    dev, dt = cache.a_k.device, cache.dtype
+    _need(positions, "positions", torch.int32, (B, n_new), dev)
+    _need(a_k, "a_k", dt, (B, n_new, cache.r_k, cache.heads), dev)
+    _need(b_k, "b_k", dt, (B, n_new, cache.r_k, cache.head_dim), dev)
+    _need(a_v, "a_v", dt, (B, n_new, cache.r_v, cache.heads), dev)
+    _need(b_v, "b_v", dt, (B, n_new, cache.r_v, cache.head_dim), dev)
+    s = cache.struct()
+    _check(lib.tpa_cache_append(ctypes.byref(s), n_new, _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v),
+                                _ptr(b_v), _stream(stream)))
+
+
+def tpa_cache_write_slots(cache: TpaCache, slots, positions, a_k, b_k, a_v, b_v, stream=None):
+    """Write n_new tokens per sequence at explicit slots [B, n_new]; lengths unchanged."""
+    lib = load_library()
+    B = cache.batch
+    n_new = positions.shape[1]
+    dev, dt = cache.a_k.device, cache.dtype
+    _need(slots, "slots", torch.int32, (B, n_new), dev)
+    _need(positions, "positions", torch.int32, (B, n_new), dev)
+    _need(a_k, "a_k", dt, (B, n_new, cache.r_k, cache.heads), dev)
+    _need(b_k, "b_k", dt, (B, n_new, cache.r_k, cache.head_dim), dev)
+    _need(a_v, "a_v", dt, (B, n_new, cache.r_v, cache.heads), dev)
+    _need(b_v, "b_v", dt, (B, n_new, cache.r_v, cache.head_dim), dev)
+    s = cache.struct()
+    _check(lib.tpa_cache_write_slots(ctypes.byref(s), n_new, _ptr(slots), _ptr(positions), _ptr(a_k), _ptr(b_k),
+                                     _ptr(a_v), _ptr(b_v), _stream(stream)))
+
+
+def tpa_decode_default_splits(cache: TpaCache, max_len: int, kernel: int = TPA_KERNEL_AUTO) -> int:
+    s = cache.struct()
+    return int(load_library().tpa_decode_default_splits(ctypes.byref(s), max_len, kernel))
+
+
+def tpa_decode_workspace_size(cache: TpaCache, max_len: int, num_splits: int = 0,
+                              kernel: int = TPA_KERNEL_AUTO) -> int:
+    s = cache.struct()
+    return int(load_library().tpa_decode_workspace_size(ctypes.byref(s), max_len, num_splits, kernel))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor | None:
+    """A 256-byte aligned device buffer of at least nbytes (None for 0)."""
+    if nbytes == 0:
+        return None
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def tpa_decode_attention(cache: TpaCache, q, q_pos, scale: float | None = None, out=None, max_len: int | None = None,
+                         num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO, workspace_buf=None, stream=None):
+    """Decode attention; returns out [B, h, d_h] float32."""
+    lib = load_library()
+    B, h, d = cache.batch, cache.heads, cache.head_dim
+    dev = cache.a_k.device
+    _need(q, "q", cache.dtype, (B, h, d), dev)
+    _need(q_pos, "q_pos", torch.int32, (B,), dev)
+    if out is None:
+        out = torch.empty(B, h, d, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, (B, h, d), dev)
+    if max_len is None:
+        max_len = cache.capacity
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    need = int(lib.tpa_decode_workspace_size(ctypes.byref(s), max_len, num_splits, kernel))
+    if workspace_buf is None:
+        workspace_buf = workspace(need, dev)
+    nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+    _check(lib.tpa_decode_attention(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out), max_len,
+                                    num_splits, kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+    return out
+
+
+def tpa_prefill_workspace_size(cache: TpaCache, n_tokens: int, r_q: int, kernel: int = TPA_KERNEL_AUTO) -> int:
+    s = cache.struct()
+    return int(load_library().tpa_prefill_workspace_size(ctypes.byref(s), n_tokens, r_q, kernel))
+
+
+def tpa_prefill_attention(cache: TpaCache, a_q, b_q, q_pos, scale: float | None = None, out=None,
+                          kernel: int = TPA_KERNEL_AUTO, workspace_buf=None, stream=None):
+    """Causal prefill of the last T cache slots; a_q [B,T,R_Q,h], b_q [B,T,R_Q,d_h] unrotated."""
+    lib = load_library()
+    B, T, r_q = a_q.shape[0], a_q.shape[1], a_q.shape[2]
+    h, d = cache.heads, cache.head_dim
+    dev = cache.a_k.device
+    _need(a_q, "a_q", cache.dtype, (B, T, r_q, h), dev)
+    _need(b_q, "b_q", cache.dtype, (B, T, r_q, d), dev)
+    _need(q_pos, "q_pos", torch.int32, (B, T), dev)
+    if B != cache.batch:
+        raise ValueError("a_q batch differs from the cache batch")
+    if out is None:
+        out = torch.empty(B, T, h, d, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, (B, T, h, d), dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    need = int(lib.tpa_prefill_workspace_size(ctypes.byref(s), T, r_q, kernel))
+    if workspace_buf is None:
+        workspace_buf = workspace(need, dev)
+    nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+    _check(lib.tpa_prefill_attention(ctypes.byref(s), T, r_q, _ptr(a_q), _ptr(b_q), _ptr(q_pos), float(scale),
+                                     _ptr(out), kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+    return out
+
+
+def tpa_read_device_error(stream=None) -> int:
+    """Synchronise the stream, return and clear the device error word."""
+    lib = load_library()
+    v = ctypes.c_uint32(0)
+    _check(lib.tpa_read_device_error(ctypes.byref(v), _stream(stream)))
+    return int(v.value)

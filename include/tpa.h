@@ -1,0 +1,209 @@
+/*
+ * tpa.h - C ABI of libtpa: softmax attention evaluated directly over a
+ * Tensor Product Attention (TPA) factorized KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Tensor Product Attention Is All You Need" (NeurIPS 2025 notes),
+ *   - section 关键设计 / 张量积分解 (tensor product decomposition):
+ *       K_t = (1/R_K) A_K(x_t)^T B_K(x_t),  V_t = (1/R_V) A_V(x_t)^T B_V(x_t),
+ *       A in R^{R x h} (head factor), B in R^{R x d_h} (feature factor);
+ *       the cache holds A_K, B_K, A_V, B_V: (R_K+R_V)(h+d_h) numbers/token.
+ *   - section 解决思路: Q_t = (1/R_Q) A_Q(x_t)^T B_Q(x_t).
+ *   - section RoPE 兼容性 (Theorem 3.1): RoPE rotates the B factors only.
+ *   - section FlashTPA: attention runs on the factors; dense K/V are never built.
+ *
+ * Readings where the page is silent (the CPU oracle uses the same ones):
+ *   RoPE pairs are adjacent elements (2j, 2j+1), angle = pos * theta_j with
+ *   theta_j = rope_base^(-2j/d_h), (x, y) -> (x cos a - y sin a, x sin a + y cos a);
+ *   angles are formed and passed to sin/cos in double precision, the rotation
+ *   itself runs in fp32 and is rounded once to the storage dtype.
+ *   The softmax scale is given by the caller (1/sqrt(d_h) in the workloads).
+ *
+ * Conventions for every call:
+ *   - The caller owns all memory.  Pointers marked "device" point to device
+ *     memory of the current CUDA device; the library allocates nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Host-side argument checks run first; a call that
+ *     returns anything but TPA_OK has launched nothing.
+ *   - Conditions only the device can see (a length above max_len or the
+ *     capacity, an append past the capacity) are recorded in a sticky device
+ *     error word read by tpa_read_device_error(); the kernel skips the
+ *     offending work and never traps.
+ *   - Supported: dtype TPA_F32 or TPA_BF16; head_dim in {16, 32, 64, 128};
+ *     1 <= heads <= 32 with heads * element size a multiple of 16 bytes;
+ *     1 <= r_k, r_v <= 4; 1 <= r_q <= 8.  Anything else: TPA_ERR_UNSUPPORTED.
+ */
+#ifndef TPA_H_
+#define TPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tpa_status {
+  TPA_OK = 0,
+  TPA_ERR_NULL = 1,        /* a required pointer is NULL */
+  TPA_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  TPA_ERR_UNSUPPORTED = 3, /* outside the supported set listed above */
+  TPA_ERR_CAPACITY = 4,    /* a host-visible length exceeds the capacity */
+  TPA_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than required */
+  TPA_ERR_ALIGNMENT = 6,   /* a pointer is not 16-byte aligned */
+  TPA_ERR_CUDA = 7         /* a CUDA runtime call failed (see tpa_last_error_message) */
+} tpa_status;
+
+typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
+
+/* Kernel choice for decode and prefill.  AUTO picks the fastest kernel that
+ * supports the shape: the tensor-core kernels for bf16 at head_dim 128,
+ * heads 32, r_k == r_v <= 2; the CUDA-core kernels otherwise. */
+typedef enum tpa_kernel {
+  TPA_KERNEL_AUTO = 0,
+  TPA_KERNEL_SIMT = 1,   /* CUDA-core fp32 FMA path (every supported shape) */
+  TPA_KERNEL_TENSOR = 2  /* tensor-core path (bf16 only; TPA_ERR_UNSUPPORTED otherwise) */
+} tpa_kernel;
+
+/* Device error word bits (tpa_read_device_error). */
+#define TPA_DEVERR_APPEND_OVERFLOW 0x1u /* an append reached a slot >= capacity */
+#define TPA_DEVERR_LEN_RANGE 0x2u       /* seq_lens[b] < 0, > capacity or > max_len */
+#define TPA_DEVERR_PREFILL_LEN 0x4u     /* prefill n_tokens > seq_lens[b] */
+
+/*
+ * A factorized KV cache of `batch` sequences, `capacity` token slots each.
+ * Planes are token-major per sequence, row-major, contiguous, 16-byte aligned:
+ *   a_k [batch][capacity][r_k][heads]     head factor of the keys
+ *   b_k [batch][capacity][r_k][head_dim]  feature factor of the keys, stored
+ *                                         rotated at the token's position
+ *   a_v [batch][capacity][r_v][heads]     head factor of the values
+ *   b_v [batch][capacity][r_v][head_dim]  feature factor of the values
+ *   seq_lens [batch] int32                tokens held by each sequence
+ * All five pointers are device pointers owned by the caller.  Slots at or
+ * past seq_lens[b] may hold anything (NaN included); no kernel reads them
+ * into a result.
+ */
+typedef struct tpa_cache {
+  int32_t batch;
+  int32_t capacity;
+  int32_t heads;    /* h */
+  int32_t head_dim; /* d_h */
+  int32_t r_k;
+  int32_t r_v;
+  int32_t dtype;    /* tpa_dtype of the four planes */
+  int32_t reserved; /* must be 0 */
+  double rope_base; /* RoPE base (10000 in the workloads); > 1 */
+  void* a_k;
+  void* b_k;
+  void* a_v;
+  void* b_v;
+  int32_t* seq_lens;
+} tpa_cache;
+
+/* (r_k + r_v) * (heads + head_dim): numbers stored per cached token
+ * (section 关键设计: 320 at h=32, d_h=128, R_K=R_V=1, against 2*h*d_h = 8192).
+ * Returns 0 for non-positive arguments. */
+size_t tpa_factor_elements_per_token(int32_t heads, int32_t head_dim, int32_t r_k, int32_t r_v);
+
+/*
+ * Append n_new tokens to every sequence (section 关键设计 for the factors,
+ * Theorem 3.1 for RoPE on B_K only).
+ *   positions [batch][n_new] int32, device: RoPE position of each new token (>= 0)
+ *   a_k [batch][n_new][r_k][heads], b_k [batch][n_new][r_k][head_dim] (NOT rotated),
+ *   a_v [batch][n_new][r_v][heads], b_v [batch][n_new][r_v][head_dim]: device,
+ *   in the cache dtype, contiguous, 16-byte aligned.
+ * Token j of sequence b goes to slot seq_lens[b] + j: A_K, A_V, B_V are copied
+ * and B_K is rotated at positions[b][j]; then seq_lens[b] += n_new on the
+ * device.  A token whose slot would be >= capacity is not written and sets
+ * TPA_DEVERR_APPEND_OVERFLOW (seq_lens[b] is then left unchanged).
+ * n_new == 0 is a no-op.  Errors: NULL, SHAPE (n_new < 0), UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+tpa_status tpa_cache_append(const tpa_cache* cache, int32_t n_new, const int32_t* positions,
+                            const void* a_k, const void* b_k, const void* a_v, const void* b_v,
+                            void* stream);
+
+/*
+ * The same factor write as tpa_cache_append (copy A_K, A_V, B_V; rotate B_K at
+ * positions[b][j]) at caller-chosen slots: token j of sequence b goes to slot
+ * slots[b][j] (int32, device, [batch][n_new]).  seq_lens is neither read nor
+ * changed, so a fixed-length cache (a ring buffer, or a benchmark that
+ * rewrites its newest token every step) keeps its lengths.  A slot outside
+ * [0, capacity) is skipped and sets TPA_DEVERR_APPEND_OVERFLOW.  Two tokens
+ * with the same slot in one call race (one of them wins).
+ * Errors: as tpa_cache_append.
+ */
+tpa_status tpa_cache_write_slots(const tpa_cache* cache, int32_t n_new, const int32_t* slots,
+                                 const int32_t* positions, const void* a_k, const void* b_k,
+                                 const void* a_v, const void* b_v, void* stream);
+
+/* Splits of the token range that decode uses when num_splits == 0. */
+int32_t tpa_decode_default_splits(const tpa_cache* cache, int32_t max_len, int32_t kernel);
+
+/* Workspace bytes tpa_decode_attention needs for this split count
+ * (num_splits == 0: the default).  0 when one split suffices. */
+size_t tpa_decode_workspace_size(const tpa_cache* cache, int32_t max_len, int32_t num_splits,
+                                 int32_t kernel);
+
+/*
+ * Decode: one query token per sequence attends every cached token
+ * 0 .. seq_lens[b]-1 (the query's own token is attended only if it was
+ * appended first).
+ *   q [batch][heads][head_dim], device, cache dtype, NOT rotated;
+ *   q_pos [batch] int32, device: position of the query (RoPE);
+ *   scale: softmax scale (1/sqrt(head_dim) in the workloads);
+ *   out [batch][heads][head_dim] float32, device:
+ *     out[b][i] = sum_s softmax_s(scale * q~_i . K_s[i]) V_s[i],
+ *     q~ = RoPE(q, q_pos), K_s, V_s the factor products of slot s;
+ *     0 for an empty sequence.
+ *   max_len: host upper bound on every seq_lens[b] (sizes the grid);
+ *   num_splits: 0 = default; the token range is cut into this many splits
+ *     whose partial softmax states are merged by log-sum-exp;
+ *   kernel: tpa_kernel;
+ *   workspace: device, >= tpa_decode_workspace_size(...) bytes, 256-byte
+ *     aligned; may be NULL when that size is 0.  Its contents on entry do not
+ *     matter; calls that share one workspace must be ordered on the GPU.
+ * Errors: NULL, SHAPE (max_len < 0), CAPACITY (max_len > capacity),
+ * UNSUPPORTED, WORKSPACE, ALIGNMENT, CUDA.
+ */
+tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int32_t* q_pos,
+                                float scale, float* out, int32_t max_len, int32_t num_splits,
+                                int32_t kernel, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* Workspace bytes tpa_prefill_attention needs. */
+size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q,
+                                  int32_t kernel);
+
+/*
+ * Causal prefill of a chunk of n_tokens queries per sequence whose K/V
+ * factors were appended first: query t of sequence b sits at slot
+ * P + t, P = seq_lens[b] - n_tokens, and attends slots 0 .. P + t.
+ *   a_q [batch][n_tokens][r_q][heads], b_q [batch][n_tokens][r_q][head_dim]
+ *     (B_Q NOT rotated): device, cache dtype;
+ *   q_pos [batch][n_tokens] int32, device: query positions (RoPE on B_Q);
+ *   query t, head i: q = (1/r_q) sum_j A_Q[t][j][i] RoPE(B_Q[t][j], q_pos[t]);
+ *   out [batch][n_tokens][heads][head_dim] float32, device.
+ *   workspace: device, >= tpa_prefill_workspace_size(...) bytes, 256-byte aligned.
+ * Errors: NULL, SHAPE (n_tokens < 0 or > capacity), UNSUPPORTED, WORKSPACE,
+ * ALIGNMENT, CUDA.  n_tokens > seq_lens[b] sets TPA_DEVERR_PREFILL_LEN and
+ * leaves out[b] untouched.
+ */
+tpa_status tpa_prefill_attention(const tpa_cache* cache, int32_t n_tokens, int32_t r_q,
+                                 const void* a_q, const void* b_q, const int32_t* q_pos,
+                                 float scale, float* out, int32_t kernel, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, copy the current device's error word to *code_out and
+ * clear it.  Errors: NULL, CUDA. */
+tpa_status tpa_read_device_error(uint32_t* code_out, void* stream);
+
+/* Static description of a status code. */
+const char* tpa_status_string(tpa_status status);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+const char* tpa_last_error_message(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* TPA_H_ */

@@ -1,0 +1,131 @@
+"""GPU parity of tpa_decode_attention against the float64 oracle.
+
+Two levels: (i) the oracle reads the cache the GPU wrote (so storage rounding
+of the rotated B_K is not charged to attention); (ii) end to end, the oracle
+starts from the unrotated factors and applies its own RoPE.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.tpa_oracle as O
+from factorized_kv_cache_b200 import synthetic as S
+from factorized_kv_cache_b200 import tpa as T
+from tests.gpu_cases import DEV, build_decode_cache, readback
+from tests.parity_util import TOL, assert_rows_close, default_scale, f64, oracle_decode_rows
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [T.TPA_KERNEL_SIMT, T.TPA_KERNEL_AUTO]
+
+
+def _check(w, cache, x, q, q_pos, out, batches=None, heads=None, end_to_end=True):
+    d = w.head_dim
+    scale = default_scale(d)
+    lengths = x["lengths"].numpy()
+    batches = list(range(cache.batch)) if batches is None else list(batches)
+    cpu = readback(cache, batches)
+    qn = f64(q)[batches]
+    ref = oracle_decode_rows(cpu, qn, x["q_pos"].numpy()[batches], lengths[batches], scale, w.rope_base,
+                             heads=heads)
+    got = f64(out)[batches]
+    if heads is not None:
+        got = got[:, list(heads)]
+    tol = TOL[cache.dtype]
+    worst = assert_rows_close(got, ref, tol, f"{w.name} cache-level")
+    if end_to_end:
+        for n, b in enumerate(batches[:2]):
+            L = int(lengths[b])
+            sel = slice(None) if heads is None else list(heads)
+            ak = f64(x["a_k"][b, :L])[:, :, sel]
+            av = f64(x["a_v"][b, :L])[:, :, sel]
+            r = O.decode_attention_from_unrotated(ak, f64(x["b_k"][b, :L]), av, f64(x["b_v"][b, :L]),
+                                                  np.arange(L), f64(x["q"][b])[sel], float(x["q_pos"][b]),
+                                                  scale, w.rope_base)
+            assert_rows_close(got[n], r, tol, f"{w.name} end-to-end b={b}")
+    return worst
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_tiny_f32_workload(kernel):
+    w = S.WORKLOADS["decode_tiny_f32"]
+    cache, x, q, q_pos = build_decode_cache(w)
+    for splits in (0, 1, 2, 4):
+        out = T.tpa_decode_attention(cache, q, q_pos, max_len=64, num_splits=splits, kernel=kernel)
+        _check(w, cache, x, q, q_pos, out)
+    assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_b8_l8k_workload_full_size(kernel):
+    """The full bf16 decode workload (B=8, L=8192); oracle on 6 heads of every sequence."""
+    w = S.WORKLOADS["decode_b8_l8k"]
+    cache, x, q, q_pos = build_decode_cache(w)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out, heads=[0, 5, 13, 21, 30, 31])
+    assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("lengths", [[0, 1, 2, 63], [64, 65, 127, 129], [1000, 777, 4095, 3]])
+@pytest.mark.parametrize("splits", [1, 3, 0])
+def test_ragged_lengths_and_splits(kernel, lengths, splits):
+    w = S.WORKLOADS["decode_b8_l8k"]
+    cache, x, q, q_pos = build_decode_cache(w, batch=4, length=max(lengths) + 5, lengths=lengths)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=max(lengths), num_splits=splits, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out, end_to_end=False)
+    empty = [b for b, L in enumerate(lengths) if L == 0]
+    for b in empty:
+        assert torch.count_nonzero(out[b]) == 0
+    assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_rank2_varlen_small(kernel):
+    w = S.WORKLOADS["decode_b32_var32k"]
+    cache, x, q, q_pos = build_decode_cache(w, batch=5, length=3000, min_length=1)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=3000, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out)
+
+
+@pytest.mark.parametrize("h,d,rk,rv,dt", [
+    (8, 64, 1, 2, "bf16"), (16, 32, 3, 1, "bf16"), (32, 16, 4, 4, "bf16"),
+    (4, 16, 2, 1, "f32"), (12, 128, 1, 1, "f32"), (32, 64, 2, 2, "f32"),
+])
+def test_other_shapes_simt(h, d, rk, rv, dt):
+    w = S.DecodeWorkload("shape", 3, h, d, rk, rv, 700, dt, seed=h + d + rk + rv, min_length=1)
+    cache, x, q, q_pos = build_decode_cache(w)
+    for splits in (1, 5):
+        out = T.tpa_decode_attention(cache, q, q_pos, max_len=700, num_splits=splits)
+        _check(w, cache, x, q, q_pos, out)
+
+
+def test_length_above_max_len_is_reported():
+    w = S.WORKLOADS["decode_b8_l8k"]
+    cache, x, q, q_pos = build_decode_cache(w, batch=2, length=256)
+    T.tpa_decode_attention(cache, q, q_pos, max_len=100, kernel=T.TPA_KERNEL_SIMT)
+    assert T.tpa_read_device_error() & T.TPA_DEVERR_LEN_RANGE
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_b32_var32k_workload_full_size(kernel):
+    """The full R=2 variable-length workload; oracle on 4 sequences x 4 heads."""
+    w = S.WORKLOADS["decode_b32_var32k"]
+    cache, x, q, q_pos = build_decode_cache(w, nan_tail=False)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
+    L = x["lengths"].numpy()
+    picks = [int(np.argmin(L)), int(np.argmax(L)), 7, 19]
+    _check(w, cache, x, q, q_pos, out, batches=picks, heads=[0, 11, 22, 31], end_to_end=False)
+    assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_long_512k_workload_full_size(kernel):
+    """The long-context workload (B=1, L=524288); oracle on 3 heads."""
+    w = S.WORKLOADS["decode_long_512k"]
+    cache, x, q, q_pos = build_decode_cache(w, nan_tail=False)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out, heads=[0, 17, 31], end_to_end=False)
+    assert T.tpa_read_device_error() == 0

@@ -1,0 +1,103 @@
+"""GPU parity of tpa_prefill_attention (causal, R_Q-factorized queries)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.tpa_oracle as O
+from factorized_kv_cache_b200 import synthetic as S
+from factorized_kv_cache_b200 import tpa as T
+from tests.gpu_cases import DEV, TORCH_DTYPE
+from tests.parity_util import TOL, assert_rows_close, default_scale, f64
+
+pytestmark = pytest.mark.gpu
+
+KERNELS = [T.TPA_KERNEL_SIMT, T.TPA_KERNEL_AUTO]
+
+
+def _prefill_case(w, batch, tokens, prior=0, nan_fill=True):
+    """Cache holding `prior` earlier tokens, then the chunk's own factors appended."""
+    x = S.prefill_inputs(w, batch=batch, tokens=prior + tokens)
+    dt = TORCH_DTYPE[w.dtype]
+    cap = prior + tokens + 9
+    cache = T.TpaCache.allocate(batch, cap, w.heads, w.head_dim, w.r_k, w.r_v, dtype=dt, rope_base=w.rope_base,
+                                fill=float("nan") if nan_fill else 0.0)
+    pos = x["positions"].to(DEV)
+    if prior:
+        T.tpa_cache_append(cache, pos[:, :prior].contiguous(), *(x[k][:, :prior].contiguous().to(DEV)
+                                                                 for k in ("a_k", "b_k", "a_v", "b_v")))
+    T.tpa_cache_append(cache, pos[:, prior:].contiguous(), *(x[k][:, prior:].contiguous().to(DEV)
+                                                             for k in ("a_k", "b_k", "a_v", "b_v")))
+    a_q = x["a_q"][:, prior:].contiguous().to(DEV)
+    b_q = x["b_q"][:, prior:].contiguous().to(DEV)
+    q_pos = pos[:, prior:].contiguous()
+    return cache, x, a_q, b_q, q_pos
+
+
+def _oracle(w, cache, x, prior, tokens, b, rows=None, heads=None, end_to_end=False):
+    L = prior + tokens
+    scale = default_scale(w.head_dim)
+    sel = slice(None) if heads is None else list(heads)
+    if end_to_end:
+        bk = O.append_rope(f64(x["b_k"][b, :L]), np.arange(L), w.rope_base)
+    else:
+        bk = f64(cache.b_k[b, :L])
+    ak = f64(cache.a_k[b, :L])[:, :, sel]
+    av = f64(cache.a_v[b, :L])[:, :, sel]
+    aq = f64(x["a_q"][b, prior:L])[:, :, sel]
+    return O.prefill_attention(ak, bk, av, f64(cache.b_v[b, :L]), aq, f64(x["b_q"][b, prior:L]),
+                               np.arange(prior, L), scale, w.rope_base, rows=rows)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("tokens,prior", [(1, 0), (200, 0), (130, 37), (257, 0)])
+def test_prefill_small(kernel, tokens, prior):
+    w = S.WORKLOADS["prefill_b4_t4k"]
+    cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, tokens, prior)
+    out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos, kernel=kernel)
+    assert T.tpa_read_device_error() == 0
+    got = f64(out)
+    for b in range(2):
+        ref = _oracle(w, cache, x, prior, tokens, b)
+        assert_rows_close(got[b], ref, TOL[cache.dtype], f"prefill b={b}")
+    ref = _oracle(w, cache, x, prior, tokens, 0, rows=[0, tokens - 1], end_to_end=True)
+    assert_rows_close(got[0][[0, tokens - 1]], ref, TOL[cache.dtype], "prefill end-to-end")
+
+
+@pytest.mark.parametrize("rq,rk,rv,h,d,dt", [
+    (1, 1, 1, 8, 64, "bf16"), (3, 2, 1, 16, 32, "bf16"), (8, 4, 4, 32, 128, "bf16"),
+    (2, 1, 1, 4, 16, "f32"), (6, 2, 2, 32, 128, "f32"),
+])
+def test_prefill_other_shapes(rq, rk, rv, h, d, dt):
+    w = S.PrefillWorkload("shape", 2, 70, h, d, rq, rk, rv, 256, dt, seed=rq + rk + h)
+    cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, 70, prior=11)
+    out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos)
+    got = f64(out)
+    for b in range(2):
+        assert_rows_close(got[b], _oracle(w, cache, x, 11, 70, b), TOL[cache.dtype], f"shape b={b}")
+
+
+def test_prefill_longer_than_cache_is_reported():
+    w = S.WORKLOADS["prefill_b4_t4k"]
+    cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, 50)
+    cache.seq_lens[1] = 20                         # sequence 1 holds fewer tokens than the chunk
+    out = torch.full((2, 50, 32, 128), 7.0, device=DEV)
+    T.tpa_prefill_attention(cache, a_q, b_q, q_pos, out=out, kernel=T.TPA_KERNEL_SIMT)
+    assert T.tpa_read_device_error() & T.TPA_DEVERR_PREFILL_LEN
+    assert bool((out[1] == 7.0).all())
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("kernel", [T.TPA_KERNEL_AUTO])
+def test_prefill_workload_full_size(kernel):
+    """The full causal prefill (B=4, T=4096); oracle on sampled rows x heads."""
+    w = S.WORKLOADS["prefill_b4_t4k"]
+    cache, x, a_q, b_q, q_pos = _prefill_case(w, w.batch, w.tokens, nan_fill=False)
+    out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos, kernel=kernel)
+    assert T.tpa_read_device_error() == 0
+    got = f64(out)
+    g = np.random.default_rng(0)
+    for b in range(w.batch):
+        rows = sorted(set([0, 1, 127, 128, w.tokens - 1] + g.integers(0, w.tokens, 12).tolist()))
+        heads = [0, 9, 31]
+        ref = _oracle(w, cache, x, 0, w.tokens, b, rows=rows, heads=heads)
+        assert_rows_close(got[b][rows][:, heads], ref, TOL[cache.dtype], f"prefill full b={b}")
