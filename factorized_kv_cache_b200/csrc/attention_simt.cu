@@ -36,7 +36,7 @@ __device__ __forceinline__ void load_slice(const T* __restrict__ p, float* out) 
 }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kSimtThreads) simt_attention_kernel(const __grid_constant__ SimtArgs a) {
+__global__ void __launch_bounds__(kSimtThreads, 2) simt_attention_kernel(const __grid_constant__ SimtArgs a) {
   constexpr int SL = D / kSlices;
   const int h = a.cache.heads;
   const int rk = a.cache.r_k, rv = a.cache.r_v;
@@ -103,46 +103,85 @@ __global__ void __launch_bounds__(kSimtThreads) simt_attention_kernel(const __gr
 #pragma unroll
   for (int k = 0; k < SL; ++k) acc[k] = 0.0f;
 
-  for (int base = s_begin; base < s_end; base += G) {
-    const int s = base + g;
-    const bool valid = lane_on && s < s_end;
-    float z = 0.0f;
+  // kU tokens per group per iteration; every load of the iteration is issued
+  // before the arithmetic that consumes it, so kU * (R_K + R_V) row loads are
+  // in flight per thread instead of one.
+  constexpr int kU = 4;
+  for (int base = s_begin; base < s_end; base += G * kU) {
+    float z[kU];
+    bool valid[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int s = base + u * G + g;
+      valid[u] = lane_on && s < s_end;
+      z[u] = 0.0f;
+    }
     for (int r = 0; r < rk; ++r) {
-      float part = 0.0f;
-      float av = 0.0f;
-      if (valid) {
-        float kb[SL];
-        load_slice<T, SL>(BK + (static_cast<size_t>(s) * rk + r) * D + c * SL, kb);
+      float kb[kU][SL];
+      float av[kU];
 #pragma unroll
-        for (int k = 0; k < SL; ++k) part = fmaf(qv[k], kb[k], part);
-        av = to_f32(AK[(static_cast<size_t>(s) * rk + r) * h + i]);
+      for (int u = 0; u < kU; ++u) {
+        const int s = base + u * G + g;
+        av[u] = 0.0f;
+        if (valid[u]) {
+          load_slice<T, SL>(BK + (static_cast<size_t>(s) * rk + r) * D + c * SL, kb[u]);
+          av[u] = to_f32(AK[(static_cast<size_t>(s) * rk + r) * h + i]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < SL; ++k) kb[u][k] = 0.0f;
+        }
       }
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      part += __shfl_xor_sync(0xffffffffu, part, 4);
-      z = fmaf(av, part, z);
-    }
-    if (valid) {
-      z *= zs;
-      const float m_new = fmaxf(m, z);
-      const float corr = exp2f(m - m_new);
-      const float p = exp2f(z - m_new);
-      l = fmaf(l, corr, p);
-      float vv[SL];
 #pragma unroll
-      for (int k = 0; k < SL; ++k) vv[k] = 0.0f;
-      for (int r = 0; r < rv; ++r) {
-        float vb[SL];
-        load_slice<T, SL>(BV + (static_cast<size_t>(s) * rv + r) * D + c * SL, vb);
-        const float w = to_f32(AV[(static_cast<size_t>(s) * rv + r) * h + i]);
+      for (int u = 0; u < kU; ++u) {
+        float part = 0.0f;
 #pragma unroll
-        for (int k = 0; k < SL; ++k) vv[k] = fmaf(w, vb[k], vv[k]);
+        for (int k = 0; k < SL; ++k) part = fmaf(qv[k], kb[u][k], part);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        z[u] = fmaf(av[u], part, z[u]);
       }
-      const float pw = p * inv_rv;
-#pragma unroll
-      for (int k = 0; k < SL; ++k) acc[k] = fmaf(acc[k], corr, pw * vv[k]);
-      m = m_new;
     }
+    float m_new = m;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      z[u] *= zs;
+      if (valid[u]) m_new = fmaxf(m_new, z[u]);
+    }
+    if (m_new == -INFINITY) continue;  // no valid token for this thread in this iteration
+    const float corr = exp2f(m - m_new);
+    float p[kU];
+    float psum = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      p[u] = valid[u] ? exp2f(z[u] - m_new) : 0.0f;
+      psum += p[u];
+    }
+    l = fmaf(l, corr, psum);
+#pragma unroll
+    for (int k = 0; k < SL; ++k) acc[k] *= corr;
+    for (int r = 0; r < rv; ++r) {
+      float vb[kU][SL];
+      float w[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int s = base + u * G + g;
+        w[u] = 0.0f;
+        if (valid[u]) {
+          load_slice<T, SL>(BV + (static_cast<size_t>(s) * rv + r) * D + c * SL, vb[u]);
+          w[u] = p[u] * inv_rv * to_f32(AV[(static_cast<size_t>(s) * rv + r) * h + i]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < SL; ++k) vb[u][k] = 0.0f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+#pragma unroll
+        for (int k = 0; k < SL; ++k) acc[k] = fmaf(w[u], vb[u][k], acc[k]);
+      }
+    }
+    m = m_new;
   }
 
   // merge the token groups of this CTA
@@ -206,27 +245,67 @@ cudaError_t launch_simt_t(const SimtArgs& a, cudaStream_t stream) {
 }
 
 // Log-sum-exp merge: M = max_j m_j, L = sum_j l_j 2^(m_j-M),
-// o = sum_j o_j 2^(m_j-M) / L (m in base-2 units).  One CTA per (query, head).
-__global__ void merge_kernel(const __grid_constant__ MergeArgs a) {
+// o = sum_j o_j 2^(m_j-M) / L (m in base-2 units).  One CTA per (query, head);
+// the split maxima and sums are reduced across the CTA, the features are
+// accumulated with eight independent loads in flight per thread.
+__device__ __forceinline__ float block_reduce(float v, bool is_max, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, w) : v + w;
+  }
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) s_red[warp] = v;
+  __syncthreads();
+  v = s_red[0];
+  for (int k = 1; k < nw; ++k) v = is_max ? fmaxf(v, s_red[k]) : v + s_red[k];
+  return v;
+}
+
+__global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ MergeArgs a) {
   // with programmatic dependent launch, wait here for the split kernel's writes
   if (a.use_pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float s_red[4];
   const int q = blockIdx.x, i = blockIdx.y;
   const size_t row = static_cast<size_t>(q) * a.splits;
+  const float* ml = a.ws_ml + 2 * (row * a.heads + i);  // split j at ml[2 * j * heads]
+  const size_t mstride = 2 * static_cast<size_t>(a.heads);
   float M = -INFINITY;
-  for (int j = 0; j < a.splits; ++j) M = fmaxf(M, a.ws_ml[2 * ((row + j) * a.heads + i)]);
+  for (int j = threadIdx.x; j < a.splits; j += blockDim.x) M = fmaxf(M, ml[j * mstride]);
+  M = block_reduce(M, true, s_red);
+  float L = 0.0f;
+  if (M != -INFINITY) {
+    for (int j = threadIdx.x; j < a.splits; j += blockDim.x) {
+      const float mj = ml[j * mstride];
+      if (mj != -INFINITY) L = fmaf(ml[j * mstride + 1], exp2f(mj - M), L);
+    }
+  }
+  L = block_reduce(L, false, s_red);
+  const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+  const size_t ostride = static_cast<size_t>(a.heads) * a.head_dim;
+  const float* o0 = a.ws_o + (row * a.heads + i) * a.head_dim;
   for (int k = threadIdx.x; k < a.head_dim; k += blockDim.x) {
-    float L = 0.0f, O = 0.0f;
+    float O = 0.0f;
     if (M != -INFINITY) {
-      for (int j = 0; j < a.splits; ++j) {
-        const size_t part = (row + j) * a.heads + i;
-        const float mj = a.ws_ml[2 * part];
-        if (mj == -INFINITY) continue;
-        const float w = exp2f(mj - M);
-        L = fmaf(a.ws_ml[2 * part + 1], w, L);
-        O = fmaf(a.ws_o[part * a.head_dim + k], w, O);
+      int j = 0;
+      for (; j + 8 <= a.splits; j += 8) {
+        float v[8], wgt[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          v[u] = o0[(j + u) * ostride + k];
+          const float mj = ml[(j + u) * mstride];
+          wgt[u] = mj == -INFINITY ? 0.0f : exp2f(mj - M);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) O = fmaf(v[u], wgt[u], O);
+      }
+      for (; j < a.splits; ++j) {
+        const float mj = ml[j * mstride];
+        if (mj != -INFINITY) O = fmaf(o0[j * ostride + k], exp2f(mj - M), O);
       }
     }
-    a.out[(static_cast<size_t>(q) * a.heads + i) * a.head_dim + k] = L > 0.0f ? O / L : 0.0f;
+    a.out[(static_cast<size_t>(q) * a.heads + i) * a.head_dim + k] = O * inv;
   }
 }
 
@@ -270,7 +349,7 @@ cudaError_t launch_simt_attention(const SimtArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream) {
   dim3 grid(a.n_queries, a.heads);
-  const int threads = a.head_dim < 32 ? 32 : a.head_dim;
+  const int threads = 128;
   if (!a.use_pdl) {
     merge_kernel<<<grid, threads, 0, stream>>>(a);
     return cudaGetLastError();

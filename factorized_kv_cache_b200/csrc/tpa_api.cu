@@ -126,11 +126,11 @@ SplitPlan plan_splits(const tpa_cache* c, int max_len, int num_splits, int kerne
     if (tensor) {
       splits = tensor_decode_default_splits(c->batch, max_len, c->r_k, sms);
     } else {
-      // about eight 256-thread CTAs per SM, splits no shorter than 256 tokens
+      // about eight 256-thread CTAs per SM, splits no shorter than 64 tokens
       const int target = sms * 8;
       splits = ceil_div(target, c->batch);
       splits = splits < 1 ? 1 : splits;
-      const int max_splits = ceil_div(max_len, 256);
+      const int max_splits = ceil_div(max_len, 64);
       if (splits > max_splits) splits = max_splits;
     }
   }
