@@ -166,6 +166,15 @@ DecodeWs carve_decode_ws(void* base, int n_queries, int heads, int head_dim, int
 
 }  // namespace
 
+void set_last_error_message(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+}
+
 void make_rope_table(double base, int head_dim, RopeTable* t) {
   memset(t, 0, sizeof(*t));
   for (int j = 0; j < head_dim / 2 && j < kMaxPairs; ++j)

@@ -18,6 +18,9 @@ struct RopeTable {
 
 void make_rope_table(double base, int head_dim, RopeTable* t);
 
+// Sets the text tpa_last_error_message() returns on this host thread.
+void set_last_error_message(const char* fmt, ...) __attribute__((format(printf, 1, 2)));
+
 struct CacheView {
   int batch, capacity, heads, head_dim, r_k, r_v, dtype;
   const void* a_k;

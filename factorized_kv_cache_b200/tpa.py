@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_decode_default_splits": (I32, [C, I32, I32]),
         "tpa_decode_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_decode_attention": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P, ctypes.c_size_t, P]),
+        "tpa_decode_attention_noalloc": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
@@ -277,6 +278,29 @@ def tpa_decode_attention(cache: TpaCache, q, q_pos, scale: float | None = None, 
     nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
     _check(lib.tpa_decode_attention(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out), max_len,
                                     num_splits, kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+    return out
+
+
+def tpa_decode_attention_noalloc(cache: TpaCache, q, q_pos, out, scale: float | None = None,
+                                 max_len: int | None = None, num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO,
+                                 stream=None):
+    """Decode attention that allocates nothing: the split partials go to the
+    library's built-in 16 MiB scratch array instead of a workspace.  The
+    caller passes every buffer, ``out`` included, so this call makes no
+    allocation on the Python side either."""
+    lib = load_library()
+    B, h, d = cache.batch, cache.heads, cache.head_dim
+    dev = cache.a_k.device
+    _need(q, "q", cache.dtype, (B, h, d), dev)
+    _need(q_pos, "q_pos", torch.int32, (B,), dev)
+    _need(out, "out", torch.float32, (B, h, d), dev)
+    if max_len is None:
+        max_len = cache.capacity
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    _check(lib.tpa_decode_attention_noalloc(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out),
+                                            max_len, num_splits, kernel, _stream(stream)))
     return out
 
 

@@ -169,6 +169,29 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
                                 int32_t kernel, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
+/*
+ * tpa_decode_attention for callers that cannot allocate device memory (no
+ * counterpart on the page; this is a deployment convenience).  Same
+ * arguments and result as tpa_decode_attention minus the workspace: the
+ * split partials live in a 16 MiB scratch array compiled into libtpa, held
+ * on every GPU that loads the library until the process exits.  Nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - num_splits == 0: the default split count, lowered if needed until the
+ *     partials fit in the 16 MiB array (one split needs no scratch at all).
+ *   - num_splits > 0 whose partials exceed 16 MiB: TPA_ERR_WORKSPACE, nothing
+ *     launched, and tpa_last_error_message() says how much was needed.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents (no call depends on them); calls that overlap on the
+ *     GPU race on the array: order them on one stream or with events.
+ * Errors: those of tpa_decode_attention, plus WORKSPACE as above.
+ */
+tpa_status tpa_decode_attention_noalloc(const tpa_cache* cache, const void* q, const int32_t* q_pos,
+                                        float scale, float* out, int32_t max_len, int32_t num_splits,
+                                        int32_t kernel, void* stream);
+
 /* Workspace bytes tpa_prefill_attention needs. */
 size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q,
                                   int32_t kernel);
