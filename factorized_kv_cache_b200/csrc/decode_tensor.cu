@@ -1,0 +1,711 @@
+// Tensor-core decode attention over the factorized cache (bf16, h = 32,
+// d_h = 128, R_K = R_V = R in {1, 2}).
+//
+// What it computes (Tensor Product Attention Is All You Need, sections
+// 关键设计 and FlashTPA; K and V are never expanded): for each cached token s
+// and head i,
+//   S'[i, (s, r)] = q~_i . B~_K[s, r]                        (tensor cores)
+//   z[i, s]       = scale/R_K * sum_r A_K[s, r, i] S'[i, (s, r)]
+//   online softmax over s, p[i, s] = 2^(z log2e - m)
+//   W[i, (s, r)]  = p[i, s] A_V[s, r, i] / R_V
+//   O[i, :]      += sum_(s, r) W[i, (s, r)] B_V[s, r, :]     (tensor cores)
+// The score contraction treats B_K rows as the shared "keys" of all 32 heads
+// (M = heads, N = token rows, K = d_h); the value contraction uses W as the
+// A operand (M = heads, K = token rows, N = d_h).  W is split into a bf16
+// high part and a bf16 remainder, two MMAs, so the softmax weights keep
+// about 16 bits; a single bf16 rounding of W costs ~1e-3 relative error,
+// too close to the 2e-3 budget.
+//
+// Data movement: one elected producer thread streams 64-row tiles of the
+// four cache planes with TMA (cp.async.bulk.tensor, no multicast) into a
+// 4-stage shared-memory ring guarded by mbarriers.  B tiles use the 128-byte
+// swizzle and A tiles the 64-byte swizzle, which makes every ldmatrix of the
+// consumers bank-conflict free.  Four consumer warps split each tile as
+// 2 head halves x 2 row halves; their softmax states merge through shared
+// memory whenever a sequence segment ends.
+//
+// Scheduling: the grid has G CTAs (one per SM by default).  The tiles of all
+// sequences are laid end to end (sequence-major) and CTA c takes tiles
+// [ceil(c NT / G), ceil((c+1) NT / G)): every CTA gets the same number of
+// tiles to within one, whatever the length mix.  A sequence whose tiles all
+// belong to one CTA is normalised and written directly.  Only the first and
+// the last sequence of a CTA's range can be shared with other CTAs; their
+// partial states (m, l, o) go to slots 2c and 2c+1, so the partials need
+// 2G slots whatever the batch size.  A small merge kernel, launched with
+// programmatic dependent launch, combines the partials of every other
+// sequence by log-sum-exp.
+#include <cuda.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "device_common.cuh"
+#include "ptx_sm100.cuh"
+#include "tma_host.h"
+#include "tpa_internal.h"
+#include "tpa_tensor.h"
+
+namespace tpa {
+namespace {
+
+constexpr int kH = 32;
+constexpr int kD = 128;
+constexpr int kRows = 64;                          // cache-plane rows per tile
+constexpr int kStages = 2;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kBoxBytes = kRows * 128;             // 64 features x kRows rows, bf16
+constexpr int kBBytes = 2 * kBoxBytes;             // one B tile (128 features)
+constexpr int kABytes = kRows * kH * 2;            // one A tile
+constexpr int kStageBytes = 2 * kBBytes + 2 * kABytes;
+constexpr int kMaxBatch = 1024;
+constexpr int kMergeFloats = 2 * 16 * kD + 2 * 16 * 2;  // two head halves: O[16][128] and (m, l)[16]
+constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kMergeFloats * 4 + 2 * kStages * 8 +
+                              (kMaxBatch + 1) * 4 + kMaxBatch * 4 + 64 * 4 + 64 * 2 * 4;
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+constexpr unsigned kErrTimeout = 0x8u;
+
+struct DecodeTcParams {
+  const int32_t* seq_lens;
+  const __nv_bfloat16* q;
+  const int32_t* q_pos;
+  int batch, capacity, max_len, grid;
+  float zs;                // scale * log2(e) / R_K
+  float* out;              // [B][32][128]
+  int32_t* ws_prefix;      // [B + 1]
+  float* ws_ml;            // [2G][32][2]
+  float* ws_o;             // [2G][32][128]
+  unsigned int* err;
+  RopeTable rope;
+};
+
+__device__ __forceinline__ int owner_of(int t, int nt, int grid) {
+  return static_cast<int>((static_cast<long long>(t) * grid) / nt);
+}
+
+// Exclusive prefix of per-sequence tile counts into s_pref[0..B], lengths into s_len.
+template <int TOK>
+__device__ void build_prefix(const DecodeTcParams& p, int32_t* s_pref, int32_t* s_len, int32_t* s_tmp) {
+  const int B = p.batch;
+  const int tid = threadIdx.x;
+  const int per = (B + kThreads - 1) / kThreads;
+  const int b0 = tid * per;
+  int local = 0;
+  for (int b = b0; b < min(B, b0 + per); ++b) {
+    int L = p.seq_lens[b];
+    if (L < 0 || L > p.capacity || L > p.max_len) {
+      if (blockIdx.x == 0) atomicOr(p.err, TPA_DEVERR_LEN_RANGE);
+      L = min(max(L, 0), min(p.capacity, p.max_len));
+    }
+    s_len[b] = L;
+    local += (L + TOK - 1) / TOK;
+  }
+  // inclusive scan of `local` over the CTA
+  const int lane = tid & 31, warp = tid >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_tmp[warp] = incl;
+  __syncthreads();
+  int warp_off = 0;
+  for (int w = 0; w < warp; ++w) warp_off += s_tmp[w];
+  int run = warp_off + incl - local;
+  for (int b = b0; b < min(B, b0 + per); ++b) {
+    s_pref[b] = run;
+    run += (s_len[b] + TOK - 1) / TOK;
+  }
+  if (tid == kThreads - 1) s_pref[B] = warp_off + incl;
+  __syncthreads();
+}
+
+template <int R>
+__global__ void __maxnreg__(200)
+    decode_tc_kernel(const __grid_constant__ DecodeTcParams p, const __grid_constant__ CUtensorMap tm_bk,
+                     const __grid_constant__ CUtensorMap tm_bv, const __grid_constant__ CUtensorMap tm_ak,
+                     const __grid_constant__ CUtensorMap tm_av) {
+  constexpr int TOK = kRows / R;  // tokens per tile
+  extern __shared__ uint8_t smem_raw[];
+  // the merge kernel may be scheduled now; it waits for this grid before reading
+  ptx::pdl_launch_dependents();
+
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  float* s_merge_o = reinterpret_cast<float*>(gbase + kStages * kStageBytes);  // [2][16][128]
+  float* s_merge_ml = s_merge_o + 2 * 16 * kD;                                  // [2][16][2]
+  uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_merge_ml + 2 * 16 * 2);      // full[kStages], empty[kStages]
+  int32_t* s_pref = reinterpret_cast<int32_t*>(s_bar + 2 * kStages);           // [kMaxBatch + 1]
+  int32_t* s_len = s_pref + kMaxBatch + 1;                                     // [kMaxBatch]
+  int32_t* s_tmp = s_len + kMaxBatch;                                          // [32] scan scratch
+  volatile int* s_abort = s_tmp + 32;                                          // set by a warp that timed out
+  float* s_cs = reinterpret_cast<float*>(s_tmp + 64);                          // [64][2] cos, sin of the query
+  const uint32_t bar_full = ptx::smem_u32(s_bar);
+  const uint32_t bar_empty = bar_full + 8 * kStages;
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(bar_full + 8 * s, 1);
+      ptx::mbar_init(bar_empty + 8 * s, kConsumerWarps);
+    }
+    *s_abort = 0;
+    ptx::fence_barrier_init();
+  }
+  build_prefix<TOK>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
+  const int B = p.batch;
+  const int NT = s_pref[B];
+  if (blockIdx.x == 0)
+    for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
+  if (NT == 0) return;
+  const int c = blockIdx.x;
+  const int t_begin = static_cast<int>((static_cast<long long>(c) * NT + p.grid - 1) / p.grid);
+  const int t_end = static_cast<int>((static_cast<long long>(c + 1) * NT + p.grid - 1) / p.grid);
+  if (t_begin >= t_end) return;
+  // first sequence with tiles in [t_begin, ...): largest b with s_pref[b] <= t_begin and s_pref[b+1] > t_begin
+  int b_first = 0;
+  {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_pref[mid] <= t_begin) lo = mid; else hi = mid - 1;
+    }
+    b_first = lo;
+    while (b_first < B && s_pref[b_first + 1] <= t_begin) ++b_first;
+  }
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_bk);
+      ptx::prefetch_tmap(&tm_bv);
+      ptx::prefetch_tmap(&tm_ak);
+      ptx::prefetch_tmap(&tm_av);
+      int it = 0;
+      bool ok = true;
+      for (int b = b_first; b < B && s_pref[b] < t_end && ok; ++b) {
+        const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
+        for (int t = ta; t < tb; ++t, ++it) {
+          const int stage = it % kStages;
+          const uint32_t par = ((it / kStages) & 1) ^ 1;
+          if (!ptx::mbar_wait_bounded(bar_empty + 8 * stage, par)) {
+            atomicOr(p.err, kErrTimeout);
+            ok = false;
+            break;
+          }
+          const int row0 = (b * p.capacity + (t - s_pref[b]) * TOK) * R;
+          const uint32_t st = sbase + stage * kStageBytes;
+          const uint32_t fb = bar_full + 8 * stage;
+          ptx::mbar_arrive_expect_tx(fb, kStageBytes);
+          ptx::tma_load_2d(st, &tm_bk, 0, row0, fb);
+          ptx::tma_load_2d(st + kBoxBytes, &tm_bk, 64, row0, fb);
+          ptx::tma_load_2d(st + kBBytes, &tm_bv, 0, row0, fb);
+          ptx::tma_load_2d(st + kBBytes + kBoxBytes, &tm_bv, 64, row0, fb);
+          ptx::tma_load_2d(st + 2 * kBBytes, &tm_ak, 0, row0, fb);
+          ptx::tma_load_2d(st + 2 * kBBytes + kABytes, &tm_av, 0, row0, fb);
+        }
+      }
+      if (!ok) {
+        // drain: let every load already issued land before the CTA can exit
+        for (int k = max(0, it - kStages); k < it; ++k)
+          ptx::mbar_wait_bounded(bar_full + 8 * (k % kStages), (k / kStages) & 1);
+      }
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int hh = warp & 1;   // head half: heads 16*hh .. 16*hh+15
+  const int rh = warp >> 1;  // row half: rows 32*rh .. 32*rh+31 of every tile
+  const int g = lane >> 2, q4 = lane & 3;
+  const int r0 = rh * 32;
+  const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: matrix index, row within matrix
+  int it = 0;
+
+  for (int b = b_first; b < B && s_pref[b] < t_end; ++b) {
+    const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
+    if (ta >= tb) continue;
+    const int len_b = s_len[b];
+    // ---- rotated query fragments for this sequence (bf16, A operand of the score MMA)
+    if (tid < kD / 2) {
+      float cs, sn;
+      rope_cos_sin(p.q_pos[b], p.rope.theta[tid], &cs, &sn);
+      s_cs[2 * tid] = cs;
+      s_cs[2 * tid + 1] = sn;
+    }
+    ptx::named_barrier(1, kConsumerWarps * 32);
+    uint32_t qa[8][4];
+    {
+      const __nv_bfloat16* qb = p.q + static_cast<size_t>(b) * kH * kD;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int j = kk * 8 + half * 4 + q4;  // RoPE pair = features (2j, 2j+1)
+          const float cs = s_cs[2 * j], sn = s_cs[2 * j + 1];
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            const int head = hh * 16 + g + 8 * hr;
+            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(qb + head * kD + 2 * j);
+            float x = __bfloat162float(v.x), y = __bfloat162float(v.y);
+            rope_pair(x, y, cs, sn);
+            qa[kk][hr + 2 * half] = ptx::pack_bf16(x, y);
+          }
+        }
+      }
+    }
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float O[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.f;
+
+    for (int t = ta; t < tb; ++t, ++it) {
+      const int stage = it % kStages;
+      if (*s_abort) break;
+      if (!ptx::mbar_wait_bounded(bar_full + 8 * stage, (it / kStages) & 1)) {
+        if (lane == 0) atomicOr(p.err, kErrTimeout);
+        *s_abort = 1;
+        break;
+      }
+      const uint32_t st = sbase + stage * kStageBytes;
+      const uint32_t s_bk = st, s_bv = st + kBBytes, s_ak = st + 2 * kBBytes, s_av = s_ak + kABytes;
+      const int tok0 = (t - s_pref[b]) * TOK;        // first token of the tile
+      const int valid_rows = min(kRows, (len_b - tok0) * R);
+      const bool partial = valid_rows < kRows;
+
+      // ---- scores S'[head][row] for the warp's 32 rows (4 n-tiles of 8)
+      float S[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) S[nt][0] = S[nt][1] = S[nt][2] = S[nt][3] = 0.f;
+#pragma unroll
+      for (int kk2 = 0; kk2 < 4; ++kk2) {
+        const int box = kk2 >> 1;
+        const int chunk = (kk2 & 1) * 4 + mi;
+        uint32_t bf[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+          const int row = r0 + nt * 8 + rr;
+          const uint32_t addr = s_bk + box * kBoxBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
+          ptx::ldsm_x4(addr, bf[nt][0], bf[nt][1], bf[nt][2], bf[nt][3]);
+        }
+        // four independent accumulators between two MMAs into the same one
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[2 * kk2], bf[nt][0], bf[nt][1]);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[2 * kk2 + 1], bf[nt][2], bf[nt][3]);
+      }
+      // ---- head factors A_K, A_V in the accumulator layout (ldmatrix.trans)
+      uint32_t akf[4][2], avf[4][2];
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int row = r0 + np * 16 + (mi >> 1) * 8 + rr;
+        const int chunk = 2 * hh + (mi & 1);
+        const uint32_t off = row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
+        ptx::ldsm_x4_t(s_ak + off, akf[2 * np][0], akf[2 * np][1], akf[2 * np + 1][0], akf[2 * np + 1][1]);
+        ptx::ldsm_x4_t(s_av + off, avf[2 * np][0], avf[2 * np][1], avf[2 * np + 1][0], avf[2 * np + 1][1]);
+      }
+      // ---- z = scale/R_K * sum_r A_K S' (log2 units), masked past the sequence end
+      // R == 1: z[nt][j] j = 0,1 head g (rows 2q4+j), j = 2,3 head g+8
+      // R == 2: z[nt][0] head g, z[nt][2] head g+8 (one token per n-tile)
+      float z[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int rowc = r0 + nt * 8 + 2 * q4;  // plane row of column 2*q4
+        if (R == 1) {
+          z[nt][0] = S[nt][0] * ptx::bf16_lo(akf[nt][0]) * p.zs;
+          z[nt][1] = S[nt][1] * ptx::bf16_hi(akf[nt][0]) * p.zs;
+          z[nt][2] = S[nt][2] * ptx::bf16_lo(akf[nt][1]) * p.zs;
+          z[nt][3] = S[nt][3] * ptx::bf16_hi(akf[nt][1]) * p.zs;
+          if (partial) {
+            if (rowc >= valid_rows) z[nt][0] = z[nt][2] = -INFINITY;
+            if (rowc + 1 >= valid_rows) z[nt][1] = z[nt][3] = -INFINITY;
+          }
+        } else {
+          z[nt][0] = (S[nt][0] * ptx::bf16_lo(akf[nt][0]) + S[nt][1] * ptx::bf16_hi(akf[nt][0])) * p.zs;
+          z[nt][2] = (S[nt][2] * ptx::bf16_lo(akf[nt][1]) + S[nt][3] * ptx::bf16_hi(akf[nt][1])) * p.zs;
+          if (partial && rowc >= valid_rows) z[nt][0] = z[nt][2] = -INFINITY;
+          z[nt][1] = z[nt][0];
+          z[nt][3] = z[nt][2];
+        }
+      }
+      // ---- online softmax per head row (the quad of lanes sharing g holds one head)
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        mx[0] = fmaxf(mx[0], fmaxf(z[nt][0], z[nt][1]));
+        mx[1] = fmaxf(mx[1], fmaxf(z[nt][2], z[nt][3]));
+      }
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+        mx[hr] = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 2));
+      }
+      float alpha[2], mn[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        mn[hr] = fmaxf(m[hr], mx[hr]);
+        alpha[hr] = (mn[hr] == -INFINITY) ? 1.f : exp2f(m[hr] - mn[hr]);
+        m[hr] = mn[hr];
+        l[hr] *= alpha[hr];
+      }
+      if (alpha[0] != 1.f || alpha[1] != 1.f) {
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          O[n][0] *= alpha[0];
+          O[n][1] *= alpha[0];
+          O[n][2] *= alpha[1];
+          O[n][3] *= alpha[1];
+        }
+      }
+      // ---- W = p A_V / R_V as hi + lo bf16 pairs (A operand of the value MMA)
+      float w[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const float p0 = (mn[0] == -INFINITY) ? 0.f : exp2f(z[nt][0] - mn[0]);
+        const float p2 = (mn[1] == -INFINITY) ? 0.f : exp2f(z[nt][2] - mn[1]);
+        if (R == 1) {
+          const float p1 = (mn[0] == -INFINITY) ? 0.f : exp2f(z[nt][1] - mn[0]);
+          const float p3 = (mn[1] == -INFINITY) ? 0.f : exp2f(z[nt][3] - mn[1]);
+          l[0] += p0 + p1;
+          l[1] += p2 + p3;
+          w[nt][0] = p0 * ptx::bf16_lo(avf[nt][0]);
+          w[nt][1] = p1 * ptx::bf16_hi(avf[nt][0]);
+          w[nt][2] = p2 * ptx::bf16_lo(avf[nt][1]);
+          w[nt][3] = p3 * ptx::bf16_hi(avf[nt][1]);
+          if (partial) {
+            const int rowc = r0 + nt * 8 + 2 * q4;
+            if (rowc >= valid_rows) w[nt][0] = w[nt][2] = 0.f;
+            if (rowc + 1 >= valid_rows) w[nt][1] = w[nt][3] = 0.f;
+          }
+        } else {
+          l[0] += p0;
+          l[1] += p2;
+          w[nt][0] = 0.5f * p0 * ptx::bf16_lo(avf[nt][0]);
+          w[nt][1] = 0.5f * p0 * ptx::bf16_hi(avf[nt][0]);
+          w[nt][2] = 0.5f * p2 * ptx::bf16_lo(avf[nt][1]);
+          w[nt][3] = 0.5f * p2 * ptx::bf16_hi(avf[nt][1]);
+          if (partial && r0 + nt * 8 + 2 * q4 >= valid_rows) w[nt][0] = w[nt][1] = w[nt][2] = w[nt][3] = 0.f;
+        }
+      }
+      // ---- O += W B_V over the warp's 32 rows (two k-chunks of 16 rows)
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc) {
+        uint32_t ahi[4], alo[4];
+        {
+          const float* w0 = w[2 * kc];
+          const float* w1 = w[2 * kc + 1];
+          ahi[0] = ptx::pack_bf16(w0[0], w0[1]);
+          ahi[1] = ptx::pack_bf16(w0[2], w0[3]);
+          ahi[2] = ptx::pack_bf16(w1[0], w1[1]);
+          ahi[3] = ptx::pack_bf16(w1[2], w1[3]);
+          alo[0] = ptx::pack_bf16(w0[0] - ptx::bf16_lo(ahi[0]), w0[1] - ptx::bf16_hi(ahi[0]));
+          alo[1] = ptx::pack_bf16(w0[2] - ptx::bf16_lo(ahi[1]), w0[3] - ptx::bf16_hi(ahi[1]));
+          alo[2] = ptx::pack_bf16(w1[0] - ptx::bf16_lo(ahi[2]), w1[1] - ptx::bf16_hi(ahi[2]));
+          alo[3] = ptx::pack_bf16(w1[2] - ptx::bf16_lo(ahi[3]), w1[3] - ptx::bf16_hi(ahi[3]));
+        }
+        const int krow = r0 + kc * 16;
+        // rows of this lane's B fragment elements (for masking a partial tile)
+        const int vr0 = krow + 2 * q4, vr1 = krow + 8 + 2 * q4;
+        // zero B_V elements of rows past the end (they may hold NaN; 0 * NaN would poison O)
+        const uint32_t m0 = partial ? ((vr0 < valid_rows ? 0x0000ffffu : 0u) | (vr0 + 1 < valid_rows ? 0xffff0000u : 0u))
+                                    : 0xffffffffu;
+        const uint32_t m1 = partial ? ((vr1 < valid_rows ? 0x0000ffffu : 0u) | (vr1 + 1 < valid_rows ? 0xffff0000u : 0u))
+                                    : 0xffffffffu;
+#pragma unroll
+        for (int g4 = 0; g4 < 2; ++g4) {
+          uint32_t v[4][4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int nd2 = g4 * 4 + u;
+            const int row = krow + (mi & 1) * 8 + rr;
+            const int d0 = nd2 * 16 + (mi >> 1) * 8;
+            const uint32_t addr = s_bv + (d0 >> 6) * kBoxBytes + row * 128 + ((((d0 & 63) >> 3) ^ (row & 7)) << 4);
+            ptx::ldsm_x4_t(addr, v[u][0], v[u][1], v[u][2], v[u][3]);
+            v[u][0] &= m0;
+            v[u][2] &= m0;
+            v[u][1] &= m1;
+            v[u][3] &= m1;
+          }
+          // eight independent accumulators between the hi and the lo MMA of each
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            ptx::mma_bf16(O[2 * (g4 * 4 + u)], ahi, v[u][0], v[u][1]);
+            ptx::mma_bf16(O[2 * (g4 * 4 + u) + 1], ahi, v[u][2], v[u][3]);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            ptx::mma_bf16(O[2 * (g4 * 4 + u)], alo, v[u][0], v[u][1]);
+            ptx::mma_bf16(O[2 * (g4 * 4 + u) + 1], alo, v[u][2], v[u][3]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_empty + 8 * stage);
+    }
+
+    // ---- end of this sequence's segment: merge row halves, write the result
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      l[hr] += __shfl_xor_sync(0xffffffffu, l[hr], 1);
+      l[hr] += __shfl_xor_sync(0xffffffffu, l[hr], 2);
+    }
+    float* mo = s_merge_o + hh * 16 * kD;
+    float* mml = s_merge_ml + hh * 32;
+    if (rh == 1) {
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const int d = n * 8 + 2 * q4;
+        *reinterpret_cast<float2*>(mo + g * kD + d) = make_float2(O[n][0], O[n][1]);
+        *reinterpret_cast<float2*>(mo + (g + 8) * kD + d) = make_float2(O[n][2], O[n][3]);
+      }
+      if (q4 == 0) {
+        mml[2 * g] = m[0];
+        mml[2 * g + 1] = l[0];
+        mml[2 * (g + 8)] = m[1];
+        mml[2 * (g + 8) + 1] = l[1];
+      }
+    }
+    ptx::named_barrier(1, kConsumerWarps * 32);
+    if (rh == 0) {
+      float M[2], Lt[2], f0[2], f1[2];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int hrow = g + 8 * hr;
+        const float m1 = mml[2 * hrow], l1 = mml[2 * hrow + 1];
+        M[hr] = fmaxf(m[hr], m1);
+        f0[hr] = (m[hr] == -INFINITY) ? 0.f : exp2f(m[hr] - M[hr]);
+        f1[hr] = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M[hr]);
+        Lt[hr] = l[hr] * f0[hr] + l1 * f1[hr];
+      }
+      const bool whole = owner_of(s_pref[b], NT, p.grid) == owner_of(s_pref[b + 1] - 1, NT, p.grid);
+      const int slot = 2 * c + (b == b_first ? 0 : 1);  // a shared sequence is the first or the last one
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        const int d = n * 8 + 2 * q4;
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int hrow = g + 8 * hr;
+          const float2 o1 = *reinterpret_cast<const float2*>(mo + hrow * kD + d);
+          float x = O[n][2 * hr] * f0[hr] + o1.x * f1[hr];
+          float y = O[n][2 * hr + 1] * f0[hr] + o1.y * f1[hr];
+          const int head = hh * 16 + hrow;
+          if (whole) {
+            const float inv = Lt[hr] > 0.f ? 1.f / Lt[hr] : 0.f;
+            *reinterpret_cast<float2*>(p.out + (static_cast<size_t>(b) * kH + head) * kD + d) =
+                make_float2(x * inv, y * inv);
+          } else {
+            *reinterpret_cast<float2*>(p.ws_o + (static_cast<size_t>(slot) * kH + head) * kD + d) =
+                make_float2(x, y);
+          }
+        }
+      }
+      if (!whole && q4 == 0) {
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int head = hh * 16 + g + 8 * hr;
+          p.ws_ml[(static_cast<size_t>(slot) * kH + head) * 2] = M[hr];
+          p.ws_ml[(static_cast<size_t>(slot) * kH + head) * 2 + 1] = Lt[hr];
+        }
+      }
+    }
+    ptx::named_barrier(1, kConsumerWarps * 32);  // merge buffer free for the next segment
+    if (*s_abort) break;  // every consumer warp sees the same flag after the barrier
+  }
+}
+
+// LSE merge of the partials of every sequence split across CTAs.  One CTA per
+// (sequence, head): the partials' (m, l) are read in parallel and reduced
+// across the CTA, then each thread accumulates one feature over the partials
+// with eight loads in flight.
+struct TcMergeParams {
+  int batch, grid;
+  const int32_t* prefix;
+  const float* ws_ml;
+  const float* ws_o;
+  float* out;
+};
+
+constexpr int kMergeThreads = 128;
+constexpr int kMergeChunk = 512;  // partials handled per pass
+
+__device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = is_max ? fmaxf(v, w) : v + w;
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  v = s_red[0];
+#pragma unroll
+  for (int k = 1; k < kMergeThreads / 32; ++k) v = is_max ? fmaxf(v, s_red[k]) : v + s_red[k];
+  return v;
+}
+
+__global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __grid_constant__ TcMergeParams p) {
+  ptx::pdl_wait();
+  __shared__ float s_w[kMergeChunk];
+  __shared__ int s_slot[kMergeChunk];
+  __shared__ float s_red[kMergeThreads / 32];
+  const int b = blockIdx.x, i = blockIdx.y, k = threadIdx.x;
+  const int NT = p.prefix[p.batch];
+  const int t0 = p.prefix[b], t1 = p.prefix[b + 1];
+  float* o = p.out + (static_cast<size_t>(b) * kH + i) * kD;
+  if (t1 <= t0) {
+    o[k] = 0.f;
+    return;
+  }
+  const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
+  if (cs == ce) return;  // written by the decode kernel
+  const int n = ce - cs + 1;
+  // CTA cc touched this sequence if its tile range [a, e) is non-empty and overlaps [t0, t1);
+  // the sequence is cc's first one (slot 2cc) when cc's range starts inside it, else its last (2cc + 1)
+  auto slot_of = [&](int cc) -> int {
+    const int a = static_cast<int>((static_cast<long long>(cc) * NT + p.grid - 1) / p.grid);
+    const int e = static_cast<int>((static_cast<long long>(cc + 1) * NT + p.grid - 1) / p.grid);
+    if (!(a < e && a < t1 && e > t0)) return -1;
+    return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
+  };
+  float M = -INFINITY;
+  for (int u = k; u < n; u += kMergeThreads) {
+    const int sl = slot_of(cs + u);
+    if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
+  }
+  M = merge_reduce(M, true, s_red);
+  float L = 0.f, acc = 0.f;
+  for (int c0 = 0; c0 < n; c0 += kMergeChunk) {
+    const int cn = min(kMergeChunk, n - c0);
+    float lpart = 0.f;
+    for (int u = k; u < cn; u += kMergeThreads) {
+      const int sl = slot_of(cs + c0 + u);
+      float w = 0.f;
+      if (sl >= 0) {
+        const float mj = p.ws_ml[2 * static_cast<size_t>(sl)];
+        w = mj == -INFINITY ? 0.f : exp2f(mj - M);
+        lpart = fmaf(p.ws_ml[2 * static_cast<size_t>(sl) + 1], w, lpart);
+      }
+      s_w[u] = w;
+      s_slot[u] = sl < 0 ? 0 : sl;
+    }
+    L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
+    int u = 0;
+    for (; u + 8 <= cn; u += 8) {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = p.ws_o[static_cast<size_t>(s_slot[u + q]) * kD + k];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc = fmaf(v[q], s_w[u + q], acc);
+    }
+    for (; u < cn; ++u) acc = fmaf(p.ws_o[static_cast<size_t>(s_slot[u]) * kD + k], s_w[u], acc);
+    __syncthreads();  // s_w, s_slot are rewritten by the next chunk
+  }
+  o[k] = L > 0.f ? acc / L : 0.f;
+}
+
+size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// The dynamic shared-memory opt-in, once per (device, rank variant).
+cudaError_t set_smem_once(int r) {
+  static std::once_flag once[64][2];
+  static cudaError_t status[64][2];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const int k = r == 1 ? 0 : 1;
+  std::call_once(once[dev][k], [dev, k]() {
+    auto kern = k == 0 ? decode_tc_kernel<1> : decode_tc_kernel<2>;
+    status[dev][k] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(kSmemBytes));
+  });
+  return status[dev][k];
+}
+
+struct TcWorkspace {
+  int32_t* prefix;
+  float* ml;
+  float* o;
+  size_t bytes;
+};
+
+TcWorkspace carve(void* base, int batch, int grid) {
+  TcWorkspace w;
+  const size_t slots = 2 * static_cast<size_t>(grid);
+  const size_t pb = round256((static_cast<size_t>(batch) + 1) * 4);
+  const size_t mlb = round256(slots * kH * 2 * 4);
+  const size_t ob = round256(slots * kH * kD * 4);
+  char* c = static_cast<char*>(base);
+  w.prefix = reinterpret_cast<int32_t*>(c);
+  w.ml = reinterpret_cast<float*>(c ? c + pb : nullptr);
+  w.o = reinterpret_cast<float*>(c ? c + pb + mlb : nullptr);
+  w.bytes = pb + mlb + ob;
+  return w;
+}
+
+}  // namespace
+
+bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_v) {
+  return dtype == TPA_BF16 && heads == kH && head_dim == kD && r_k == r_v && (r_k == 1 || r_k == 2);
+}
+
+bool tensor_decode_batch_ok(int batch) { return batch >= 1 && batch <= kMaxBatch; }
+
+int tensor_decode_default_ctas(int sms) { return 2 * (sms > 0 ? sms : 148); }  // two CTAs per SM
+
+size_t tensor_decode_workspace_bytes(int batch, int grid) { return carve(nullptr, batch, grid).bytes; }
+
+cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream) {
+  const CacheView& cv = a.cache;
+  const uint64_t rows_k = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_k;
+  const uint64_t rows_v = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_v;
+  CUtensorMap tbk, tbv, tak, tav;
+  cudaError_t e;
+  if ((e = encode_bf16_2d(&tbk, cv.b_k, kD, rows_k, 64, kRows, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tbv, cv.b_v, kD, rows_v, 64, kRows, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows_k, kH, kRows, 64)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows_v, kH, kRows, 64)) != cudaSuccess) return e;
+  TcWorkspace ws = carve(a.workspace, cv.batch, a.grid);
+  DecodeTcParams p;
+  p.seq_lens = cv.seq_lens;
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.q_pos = a.q_pos;
+  p.batch = cv.batch;
+  p.capacity = cv.capacity;
+  p.max_len = a.max_len;
+  p.grid = a.grid;
+  p.zs = a.scale * kLog2e / static_cast<float>(cv.r_k);
+  p.out = a.out;
+  p.ws_prefix = ws.prefix;
+  p.ws_ml = ws.ml;
+  p.ws_o = ws.o;
+  p.err = a.err;
+  p.rope = a.rope;
+  auto kern = cv.r_k == 1 ? decode_tc_kernel<1> : decode_tc_kernel<2>;
+  if ((e = set_smem_once(cv.r_k)) != cudaSuccess) return e;
+  kern<<<a.grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  TcMergeParams mp;
+  mp.batch = cv.batch;
+  mp.grid = a.grid;
+  mp.prefix = ws.prefix;
+  mp.ws_ml = ws.ml;
+  mp.ws_o = ws.o;
+  mp.out = a.out;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cv.batch, kH);
+  cfg.blockDim = dim3(kD);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel, mp);
+}
+
+}  // namespace tpa

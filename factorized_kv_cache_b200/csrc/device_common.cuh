@@ -54,9 +54,21 @@ __device__ __forceinline__ void store16_from_f32(T* __restrict__ p, const float*
 
 // cos/sin of pos * theta, the angle formed and evaluated in double precision
 // (positions reach 2^19, where an fp32 angle would be off by ~0.03 rad).
+// The angle is first reduced by 2*pi (Cody-Waite: 2*pi split into a 32-bit
+// head, so k * head is exact for k < 2^21, and a double tail); the reduced
+// |r| <= pi then takes sincos' short-argument path, which keeps the large
+// positions of long contexts as cheap as small ones.  The reduction is exact
+// up to |pos * theta| < 2^21 * 2*pi (1.3e7 rad) and off by less than 1e-15 rad there.
 __device__ __forceinline__ void rope_cos_sin(int pos, double theta, float* c, float* s) {
+  const double kTwoPiHi = 0x1.921fb544p+2;             // 2*pi rounded to 32 significant bits
+  const double kTwoPiLo = 0x1.0b4611a626331p-32;       // 2*pi - kTwoPiHi
+  const double kInvTwoPi = 0.15915494309189535;        // 1 / (2*pi)
+  const double x = static_cast<double>(pos) * theta;
+  const double k = rint(x * kInvTwoPi);
+  double r = fma(-k, kTwoPiHi, x);
+  r = fma(-k, kTwoPiLo, r);
   double sd, cd;
-  sincos(static_cast<double>(pos) * theta, &sd, &cd);
+  sincos(r, &sd, &cd);
   *c = static_cast<float>(cd);
   *s = static_cast<float>(sd);
 }

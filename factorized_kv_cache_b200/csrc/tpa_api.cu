@@ -109,13 +109,14 @@ int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b
 
 bool use_tensor_decode(const tpa_cache* c, int kernel) {
   if (kernel == TPA_KERNEL_SIMT) return false;
-  return tensor_decode_supported(c->dtype, c->heads, c->head_dim, c->r_k, c->r_v);
+  return tensor_decode_supported(c->dtype, c->heads, c->head_dim, c->r_k, c->r_v) &&
+         tensor_decode_batch_ok(c->batch);
 }
 
-SplitPlan plan_splits(const tpa_cache* c, int max_len, int num_splits, int kernel, int sms) {
+// CUDA-core decode: split j of sequence b covers tokens [j*chunk, (j+1)*chunk).
+SplitPlan plan_splits(const tpa_cache* c, int max_len, int num_splits, int sms) {
   SplitPlan p;
-  const bool tensor = use_tensor_decode(c, kernel);
-  const int granule = tensor ? tensor_decode_token_granule(c->r_k) : 16;
+  const int granule = 16;
   if (max_len <= 0) {
     p.splits = 1;
     p.chunk = granule;
@@ -123,16 +124,12 @@ SplitPlan plan_splits(const tpa_cache* c, int max_len, int num_splits, int kerne
   }
   int splits = num_splits;
   if (splits <= 0) {
-    if (tensor) {
-      splits = tensor_decode_default_splits(c->batch, max_len, c->r_k, sms);
-    } else {
-      // about eight 256-thread CTAs per SM, splits no shorter than 64 tokens
-      const int target = sms * 8;
-      splits = ceil_div(target, c->batch);
-      splits = splits < 1 ? 1 : splits;
-      const int max_splits = ceil_div(max_len, 64);
-      if (splits > max_splits) splits = max_splits;
-    }
+    // about eight 256-thread CTAs per SM, splits no shorter than 64 tokens
+    const int target = sms * 8;
+    splits = ceil_div(target, c->batch);
+    splits = splits < 1 ? 1 : splits;
+    const int max_splits = ceil_div(max_len, 64);
+    if (splits > max_splits) splits = max_splits;
   }
   if (splits < 1) splits = 1;
   int chunk = ceil_div(ceil_div(max_len, splits), granule) * granule;
@@ -244,14 +241,17 @@ int32_t tpa_decode_default_splits(const tpa_cache* cache, int32_t max_len, int32
   if (check_cache(cache) != TPA_OK || max_len < 0) return 0;
   int sms = 148;
   if (device_info(&sms, nullptr) != cudaSuccess) sms = 148;
-  return plan_splits(cache, max_len, 0, kernel, sms).splits;
+  if (use_tensor_decode(cache, kernel)) return tensor_decode_default_ctas(sms);
+  return plan_splits(cache, max_len, 0, sms).splits;
 }
 
 size_t tpa_decode_workspace_size(const tpa_cache* cache, int32_t max_len, int32_t num_splits, int32_t kernel) {
   if (check_cache(cache) != TPA_OK || max_len < 0) return 0;
   int sms = 148;
   if (device_info(&sms, nullptr) != cudaSuccess) sms = 148;
-  const SplitPlan p = plan_splits(cache, max_len, num_splits, kernel, sms);
+  if (use_tensor_decode(cache, kernel))
+    return tensor_decode_workspace_bytes(cache->batch, num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms));
+  const SplitPlan p = plan_splits(cache, max_len, num_splits, sms);
   return carve_decode_ws(nullptr, cache->batch, cache->heads, cache->head_dim, p.splits).bytes;
 }
 
@@ -276,7 +276,34 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
   unsigned int* err = nullptr;
   cudaError_t e = device_info(&sms, &err);
   if (e != cudaSuccess) return cuda_fail(e, "device query");
-  const SplitPlan plan = plan_splits(cache, max_len, num_splits, kernel, sms);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RopeTable rope;
+  make_rope_table(cache->rope_base, cache->head_dim, &rope);
+  if (kernel == TPA_KERNEL_TENSOR && !tensor_decode_batch_ok(cache->batch))
+    return fail(TPA_ERR_UNSUPPORTED, "tensor-core decode takes at most 1024 sequences per call");
+  if (use_tensor_decode(cache, kernel)) {
+    const int grid = num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms);
+    const size_t need = tensor_decode_workspace_bytes(cache->batch, grid);
+    if (!workspace) return fail(TPA_ERR_WORKSPACE, "workspace is NULL, %zu bytes needed", need);
+    if (workspace_bytes < need)
+      return fail(TPA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, need);
+    if (!aligned256(workspace)) return fail(TPA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+    TensorDecodeArgs a;
+    a.cache = view_of(cache);
+    a.q = q;
+    a.q_pos = q_pos;
+    a.scale = scale;
+    a.max_len = max_len;
+    a.grid = grid;
+    a.out = out;
+    a.workspace = workspace;
+    a.rope = rope;
+    a.err = err;
+    e = launch_tensor_decode(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
+    return TPA_OK;
+  }
+  const SplitPlan plan = plan_splits(cache, max_len, num_splits, sms);
   DecodeWs ws = carve_decode_ws(workspace, cache->batch, cache->heads, cache->head_dim, plan.splits);
   if (ws.bytes > 0) {
     if (!workspace) return fail(TPA_ERR_WORKSPACE, "workspace is NULL, %zu bytes needed", ws.bytes);
@@ -284,43 +311,23 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
       return fail(TPA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", workspace_bytes, ws.bytes);
     if (!aligned256(workspace)) return fail(TPA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
   }
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  RopeTable rope;
-  make_rope_table(cache->rope_base, cache->head_dim, &rope);
-  if (use_tensor_decode(cache, kernel)) {
-    TensorDecodeArgs a;
-    a.cache = view_of(cache);
-    a.q = q;
-    a.q_pos = q_pos;
-    a.scale = scale;
-    a.max_len = max_len;
-    a.plan = plan;
-    a.out = out;
-    a.ws_ml = ws.ml;
-    a.ws_o = ws.o;
-    a.rope = rope;
-    a.err = err;
-    e = launch_tensor_decode(a, st);
-    if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
-  } else {
-    SimtArgs a;
-    a.cache = view_of(cache);
-    a.q = q;
-    a.q_rotated_f32 = 0;
-    a.q_pos = q_pos;
-    a.q_per_seq = 1;
-    a.causal = 0;
-    a.scale = scale;
-    a.max_len = max_len;
-    a.plan = plan;
-    a.out = out;
-    a.ws_ml = ws.ml;
-    a.ws_o = ws.o;
-    a.rope = rope;
-    a.err = err;
-    e = launch_simt_attention(a, st);
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  }
+  SimtArgs a;
+  a.cache = view_of(cache);
+  a.q = q;
+  a.q_rotated_f32 = 0;
+  a.q_pos = q_pos;
+  a.q_per_seq = 1;
+  a.causal = 0;
+  a.scale = scale;
+  a.max_len = max_len;
+  a.plan = plan;
+  a.out = out;
+  a.ws_ml = ws.ml;
+  a.ws_o = ws.o;
+  a.rope = rope;
+  a.err = err;
+  e = launch_simt_attention(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   if (plan.splits > 1) {
     MergeArgs m;
     m.n_queries = cache->batch;

@@ -8,10 +8,12 @@
 
 namespace tpa {
 
-// ---- decode (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2})
+// ---- decode (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2}, batch <= 1024)
+// The grid is `grid` CTAs sharing the batch's tiles evenly (see decode_tensor.cu).
 bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_v);
-int tensor_decode_token_granule(int r_k);  // split lengths are multiples of this
-int tensor_decode_default_splits(int batch, int max_len, int r_k, int sms);
+bool tensor_decode_batch_ok(int batch);
+int tensor_decode_default_ctas(int sms);
+size_t tensor_decode_workspace_bytes(int batch, int grid);
 
 struct TensorDecodeArgs {
   CacheView cache;
@@ -19,10 +21,9 @@ struct TensorDecodeArgs {
   const int32_t* q_pos;
   float scale;
   int max_len;
-  SplitPlan plan;
+  int grid;
   float* out;
-  float* ws_ml;
-  float* ws_o;
+  void* workspace;  // tensor_decode_workspace_bytes(batch, grid) bytes, 256-byte aligned
   RopeTable rope;
   unsigned int* err;
 };

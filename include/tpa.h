@@ -57,7 +57,9 @@ typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
 
 /* Kernel choice for decode and prefill.  AUTO picks the fastest kernel that
  * supports the shape: the tensor-core kernels for bf16 at head_dim 128,
- * heads 32, r_k == r_v <= 2; the CUDA-core kernels otherwise. */
+ * heads 32, r_k == r_v <= 2 (decode: batch <= 1024); the CUDA-core kernels
+ * otherwise.  For the tensor-core decode, num_splits is the number of CTAs
+ * that share the batch's token tiles evenly (default: two per SM). */
 typedef enum tpa_kernel {
   TPA_KERNEL_AUTO = 0,
   TPA_KERNEL_SIMT = 1,   /* CUDA-core fp32 FMA path (every supported shape) */

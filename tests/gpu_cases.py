@@ -15,6 +15,8 @@ TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 def build_decode_cache(w: S.DecodeWorkload, batch=None, length=None, min_length=None, lengths=None,
                        nan_tail=True):
+    if lengths is not None:
+        min_length = 0          # explicit lengths replace the drawn ones
     x = S.decode_inputs(w, batch=batch, length=length, min_length=min_length)
     B, cap = x["a_k"].shape[:2]
     if lengths is not None:

@@ -129,3 +129,17 @@ def test_long_512k_workload_full_size(kernel):
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
     _check(w, cache, x, q, q_pos, out, heads=[0, 17, 31], end_to_end=False)
     assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("grid", [1, 2, 5, 37, 148, 300])
+@pytest.mark.parametrize("name", ["decode_b8_l8k", "decode_b32_var32k"])
+def test_tensor_kernel_partition_grids(grid, name):
+    """The tensor-core kernel's even split of all tiles over `grid` CTAs: sequences spanning
+    many CTAs, CTAs spanning many sequences, empty sequences, more CTAs than tiles."""
+    w = S.WORKLOADS[name]
+    lengths = [5000, 1, 0, 64, 65, 130, 3000, 7]
+    cache, x, q, q_pos = build_decode_cache(w, batch=8, length=5000, lengths=lengths)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=5000, num_splits=grid, kernel=T.TPA_KERNEL_TENSOR)
+    _check(w, cache, x, q, q_pos, out, end_to_end=False)
+    assert torch.count_nonzero(out[2]) == 0
+    assert T.tpa_read_device_error() == 0

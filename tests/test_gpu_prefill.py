@@ -49,9 +49,10 @@ def _oracle(w, cache, x, prior, tokens, b, rows=None, heads=None, end_to_end=Fal
 
 
 @pytest.mark.parametrize("kernel", KERNELS)
-@pytest.mark.parametrize("tokens,prior", [(1, 0), (200, 0), (130, 37), (257, 0)])
-def test_prefill_small(kernel, tokens, prior):
-    w = S.WORKLOADS["prefill_b4_t4k"]
+@pytest.mark.parametrize("rank", [2, 1])
+@pytest.mark.parametrize("tokens,prior", [(1, 0), (200, 0), (130, 37), (257, 0), (128, 300)])
+def test_prefill_small(kernel, rank, tokens, prior):
+    w = S.WORKLOADS["prefill_b4_t4k"].replace(r_k=rank, r_v=rank)
     cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, tokens, prior)
     out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos, kernel=kernel)
     assert T.tpa_read_device_error() == 0
@@ -76,18 +77,19 @@ def test_prefill_other_shapes(rq, rk, rv, h, d, dt):
         assert_rows_close(got[b], _oracle(w, cache, x, 11, 70, b), TOL[cache.dtype], f"shape b={b}")
 
 
-def test_prefill_longer_than_cache_is_reported():
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_longer_than_cache_is_reported(kernel):
     w = S.WORKLOADS["prefill_b4_t4k"]
     cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, 50)
     cache.seq_lens[1] = 20                         # sequence 1 holds fewer tokens than the chunk
     out = torch.full((2, 50, 32, 128), 7.0, device=DEV)
-    T.tpa_prefill_attention(cache, a_q, b_q, q_pos, out=out, kernel=T.TPA_KERNEL_SIMT)
+    T.tpa_prefill_attention(cache, a_q, b_q, q_pos, out=out, kernel=kernel)
     assert T.tpa_read_device_error() & T.TPA_DEVERR_PREFILL_LEN
     assert bool((out[1] == 7.0).all())
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("kernel", [T.TPA_KERNEL_AUTO])
+@pytest.mark.parametrize("kernel", KERNELS)
 def test_prefill_workload_full_size(kernel):
     """The full causal prefill (B=4, T=4096); oracle on sampled rows x heads."""
     w = S.WORKLOADS["prefill_b4_t4k"]

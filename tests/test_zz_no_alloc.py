@@ -48,18 +48,22 @@ def test_noalloc_too_many_splits_is_rejected_and_default_fits():
     w = S.WORKLOADS["decode_b8_l8k"]
     cache, x, q, q_pos = build_decode_cache(w, batch=64, length=600, min_length=300)
     out = torch.full((64, 32, 128), 3.0, dtype=torch.float32, device=DEV)
-    # 64 sequences x 32 splits x 32 heads x (128 + 2) floats = 34 MB > 16 MiB of scratch
+    # 2000 splits: CUDA-core partials 64 x 38 x 32 x (128 + 2) floats = 40 MB, tensor-core
+    # partials 2 x 2000 x 32 x (128 + 2) floats = 33 MB; either way above the 16 MiB of scratch
     with pytest.raises(T.TpaError) as e:
-        T.tpa_decode_attention_noalloc(cache, q, q_pos, out, max_len=600, num_splits=32)
+        T.tpa_decode_attention_noalloc(cache, q, q_pos, out, max_len=600, num_splits=2000)
     assert e.value.status == 5 and "scratch" in str(e.value)
     assert bool((out == 3.0).all())                        # nothing was launched
-    # 512 sequences: the default split count would need more than 16 MiB, so it is lowered
+    # 512 sequences on the CUDA-core kernel: the default split count would need more than
+    # 16 MiB of partials, so the entry point lowers it
     big, xb, qb, qpb = build_decode_cache(w, batch=512, length=600, min_length=1)
-    assert T.tpa_decode_workspace_size(big, 600) > (16 << 20) or T.tpa_decode_default_splits(big, 600) == 1
+    simt = T.TPA_KERNEL_SIMT
+    assert T.tpa_decode_workspace_size(big, 600, 0, simt) > (16 << 20)
     out_big = torch.empty(512, 32, 128, dtype=torch.float32, device=DEV)
-    for c, qq, qp, o in ((cache, q, q_pos, out), (big, qb, qpb, out_big)):   # two calls in a row
-        T.tpa_decode_attention_noalloc(c, qq, qp, o, max_len=600)
-    for c, qq, qp, o in ((cache, q, q_pos, out), (big, qb, qpb, out_big)):
-        ref = T.tpa_decode_attention(c, qq, qp, max_len=600)
+    calls = ((cache, q, q_pos, out, T.TPA_KERNEL_AUTO), (big, qb, qpb, out_big, simt))
+    for c, qq, qp, o, k in calls:                          # two calls in a row
+        T.tpa_decode_attention_noalloc(c, qq, qp, o, max_len=600, kernel=k)
+    for c, qq, qp, o, k in calls:
+        ref = T.tpa_decode_attention(c, qq, qp, max_len=600, kernel=k)
         assert_rows_close(o.double().cpu().numpy(), ref.double().cpu().numpy(), TOL[c.dtype], "default")
     assert T.tpa_read_device_error() == 0
