@@ -386,8 +386,55 @@ def add_cpu_baseline(res, x, w, lengths, target_s):
                                      f"{info['seconds']:.1f} s on {workers} spawned processes"}
 
 
+def run_reference_prefill(args, w):
+    """Reference arm for the prefill workload: the float64 oracle on sampled query rows."""
+    from factorized_kv_cache_b200 import synthetic as S
+    x = S.prefill_inputs(w)
+    host = {k: x[k].float().numpy() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v")}
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    K, W = args.steps, args.warmup
+    budget = 150.0 / max(1, K + W)
+    g = np.random.default_rng(0)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    rows_per_task = 8
+
+    def tasks(n):
+        return [(host["a_k"][t % w.batch], host["b_k"][t % w.batch], host["a_v"][t % w.batch],
+                 host["b_v"][t % w.batch], host["a_q"][t % w.batch], host["b_q"][t % w.batch],
+                 np.sort(g.integers(0, w.tokens, rows_per_task)), scale, w.rope_base) for t in range(n)]
+
+    t0 = time.perf_counter()
+    _prefill_oracle_task(tasks(1)[0])
+    per_task = time.perf_counter() - t0
+    tasks_per_step = max(1, min(workers, int(budget * workers / max(per_task, 1e-6))))
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        for _ in range(W):
+            pool.map(_prefill_oracle_task, tasks(tasks_per_step))
+        t0 = time.perf_counter()
+        done = 0
+        for _ in range(K):
+            done += sum(pool.map(_prefill_oracle_task, tasks(tasks_per_step)))
+        dt = time.perf_counter() - t0
+    value = done / dt
+    sample = (f"each step: {tasks_per_step} oracle prefills of {rows_per_task} random query rows (all heads, full "
+              f"causal prefix) of {w.name}, float64 oracle on {workers} spawned processes")
+    return {
+        "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": K,
+        "warmup": W, "ms_per_step": dt / max(1, K) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.tokens, "heads": w.heads,
+                   "head_dim": w.head_dim, "r_q": w.r_q, "r_k": w.r_k, "r_v": w.r_v},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
 def run_reference(args, w):
     """The float64 CPU oracle as the reference arm (host cores only)."""
+    from factorized_kv_cache_b200 import synthetic as S
+    if isinstance(w, S.PrefillWorkload):
+        return run_reference_prefill(args, w)
     x = decode_host_inputs(w, 0)
     lengths = x["lengths"].numpy().astype(np.int64)
     host = _host_arrays(x, lengths)
@@ -422,13 +469,190 @@ def run_reference(args, w):
     }
 
 
+# --------------------------------------------------------------------------- prefill bench
+PREFILL_METRIC = "causal prefill query tokens/sec (TPA, R_Q-factorized queries) + tensor TFLOP/s vs peak, 1×B200"
+
+
+def _prefill_oracle_task(args):
+    """Oracle prefill of a few query rows of one sequence (runs in a spawned worker)."""
+    import oracle.tpa_oracle as O
+    a_k, b_k, a_v, b_v, a_q, b_q, rows, scale, base = args
+    f = lambda a: np.asarray(a, dtype=np.float64)
+    L = a_k.shape[0]
+    pos = np.arange(L)
+    O.prefill_attention(f(a_k), O.append_rope(f(b_k), pos, base), f(a_v), f(b_v), f(a_q), f(b_q), pos, scale, base,
+                        rows=rows)
+    return len(rows)
+
+
+def run_ours_prefill(args, w, rank, world, dev):
+    import torch
+    import torch.distributed as dist
+    from factorized_kv_cache_b200 import synthetic as S
+    from factorized_kv_cache_b200 import tpa as T
+
+    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR}[args.kernel]
+    ww = w.replace(seed=w.seed + 1000 * rank) if rank else w
+    x = S.prefill_inputs(ww)
+    B, Tn = w.batch, w.tokens
+    cache = T.TpaCache.allocate(B, Tn, w.heads, w.head_dim, w.r_k, w.r_v, dtype=torch.bfloat16,
+                                rope_base=w.rope_base, device=dev)
+    cache.seq_lens.fill_(Tn)
+    d = {k: x[k].to(dev) for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v", "positions")}
+    slots = d["positions"]
+    out = torch.empty(B, Tn, w.heads, w.head_dim, dtype=torch.float32, device=dev)
+    ws = T.workspace(T.tpa_prefill_workspace_size(cache, Tn, w.r_q, kernel), dev)
+
+    def write():
+        T.tpa_cache_write_slots(cache, slots, d["positions"], d["a_k"], d["b_k"], d["a_v"], d["b_v"])
+
+    def prefill():
+        T.tpa_prefill_attention(cache, d["a_q"], d["b_q"], d["positions"], out=out, kernel=kernel, workspace_buf=ws)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        write()
+        prefill()
+    torch.cuda.synchronize(dev)
+    gw, gp = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw, stream=stream):
+        write()
+    with torch.cuda.graph(gp, stream=stream):
+        prefill()
+    torch.cuda.synchronize(dev)
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set after set-up")
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for _ in range(W):
+            gw.replay()
+            gp.replay()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for k in range(K):
+            gw.replay()
+            ev[k][0].record(stream)
+            gp.replay()
+            ev[k][1].record(stream)
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    pre_ms = [a.elapsed_time(b) for a, b in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    # e2e: host factors and queries in, output back, through the public API
+    host = {k: x[k].pin_memory() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v", "positions")}
+    host_out = torch.empty_like(out, device="cpu").pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = host_out.numel() * 4
+    e2e_steps = max(1, min(K, 20))
+
+    def e2e_step():
+        with torch.cuda.stream(stream):
+            for k2, v in host.items():
+                d[k2].copy_(v, non_blocking=True)
+            T.tpa_cache_write_slots(cache, d["positions"], d["positions"], d["a_k"], d["b_k"], d["a_v"], d["b_v"],
+                                    stream=stream)
+            T.tpa_prefill_attention(cache, d["a_q"], d["b_q"], d["positions"], out=out, kernel=kernel,
+                                    workspace_buf=ws, stream=stream)
+            host_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    e2e_step()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2e_s = time.perf_counter() - t0
+
+    pairs = B * Tn * (Tn + 1) // 2
+    flops = pairs * w.heads * 2 * w.head_dim * (w.r_k + w.r_v)   # score + value contractions, per (query, key) pair
+    mean_s = statistics.mean(pre_ms) / 1e3
+    peaks, kind = measured_peaks()
+    achieved = flops / mean_s / 1e12
+    tensor = kernel != T.TPA_KERNEL_SIMT
+    src = ["factorized_kv_cache_b200/csrc/prefill_tensor.cu"] if tensor else ["factorized_kv_cache_b200/csrc/attention_simt.cu"]
+    res = {
+        "metric": PREFILL_METRIC, "value": world * B * Tn * K / (elapsed_ms / 1e3), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (x~N(0,1) width 2048, factors x W with W~N(0,1/2048))",
+        "config": {"workload": w.name, "batch": B, "seq_len": Tn, "heads": w.heads, "head_dim": w.head_dim,
+                   "r_q": w.r_q, "r_k": w.r_k, "r_v": w.r_v, "kernel": args.kernel,
+                   "step": "write prompt factors (RoPE on B_K) + causal prefill, CUDA graphs",
+                   "l2": "inputs larger than L2 (query workspace 134 MB + output 268 MB per step)",
+                   "parallelism": f"dp{world} (independent batches, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": ncu_traffic(w.name, src), "peak_kind": kind + " (bf16 burst)",
+                     "kernel": "prefill attention call (query build + causal attention)",
+                     "algorithmic_flops_per_launch": flops, "mean_launch_us": mean_s * 1e6},
+        "e2e": {"value": world * B * Tn * e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": K * 3,
+        "clocks": clk,
+    }
+    return res, x
+
+
+def add_prefill_cpu_baseline(res, x, w, target_s):
+    host = {k: x[k].float().numpy() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v")}
+    workers = max(1, min(os.cpu_count() or 1, 16))
+    rows_per_task = 16
+    g = np.random.default_rng(0)
+    scale = 1.0 / math.sqrt(w.head_dim)
+
+    def tasks(n):
+        out = []
+        for t in range(n):
+            b = t % w.batch
+            rows = np.sort(g.integers(0, w.tokens, rows_per_task))
+            out.append((host["a_k"][b], host["b_k"][b], host["a_v"][b], host["b_v"][b], host["a_q"][b],
+                        host["b_q"][b], rows, scale, w.rope_base))
+        return out
+
+    t0 = time.perf_counter()
+    _prefill_oracle_task(tasks(1)[0])
+    per_task = time.perf_counter() - t0
+    n = max(workers, int(target_s * workers / max(per_task, 1e-6)))
+    n = (n + workers - 1) // workers * workers
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers) as pool:
+        tl = tasks(n)
+        t0 = time.perf_counter()
+        done = sum(pool.map(_prefill_oracle_task, tl, chunksize=1))
+        dt = time.perf_counter() - t0
+    res["cpu_baseline"] = {"value": done / dt, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                           "sample": f"{n} oracle prefills of {rows_per_task} random query rows (all heads, full "
+                                     f"causal prefix, RoPE included) of {w.name}; {dt:.1f} s on {workers} "
+                                     f"spawned processes"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode_b8_l8k")
+    ap.add_argument("--workload", default="decode_b8_l8k",
+                    choices=["decode_tiny_f32", "decode_b8_l8k", "decode_b32_var32k", "prefill_b4_t4k",
+                             "decode_long_512k"])
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
     args = ap.parse_args()
@@ -454,9 +678,14 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     try:
-        res, x, lengths = run_ours_decode(args, w, rank, world, dev)
-        if rank == 0 and args.cpu_seconds > 0:
-            add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
+        if isinstance(w, S.PrefillWorkload):
+            res, x = run_ours_prefill(args, w, rank, world, dev)
+            if rank == 0 and args.cpu_seconds > 0:
+                add_prefill_cpu_baseline(res, x, w, args.cpu_seconds)
+        else:
+            res, x, lengths = run_ours_decode(args, w, rank, world, dev)
+            if rank == 0 and args.cpu_seconds > 0:
+                add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -592,15 +592,23 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       s_slot[u] = sl < 0 ? 0 : sl;
     }
     L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
+    // partials of CTAs that did not touch this sequence carry weight 0 and point at slot 0,
+    // whose contents may be anything: select, never multiply, them away
     int u = 0;
     for (; u + 8 <= cn; u += 8) {
       float v[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) v[q] = p.ws_o[static_cast<size_t>(s_slot[u + q]) * kD + k];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc = fmaf(v[q], s_w[u + q], acc);
+      for (int q = 0; q < 8; ++q) {
+        const float wq = s_w[u + q];
+        acc = fmaf(wq != 0.f ? v[q] : 0.f, wq, acc);
+      }
     }
-    for (; u < cn; ++u) acc = fmaf(p.ws_o[static_cast<size_t>(s_slot[u]) * kD + k], s_w[u], acc);
+    for (; u < cn; ++u) {
+      const float wq = s_w[u];
+      if (wq != 0.f) acc = fmaf(p.ws_o[static_cast<size_t>(s_slot[u]) * kD + k], wq, acc);
+    }
     __syncthreads();  // s_w, s_slot are rewritten by the next chunk
   }
   o[k] = L > 0.f ? acc / L : 0.f;
