@@ -655,12 +655,21 @@ def main():
                              "decode_long_512k"])
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
+    ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     from factorized_kv_cache_b200 import synthetic as S
     w = S.WORKLOADS[args.workload]
+    if args.batch > 0:
+        w = w.replace(batch=args.batch)
+    if args.seq_len > 0:
+        if isinstance(w, S.PrefillWorkload):
+            w = w.replace(tokens=args.seq_len)
+        else:
+            w = w.replace(length=args.seq_len, min_length=min(w.min_length, args.seq_len))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -59,10 +59,14 @@ constexpr int kBBytes = 2 * kBoxBytes;             // one B tile (128 features)
 constexpr int kABytes = kRows * kH * 2;            // one A tile
 constexpr int kStageBytes = 2 * kBBytes + 2 * kABytes;
 constexpr int kMaxBatch = 1024;
-constexpr int kMergeFloats = 2 * 16 * kD + 2 * 16 * 2;  // two head halves: O[16][128] and (m, l)[16]
+// Per-segment scratch: the rotated query (bf16 [32][128], 8 KB, swizzled for
+// ldmatrix) while tiles are processed, then the row-half merge buffers
+// (O[2][16][128] and (m, l)[2][16]) at the end of the segment.
+constexpr int kMergeFloats = 2 * 16 * kD + 2 * 16 * 2;
 constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kMergeFloats * 4 + 2 * kStages * 8 +
                               (kMaxBatch + 1) * 4 + kMaxBatch * 4 + 64 * 4 + 64 * 2 * 4;
 static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(kH * kD * 2 <= 2 * 16 * kD * 4, "query fits in the merge buffer");
 constexpr unsigned kErrTimeout = 0x8u;
 
 struct DecodeTcParams {
@@ -122,7 +126,7 @@ __device__ void build_prefix(const DecodeTcParams& p, int32_t* s_pref, int32_t* 
 }
 
 template <int R>
-__global__ void __maxnreg__(200)
+__global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition: two CTAs per SM
     decode_tc_kernel(const __grid_constant__ DecodeTcParams p, const __grid_constant__ CUtensorMap tm_bk,
                      const __grid_constant__ CUtensorMap tm_bv, const __grid_constant__ CUtensorMap tm_ak,
                      const __grid_constant__ CUtensorMap tm_av) {
@@ -135,6 +139,7 @@ __global__ void __maxnreg__(200)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw);
   float* s_merge_o = reinterpret_cast<float*>(gbase + kStages * kStageBytes);  // [2][16][128]
+  const uint32_t s_q = sbase + kStages * kStageBytes;  // rotated query, aliases s_merge_o during a segment
   float* s_merge_ml = s_merge_o + 2 * 16 * kD;                                  // [2][16][2]
   uint64_t* s_bar = reinterpret_cast<uint64_t*>(s_merge_ml + 2 * 16 * 2);      // full[kStages], empty[kStages]
   int32_t* s_pref = reinterpret_cast<int32_t*>(s_bar + 2 * kStages);           // [kMaxBatch + 1]
@@ -237,26 +242,21 @@ __global__ void __maxnreg__(200)
       s_cs[2 * tid + 1] = sn;
     }
     ptx::named_barrier(1, kConsumerWarps * 32);
-    uint32_t qa[8][4];
     {
+      // q~ as bf16 rows of 256 B, 16-byte chunks XOR-swizzled by (row & 7) within each 128-byte half
       const __nv_bfloat16* qb = p.q + static_cast<size_t>(b) * kH * kD;
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int j = kk * 8 + half * 4 + q4;  // RoPE pair = features (2j, 2j+1)
-          const float cs = s_cs[2 * j], sn = s_cs[2 * j + 1];
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            const int head = hh * 16 + g + 8 * hr;
-            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(qb + head * kD + 2 * j);
-            float x = __bfloat162float(v.x), y = __bfloat162float(v.y);
-            rope_pair(x, y, cs, sn);
-            qa[kk][hr + 2 * half] = ptx::pack_bf16(x, y);
-          }
-        }
+      uint8_t* sq = gbase + kStages * kStageBytes;
+      for (int e = tid; e < kH * kD / 2; e += kConsumerWarps * 32) {
+        const int head = e / (kD / 2), j = e % (kD / 2);  // RoPE pair j = features (2j, 2j+1)
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(qb + head * kD + 2 * j);
+        float x = __bfloat162float(v.x), y = __bfloat162float(v.y);
+        rope_pair(x, y, s_cs[2 * j], s_cs[2 * j + 1]);
+        const int c = j >> 2;
+        const int pc = (c & 8) | ((c & 7) ^ (head & 7));
+        *reinterpret_cast<uint32_t*>(sq + head * 256 + pc * 16 + (j & 3) * 4) = ptx::pack_bf16(x, y);
       }
     }
+    ptx::named_barrier(1, kConsumerWarps * 32);
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     float O[16][4];
 #pragma unroll
@@ -284,6 +284,15 @@ __global__ void __maxnreg__(200)
       for (int kk2 = 0; kk2 < 4; ++kk2) {
         const int box = kk2 >> 1;
         const int chunk = (kk2 & 1) * 4 + mi;
+        // query fragments of k-steps 2*kk2 and 2*kk2+1 (A operand: heads x 16 features)
+        uint32_t qa[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int qrow = hh * 16 + (mi & 1) * 8 + rr;
+          const int c = (2 * kk2 + u) * 2 + (mi >> 1);
+          const int pc = (c & 8) | ((c & 7) ^ (qrow & 7));
+          ptx::ldsm_x4(s_q + qrow * 256 + pc * 16, qa[u][0], qa[u][1], qa[u][2], qa[u][3]);
+        }
         uint32_t bf[4][4];
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
@@ -293,9 +302,9 @@ __global__ void __maxnreg__(200)
         }
         // four independent accumulators between two MMAs into the same one
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[2 * kk2], bf[nt][0], bf[nt][1]);
+        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[0], bf[nt][0], bf[nt][1]);
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[2 * kk2 + 1], bf[nt][2], bf[nt][3]);
+        for (int nt = 0; nt < 4; ++nt) ptx::mma_bf16(S[nt], qa[1], bf[nt][2], bf[nt][3]);
       }
       // ---- head factors A_K, A_V in the accumulator layout (ldmatrix.trans)
       uint32_t akf[4][2], avf[4][2];
@@ -454,6 +463,7 @@ __global__ void __maxnreg__(200)
     }
     float* mo = s_merge_o + hh * 16 * kD;
     float* mml = s_merge_ml + hh * 32;
+    ptx::named_barrier(1, kConsumerWarps * 32);  // every warp is done with the query (same bytes)
     if (rh == 1) {
 #pragma unroll
       for (int n = 0; n < 16; ++n) {
@@ -517,9 +527,11 @@ __global__ void __maxnreg__(200)
 }
 
 // LSE merge of the partials of every sequence split across CTAs.  One CTA per
-// (sequence, head): the partials' (m, l) are read in parallel and reduced
-// across the CTA, then each thread accumulates one feature over the partials
-// with eight loads in flight.
+// (sequence, head).  The touched CTAs of sequence b are cs..ce; when every CTA
+// owns at least one tile (G <= NT) they all touched b, b is the first sequence
+// of each of them but possibly cs, and only cs needs a division.  The (m, l)
+// pairs are reduced across the CTA; the features are then summed with every
+// partial's float4 loads in flight at once (4 partial groups x 32 float4).
 struct TcMergeParams {
   int batch, grid;
   const int32_t* prefix;
@@ -529,7 +541,7 @@ struct TcMergeParams {
 };
 
 constexpr int kMergeThreads = 128;
-constexpr int kMergeChunk = 512;  // partials handled per pass
+constexpr int kMergeMax = 1024;  // partials per pass
 
 __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red) {
 #pragma unroll
@@ -546,42 +558,51 @@ __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red
   return v;
 }
 
+__device__ __forceinline__ int ceil_tile(int c, int nt, int grid) {
+  return static_cast<int>((static_cast<long long>(c) * nt + grid - 1) / grid);
+}
+
 __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __grid_constant__ TcMergeParams p) {
   ptx::pdl_wait();
-  __shared__ float s_w[kMergeChunk];
-  __shared__ int s_slot[kMergeChunk];
+  __shared__ float s_w[kMergeMax];
+  __shared__ int s_slot[kMergeMax];
   __shared__ float s_red[kMergeThreads / 32];
-  const int b = blockIdx.x, i = blockIdx.y, k = threadIdx.x;
+  __shared__ float4 s_acc[4][32];
+  const int b = blockIdx.x, i = blockIdx.y, tid = threadIdx.x;
   const int NT = p.prefix[p.batch];
   const int t0 = p.prefix[b], t1 = p.prefix[b + 1];
   float* o = p.out + (static_cast<size_t>(b) * kH + i) * kD;
   if (t1 <= t0) {
-    o[k] = 0.f;
+    o[tid] = 0.f;
     return;
   }
   const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
   if (cs == ce) return;  // written by the decode kernel
   const int n = ce - cs + 1;
-  // CTA cc touched this sequence if its tile range [a, e) is non-empty and overlaps [t0, t1);
-  // the sequence is cc's first one (slot 2cc) when cc's range starts inside it, else its last (2cc + 1)
-  auto slot_of = [&](int cc) -> int {
-    const int a = static_cast<int>((static_cast<long long>(cc) * NT + p.grid - 1) / p.grid);
-    const int e = static_cast<int>((static_cast<long long>(cc + 1) * NT + p.grid - 1) / p.grid);
+  const bool dense = p.grid <= NT;
+  const bool cs_first = ceil_tile(cs, NT, p.grid) >= t0;
+  // slot (in units of [slot][head]) of CTA cs + u for this sequence, -1 if it did not touch it
+  auto slot_of = [&](int u) -> int {
+    const int cc = cs + u;
+    if (dense) return (2 * cc + ((u > 0 || cs_first) ? 0 : 1)) * kH + i;
+    const int a = ceil_tile(cc, NT, p.grid), e = ceil_tile(cc + 1, NT, p.grid);
     if (!(a < e && a < t1 && e > t0)) return -1;
     return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
   };
   float M = -INFINITY;
-  for (int u = k; u < n; u += kMergeThreads) {
-    const int sl = slot_of(cs + u);
+  for (int u = tid; u < n; u += kMergeThreads) {
+    const int sl = slot_of(u);
     if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
   }
   M = merge_reduce(M, true, s_red);
-  float L = 0.f, acc = 0.f;
-  for (int c0 = 0; c0 < n; c0 += kMergeChunk) {
-    const int cn = min(kMergeChunk, n - c0);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
+  for (int c0 = 0; c0 < n; c0 += kMergeMax) {
+    const int cn = min(kMergeMax, n - c0);
     float lpart = 0.f;
-    for (int u = k; u < cn; u += kMergeThreads) {
-      const int sl = slot_of(cs + c0 + u);
+    for (int u = tid; u < cn; u += kMergeThreads) {
+      const int sl = slot_of(c0 + u);
       float w = 0.f;
       if (sl >= 0) {
         const float mj = p.ws_ml[2 * static_cast<size_t>(sl)];
@@ -589,29 +610,35 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
         lpart = fmaf(p.ws_ml[2 * static_cast<size_t>(sl) + 1], w, lpart);
       }
       s_w[u] = w;
-      s_slot[u] = sl < 0 ? 0 : sl;
+      s_slot[u] = sl;
     }
     L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
-    // partials of CTAs that did not touch this sequence carry weight 0 and point at slot 0,
-    // whose contents may be anything: select, never multiply, them away
-    int u = 0;
-    for (; u + 8 <= cn; u += 8) {
-      float v[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = p.ws_o[static_cast<size_t>(s_slot[u + q]) * kD + k];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float wq = s_w[u + q];
-        acc = fmaf(wq != 0.f ? v[q] : 0.f, wq, acc);
-      }
+    for (int u = grp; u < cn; u += 4) {
+      const int sl = s_slot[u];
+      if (sl < 0) continue;  // never read a partial this sequence did not write
+      const float w = s_w[u];
+      const float4 v = reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4];
+      acc.x = fmaf(v.x, w, acc.x);
+      acc.y = fmaf(v.y, w, acc.y);
+      acc.z = fmaf(v.z, w, acc.z);
+      acc.w = fmaf(v.w, w, acc.w);
     }
-    for (; u < cn; ++u) {
-      const float wq = s_w[u];
-      if (wq != 0.f) acc = fmaf(p.ws_o[static_cast<size_t>(s_slot[u]) * kD + k], wq, acc);
-    }
-    __syncthreads();  // s_w, s_slot are rewritten by the next chunk
+    __syncthreads();  // s_w, s_slot are rewritten by the next pass
   }
-  o[k] = L > 0.f ? acc / L : 0.f;
+  s_acc[grp][f4] = acc;
+  __syncthreads();
+  if (tid < 32) {
+    float4 r = s_acc[0][tid];
+#pragma unroll
+    for (int g2 = 1; g2 < 4; ++g2) {
+      r.x += s_acc[g2][tid].x;
+      r.y += s_acc[g2][tid].y;
+      r.z += s_acc[g2][tid].z;
+      r.w += s_acc[g2][tid].w;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    reinterpret_cast<float4*>(o)[tid] = make_float4(r.x * inv, r.y * inv, r.z * inv, r.w * inv);
+  }
 }
 
 size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
@@ -627,10 +654,29 @@ cudaError_t set_smem_once(int r) {
   const int k = r == 1 ? 0 : 1;
   std::call_once(once[dev][k], [dev, k]() {
     auto kern = k == 0 ? decode_tc_kernel<1> : decode_tc_kernel<2>;
-    status[dev][k] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(kSmemBytes));
+    if (e2 == cudaSuccess)
+      e2 = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    status[dev][k] = e2;
   });
   return status[dev][k];
+}
+
+// CTAs of the decode kernel resident per SM (queried once per device).
+int ctas_per_sm() {
+  static std::once_flag once[64];
+  static int occ[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::call_once(once[dev], [dev]() {
+    int n = 1;
+    if (set_smem_once(1) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<1>, kThreads, kSmemBytes) != cudaSuccess)
+      n = 1;
+    occ[dev] = n < 1 ? 1 : n;
+  });
+  return occ[dev];
 }
 
 struct TcWorkspace {
@@ -662,7 +708,8 @@ bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_
 
 bool tensor_decode_batch_ok(int batch) { return batch >= 1 && batch <= kMaxBatch; }
 
-int tensor_decode_default_ctas(int sms) { return 2 * (sms > 0 ? sms : 148); }  // two CTAs per SM
+// One wave: every resident CTA slot of the GPU.
+int tensor_decode_default_ctas(int sms) { return ctas_per_sm() * (sms > 0 ? sms : 148); }
 
 size_t tensor_decode_workspace_bytes(int batch, int grid) { return carve(nullptr, batch, grid).bytes; }
 

@@ -10,8 +10,9 @@
 //   z[t, s]     = scale/R_K sum_r A_K[s, r, i] S[t, (s, r)],  s <= P + t
 //   W[t, (s,r)] = softmax_s(z)[t, s] A_V[s, r, i] / R_V
 //   O[t, i, :]  = sum_(s,r) W[t, (s,r)] B_V[s, r, :]         (tensor cores)
-// The dense per-head query tile is the only thing expanded: it is built once
-// per chunk by prefill_q_kernel (bf16) and read by TMA.  Keys and values stay
+// The dense per-head query is the only thing expanded: it is built once per
+// chunk in fp32 by prefill_q_kernel, then each softmax thread splits its own
+// query row into bf16 high and low parts in TMEM.  Keys and values stay
 // factorized: the score MMA contracts the query with B_K rows, and the value
 // MMA contracts the softmax weights with B_V rows.  Putting the head factors
 // on the query side of the MMA (a dense Q tile per head) costs 2 h d_h R_K
@@ -20,18 +21,20 @@
 // FMAs per pair to apply A_Q and A_K, which is slower on this machine.
 //
 // CTA = (sequence, head, tile of 128 queries); heavy (late) query tiles are
-// dispatched first.  Roles: warp 0 issues TMA loads (query tile once, then a
-// 2-stage ring of {B_K, B_V, A_K, A_V} tiles of 128 cache rows); warp 1
-// allocates 256 TMEM columns and one of its threads issues the MMAs; warps
-// 2-5 (one TMEM lane = one query row per thread) run the softmax.
-// Per key tile: S = Q B_K^T (M = 128 queries, N = 128 rows, K = 128) into
-// TMEM columns [0, 128); the softmax reads S, applies A_K, the causal mask
+// dispatched first.  Roles: warp 0 issues TMA loads (a 2-stage ring of
+// {B_K, B_V, A_K, A_V} tiles of 128 cache rows); warp 1 allocates 512 TMEM
+// columns and one of its threads issues the MMAs; warps 2-5 (one TMEM lane =
+// one query row per thread) stage the query and run the softmax.
+// Per key tile: S = (Q_hi + Q_lo) B_K^T (M = 128 queries, N = 128 rows,
+// K = 128; A from TMEM columns [256, 384)) into TMEM columns [0, 128); the
+// softmax reads S, applies A_K, the causal mask
 // and the online softmax, rescales O in TMEM when the running maximum grows
 // by more than 2^8, and writes W as bf16 hi and lo halves into TMEM columns
 // [0, 64) and [64, 128) (over S); then O += W_hi B_V + W_lo B_V (A from TMEM,
-// B_V as an MN-major operand) into columns [128, 256).  The split of W into
-// two bf16 parts keeps the weights to ~16 bits (one bf16 rounding costs ~3e-3
-// relative error on this workload).
+// B_V as an MN-major operand) into columns [128, 256).  Both the query and W
+// are split into two bf16 parts, which keeps them to ~16 bits: one bf16
+// rounding of either costs ~3.5e-3 relative error on the prefill workload,
+// above its 2e-3 budget.
 #include <cuda.h>
 #include <math.h>
 
@@ -52,19 +55,18 @@ constexpr int kQ = 128;                 // queries per CTA
 constexpr int kKRows = 128;             // cache rows per key tile
 constexpr int kStages = 2;
 constexpr int kThreads = 192;
-constexpr int kQBytes = kQ * kD * 2;    // 32 KB: two 64-feature boxes
 constexpr int kBox = kKRows * 128;      // 16 KB: one 64-feature box of a B tile
 constexpr int kBTile = 2 * kBox;
 constexpr int kATile = kKRows * kH * 2; // 8 KB
 constexpr int kStageBytes = 2 * kBTile + 2 * kATile;
-constexpr int kOffStages = kQBytes;
+constexpr int kOffStages = 0;
 constexpr int kOffAf = kOffStages + kStages * kStageBytes;  // fp32 A_K, A_V of the head: [2 stages][2][128]
 constexpr int kOffBar = kOffAf + kStages * 2 * kKRows * 4;
-constexpr int kNumBars = 2 * kStages + 5;  // full[2], empty[2], q_full, s_full, w_ready, o_done, final
+constexpr int kNumBars = 2 * kStages + 5;  // full[2], empty[2], q_ready, s_full, w_ready, o_done, final
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 constexpr unsigned kErrTimeout = 0x8u;
 
 // instruction descriptors, kind::f16: D fp32, A and B bf16, M = 128, N = 128
@@ -76,13 +78,14 @@ struct PrefillTcParams {
   int batch, capacity, n_tokens, n_qtiles;
   float zs;       // scale * log2(e) / R_K
   float inv_rv;   // 1 / R_V
-  float* out;     // [B][T][32][128]
+  const float* q;  // [B][T][32][128] fp32 rotated queries
+  float* out;      // [B][T][32][128]
   unsigned int* err;
 };
 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_tc_kernel(const __grid_constant__ PrefillTcParams p, const __grid_constant__ CUtensorMap tm_q,
+    prefill_tc_kernel(const __grid_constant__ PrefillTcParams p,
                       const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ CUtensorMap tm_bv,
                       const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_av) {
   constexpr int TOK = kKRows / R;  // tokens per key tile
@@ -116,7 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (key_end + TOK - 1) / TOK;
 
   if (tid == 0) {
-    for (int s = 0; s < kNumBars; ++s) ptx::mbar_init(bar0 + 8 * s, bar0 + 8 * s == bar_w ? 4 : 1);  // W: one arrival per softmax warp
+    // W and the query: one arrival per softmax warp
+    for (int s = 0; s < kNumBars; ++s) ptx::mbar_init(bar0 + 8 * s, (bar0 + 8 * s == bar_w || bar0 + 8 * s == bar_q) ? 4 : 1);
     *s_abort = 0;
     ptx::fence_barrier_init();
   }
@@ -130,17 +134,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tbase = *s_taddr;
   const uint32_t t_s = tbase;          // S, later W hi (cols 0..63) and W lo (64..127)
   const uint32_t t_o = tbase + 128;    // O
+  const uint32_t t_q = tbase + 256;    // query hi (cols 256..319) and lo (320..383)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      ptx::prefetch_tmap(&tm_q);
       ptx::prefetch_tmap(&tm_bk);
       ptx::prefetch_tmap(&tm_bv);
-      const int qrow = (b * kH + i) * p.n_tokens + q0;
-      ptx::mbar_arrive_expect_tx(bar_q, kQBytes);
-      ptx::tma_load_2d(sbase, &tm_q, 0, qrow, bar_q);
-      ptx::tma_load_2d(sbase + kQBytes / 2, &tm_q, 64, qrow, bar_q);
       int issued = 0;
       for (int j = 0; j < nk; ++j) {
         const int st = j % kStages;
@@ -163,7 +163,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++issued;
       }
       // every issued load has landed before this CTA can finish
-      ptx::mbar_wait_bounded(bar_q, 0);
       for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
         ptx::mbar_wait_bounded(bar_full(j % kStages), (j / kStages) & 1);
     }
@@ -181,11 +180,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint32_t sb = sbase + kOffStages + st * kStageBytes;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {  // K = 128 features in steps of 16
-          const uint32_t koff = (k >> 2) * (kQBytes / 2) + (k & 3) * 32;
-          const uint64_t da = ptx::umma_desc_sw128(sbase + koff, 16, 1024);
-          const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBox + (k & 3) * 32, 16, 1024);
-          ptx::umma_ss(t_s, da, db, kIdescSS, k > 0 ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {  // query hi, then query lo
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {         // K = 128 features in steps of 16
+            const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBox + (k & 3) * 32, 16, 1024);
+            ptx::umma_ts(t_s, t_q + half * 64 + k * 8, db, kIdescSS, (half > 0 || k > 0) ? 1u : 0u);
+          }
         }
         ptx::umma_commit(bar_s);
         ok = ptx::mbar_wait_bounded(bar_w, j & 1);
@@ -218,6 +218,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int tq = q0 + row;                   // query index in the chunk
     const int qslot = P + tq;                  // its cache slot: keys s <= qslot
+    // stage this thread's query row as bf16 hi + lo into TMEM (zeros past the chunk)
+    {
+      const float* qr = p.q + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + i) * kD;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t hi[32], lo[32];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (tq < p.n_tokens) v = *reinterpret_cast<const float4*>(qr + c2 * 64 + 2 * e);
+          hi[e] = ptx::pack_bf16(v.x, v.y);
+          hi[e + 1] = ptx::pack_bf16(v.z, v.w);
+          lo[e] = ptx::pack_bf16(v.x - ptx::bf16_lo(hi[e]), v.y - ptx::bf16_hi(hi[e]));
+          lo[e + 1] = ptx::pack_bf16(v.z - ptx::bf16_lo(hi[e + 1]), v.w - ptx::bf16_hi(hi[e + 1]));
+        }
+        ptx::tmem_st32(t_q + lane_off + c2 * 32, hi);
+        ptx::tmem_st32(t_q + lane_off + 64 + c2 * 32, lo);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_q);
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
@@ -361,40 +384,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// Dense rotated queries in bf16, head-major: Q[b][i][t][:] =
-// bf16((1/R_Q) sum_j A_Q[b,t,j,i] RoPE(B_Q[b,t,j,:], pos_t)), angle in double, math in fp32.
-__global__ void __launch_bounds__(128) prefill_q_bf16_kernel(const __nv_bfloat16* __restrict__ a_q,
-                                                             const __nv_bfloat16* __restrict__ b_q,
-                                                             const int32_t* __restrict__ q_pos, int n_tokens,
-                                                             int r_q, __nv_bfloat16* __restrict__ q_out,
-                                                             const __grid_constant__ RopeTable rope) {
-  __shared__ float s_bq[8][kD];
-  __shared__ float s_aq[8][kH];
-  const int t = blockIdx.x, b = blockIdx.y;
-  const size_t tok = static_cast<size_t>(b) * n_tokens + t;
-  const int pos = q_pos[tok];
-  for (int e = threadIdx.x; e < r_q * (kD / 2); e += blockDim.x) {
-    const int j = e / (kD / 2), pr = e % (kD / 2);
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(b_q + (tok * r_q + j) * kD + 2 * pr);
-    float x = __bfloat162float(v.x), y = __bfloat162float(v.y);
-    float cs, sn;
-    rope_cos_sin(pos, rope.theta[pr], &cs, &sn);
-    rope_pair(x, y, cs, sn);
-    s_bq[j][2 * pr] = x;
-    s_bq[j][2 * pr + 1] = y;
-  }
-  for (int e = threadIdx.x; e < r_q * kH; e += blockDim.x)
-    s_aq[e / kH][e % kH] = __bfloat162float(a_q[tok * r_q * kH + e]);
-  __syncthreads();
-  const float inv = 1.f / static_cast<float>(r_q);
-  const int k = threadIdx.x;  // feature
-  for (int i = 0; i < kH; ++i) {
-    float acc = 0.f;
-    for (int j = 0; j < r_q; ++j) acc = fmaf(s_aq[j][i], s_bq[j][k], acc);
-    q_out[((static_cast<size_t>(b) * kH + i) * n_tokens + t) * kD + k] = __float2bfloat16_rn(acc * inv);
-  }
-}
-
 cudaError_t set_smem_once(int r) {
   static std::once_flag once[64][2];
   static cudaError_t status[64][2];
@@ -421,23 +410,30 @@ bool tensor_prefill_supported(int dtype, int heads, int head_dim, int r_k, int r
 }
 
 size_t tensor_prefill_workspace_bytes(int batch, int n_tokens, int heads, int head_dim) {
-  return round256(static_cast<size_t>(batch) * heads * n_tokens * head_dim * 2);
+  return round256(static_cast<size_t>(batch) * heads * n_tokens * head_dim * 4);  // fp32 rotated queries
 }
 
 cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t stream) {
   const CacheView& cv = a.cache;
   const int T = a.n_tokens;
-  __nv_bfloat16* qws = static_cast<__nv_bfloat16*>(a.workspace);
-  prefill_q_bf16_kernel<<<dim3(T, cv.batch), 128, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.a_q),
-                                                               static_cast<const __nv_bfloat16*>(a.b_q), a.q_pos, T,
-                                                               a.r_q, qws, a.rope);
-  cudaError_t e = cudaGetLastError();
+  float* qws = static_cast<float*>(a.workspace);
+  PrefillQArgs qa;
+  qa.batch = cv.batch;
+  qa.n_tokens = T;
+  qa.heads = cv.heads;
+  qa.head_dim = cv.head_dim;
+  qa.r_q = a.r_q;
+  qa.dtype = cv.dtype;
+  qa.a_q = a.a_q;
+  qa.b_q = a.b_q;
+  qa.q_pos = a.q_pos;
+  qa.q_out = qws;
+  qa.rope = a.rope;
+  cudaError_t e = launch_prefill_q(qa, stream);
   if (e != cudaSuccess) return e;
   const uint64_t rows_k = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_k;
   const uint64_t rows_v = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_v;
-  CUtensorMap tq, tbk, tbv, tak, tav;
-  if ((e = encode_bf16_2d(&tq, qws, kD, static_cast<uint64_t>(cv.batch) * kH * T, 64, kQ, 128)) != cudaSuccess)
-    return e;
+  CUtensorMap tbk, tbv, tak, tav;
   if ((e = encode_bf16_2d(&tbk, cv.b_k, kD, rows_k, 64, kKRows, 128)) != cudaSuccess) return e;
   if ((e = encode_bf16_2d(&tbv, cv.b_v, kD, rows_v, 64, kKRows, 128)) != cudaSuccess) return e;
   if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows_k, kH, kKRows, 64)) != cudaSuccess) return e;
@@ -451,11 +447,12 @@ cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t strea
   p.n_qtiles = (T + kQ - 1) / kQ;
   p.zs = a.scale * kLog2e / static_cast<float>(cv.r_k);
   p.inv_rv = 1.f / static_cast<float>(cv.r_v);
+  p.q = qws;
   p.out = a.out;
   p.err = a.err;
   dim3 grid(cv.batch * kH, p.n_qtiles);
   auto kern = cv.r_k == 1 ? prefill_tc_kernel<1> : prefill_tc_kernel<2>;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(p, tq, tbk, tbv, tak, tav);
+  kern<<<grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
   return cudaGetLastError();
 }
 

@@ -143,3 +143,15 @@ def test_tensor_kernel_partition_grids(grid, name):
     _check(w, cache, x, q, q_pos, out, end_to_end=False)
     assert torch.count_nonzero(out[2]) == 0
     assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("grid", [0, 5, 300])
+def test_workspace_contents_do_not_matter(kernel, grid):
+    """A workspace full of NaN (unwritten partial slots included) gives the same result."""
+    w = S.WORKLOADS["decode_b8_l8k"]
+    cache, x, q, q_pos = build_decode_cache(w, batch=4, length=600, lengths=[600, 1, 0, 333])
+    nbytes = T.tpa_decode_workspace_size(cache, 600, grid, kernel)
+    ws = torch.full((max(nbytes, 4) // 4,), float("nan"), dtype=torch.float32, device=DEV).view(torch.uint8)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=600, num_splits=grid, kernel=kernel, workspace_buf=ws)
+    _check(w, cache, x, q, q_pos, out, end_to_end=False)
