@@ -36,12 +36,17 @@ Readings of points the page leaves open (each is stated where it is used):
 * Causal prefill: the T queries of a chunk are the last T cache slots; query
   t (slot P + t, P = L - T) attends slots 0..P+t inclusive.
 * Outputs are float64 here; the CUDA library writes fp32.
+* The cache stores its factors in the storage dtype (bf16 or fp32), and B_K
+  is rotated before it is stored (append applies RoPE): the stored B~_K is
+  the rotated value rounded once to the storage dtype (round to nearest,
+  ties to even).  ``append_rope(..., storage=...)`` models that rounding.
 """
 from __future__ import annotations
 
 import numpy as np
 
 __all__ = [
+    "round_to_storage",
     "factor_elements_per_token",
     "dense_elements_per_token",
     "rope_frequencies",
@@ -67,6 +72,28 @@ def factor_elements_per_token(h: int, d_h: int, r_k: int, r_v: int) -> int:
 def dense_elements_per_token(h: int, d_h: int) -> int:
     """Numbers stored per token by a dense K/V cache: 2 h d_h (same section)."""
     return 2 * h * d_h
+
+
+def round_to_storage(x: np.ndarray, storage: str | None) -> np.ndarray:
+    """Round float64 values once to the storage dtype, ties to even.
+
+    ``"f32"``: IEEE binary32.  ``"bf16"``: 8 significant bits (binary32
+    exponent range), written out as m * 2^e with m rounded at 2^-8 relative
+    to the leading bit (np.rint rounds half to even); values below the
+    smallest normal use the subnormal spacing 2^-133.  ``None``: unchanged.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if storage is None:
+        return x
+    if storage == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if storage != "bf16":
+        raise ValueError(storage)
+    mant, expo = np.frexp(x)                     # x = mant * 2^expo, 0.5 <= |mant| < 1
+    normal = np.ldexp(np.rint(np.ldexp(mant, 8)), expo - 8)
+    tiny = np.ldexp(np.rint(np.ldexp(x, 133)), -133)
+    out = np.where(np.abs(x) >= 2.0 ** -126, normal, tiny)
+    return np.where(np.abs(out) > 3.3895313892515355e38, np.copysign(np.inf, x), out)
 
 
 def rope_frequencies(d_h: int, base: float) -> np.ndarray:
@@ -105,13 +132,15 @@ def tensor_product(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.einsum("...ri,...rk->...ik", a, b) / rank
 
 
-def append_rope(b_k: np.ndarray, positions: np.ndarray, base: float) -> np.ndarray:
+def append_rope(b_k: np.ndarray, positions: np.ndarray, base: float, storage: str | None = None) -> np.ndarray:
     """B~_K: every rank row of token s rotated at that token's position.
 
     b_k [..., S, R_K, d_h], positions [..., S].  RoPE acts on the B factor only
     (section RoPE 兼容性, Theorem 3.1); A_K, A_V and B_V are stored unchanged.
+    ``storage`` rounds the rotated rows once to the cache dtype, as the cache
+    keeps them.
     """
-    return rope(b_k, np.asarray(positions)[..., None], base)
+    return round_to_storage(rope(b_k, np.asarray(positions)[..., None], base), storage)
 
 
 def softmax_attention(z: np.ndarray, v: np.ndarray) -> np.ndarray:
@@ -163,9 +192,10 @@ def decode_attention(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block: int =
     return o
 
 
-def decode_attention_from_unrotated(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base):
-    """End-to-end decode: rotate B_K at each token's position, then attend."""
-    return decode_attention(a_k, append_rope(b_k, positions, base), a_v, b_v, q, q_pos, scale, base)
+def decode_attention_from_unrotated(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, storage=None):
+    """End-to-end decode: rotate B_K at each token's position (stored in the
+    cache dtype when ``storage`` is given), then attend."""
+    return decode_attention(a_k, append_rope(b_k, positions, base, storage), a_v, b_v, q, q_pos, scale, base)
 
 
 def prefill_queries(a_q, b_q, q_pos, base):

@@ -326,7 +326,30 @@ def pin_prefill_first_row(O):
     assert np.allclose(o[0], v0, rtol=0, atol=1e-13)
 
 
+def pin_storage_rounding(O):
+    """bf16 storage rounding: closed-form ties to even and PyTorch's float32 -> bfloat16 conversion."""
+    r = lambda v: float(O.round_to_storage(np.array([v]), "bf16")[0])
+    assert r(1.0 + 2.0 ** -8) == 1.0                    # exact tie, round to the even significand
+    assert r(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6    # exact tie, round up to even
+    assert r(1.0 + 2.0 ** -8 + 2.0 ** -30) == 1.0 + 2.0 ** -7
+    assert r(-(1.0 + 2.0 ** -9)) == -1.0
+    assert r(0.0) == 0.0 and r(2.0 ** -130) == 2.0 ** -130
+    g = np.random.default_rng(31)
+    x = (g.standard_normal(200000) * np.exp(g.uniform(-30, 30, 200000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(O.round_to_storage(x.astype(np.float64), "bf16"), ref)
+    f = O.round_to_storage(np.array([1.0 + 2.0 ** -30]), "f32")
+    assert f[0] == 1.0
+    # the stored rotated rows are bf16 values within half a bf16 ulp (2^-8 relative) of the rotation
+    b = g.standard_normal((5, 2, 8))
+    pos = np.arange(5)
+    st, ex = O.append_rope(b, pos, 100.0, "bf16"), O.append_rope(b, pos, 100.0)
+    assert np.array_equal(torch.from_numpy(st).to(torch.bfloat16).double().numpy(), st)
+    assert (np.abs(st - ex) <= 2.0 ** -8 * np.abs(ex) * (1 + 1e-12)).all()
+
+
 ALL_PINS = [
+    pin_storage_rounding,
     pin_cache_size,
     pin_rope_closed_form,
     pin_rope_complex,

@@ -41,7 +41,7 @@ def _check(w, cache, x, q, q_pos, out, batches=None, heads=None, end_to_end=True
             av = f64(x["a_v"][b, :L])[:, :, sel]
             r = O.decode_attention_from_unrotated(ak, f64(x["b_k"][b, :L]), av, f64(x["b_v"][b, :L]),
                                                   np.arange(L), f64(x["q"][b])[sel], float(x["q_pos"][b]),
-                                                  scale, w.rope_base)
+                                                  scale, w.rope_base, storage=w.dtype)
             assert_rows_close(got[n], r, tol, f"{w.name} end-to-end b={b}")
     return worst
 

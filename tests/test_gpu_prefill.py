@@ -37,8 +37,8 @@ def _oracle(w, cache, x, prior, tokens, b, rows=None, heads=None, end_to_end=Fal
     L = prior + tokens
     scale = default_scale(w.head_dim)
     sel = slice(None) if heads is None else list(heads)
-    if end_to_end:
-        bk = O.append_rope(f64(x["b_k"][b, :L]), np.arange(L), w.rope_base)
+    if end_to_end:   # the oracle's own RoPE, stored in the cache dtype as the append stores it
+        bk = O.append_rope(f64(x["b_k"][b, :L]), np.arange(L), w.rope_base, storage=w.dtype)
     else:
         bk = f64(cache.b_k[b, :L])
     ak = f64(cache.a_k[b, :L])[:, :, sel]

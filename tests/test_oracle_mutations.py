@@ -13,6 +13,7 @@ _tp = O.tensor_product
 _freq = O.rope_frequencies
 _decode = O.decode_attention
 _prefill_q = O.prefill_queries
+_round = O.round_to_storage
 
 
 def _rope_flipped(x, pos, base):              # wrong rotation sense
@@ -61,7 +62,26 @@ def _prefill_q_no_rope(a_q, b_q, q_pos, base):
     return _tp(a_q, b_q)
 
 
+def _round_truncate(x, storage):               # truncation instead of round-to-nearest-even
+    if storage != "bf16":
+        return _round(x, storage)
+    x = np.asarray(x, dtype=np.float64)
+    mant, expo = np.frexp(x)
+    return np.ldexp(np.trunc(np.ldexp(mant, 8)), expo - 8)
+
+
+def _round_ties_away(x, storage):              # ties away from zero instead of to even
+    if storage != "bf16":
+        return _round(x, storage)
+    x = np.asarray(x, dtype=np.float64)
+    mant, expo = np.frexp(x)
+    m = np.ldexp(mant, 8)
+    return np.ldexp(np.sign(m) * np.floor(np.abs(m) + 0.5), expo - 8)
+
+
 MUTANTS = {
+    "round_truncate": ("round_to_storage", _round_truncate),
+    "round_ties_away": ("round_to_storage", _round_ties_away),
     "rope_flipped": ("rope", _rope_flipped),
     "rope_rotate_half": ("rope", _rope_rotate_half),
     "freq_no_two": ("rope_frequencies", _freq_no_two),
