@@ -62,7 +62,7 @@ constexpr int kStageBytes = 2 * kBTile + 2 * kATile;
 constexpr int kOffStages = 0;
 constexpr int kOffAf = kOffStages + kStages * kStageBytes;  // fp32 A_K, A_V of the head: [2 stages][2][128]
 constexpr int kOffBar = kOffAf + kStages * 2 * kKRows * 4;
-constexpr int kNumBars = 2 * kStages + 5;  // full[2], empty[2], q_ready, s_full, w_ready, o_done, final
+constexpr int kNumBars = 2 * kStages + 6;  // full[2], empty[2], q_ready, s_full, w_ready, o_done, final, staged
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   const uint32_t bar_q = bar0 + 8 * (2 * kStages);
   const uint32_t bar_s = bar_q + 8, bar_w = bar_q + 16, bar_o = bar_q + 24, bar_fin = bar_q + 32;
+  const uint32_t bar_a = bar_q + 40;  // the four softmax warps have staged this tile's A_K, A_V
   volatile uint32_t* s_taddr = reinterpret_cast<volatile uint32_t*>(gbase + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
 
@@ -119,8 +120,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk = (key_end + TOK - 1) / TOK;
 
   if (tid == 0) {
-    // W and the query: one arrival per softmax warp
-    for (int s = 0; s < kNumBars; ++s) ptx::mbar_init(bar0 + 8 * s, (bar0 + 8 * s == bar_w || bar0 + 8 * s == bar_q) ? 4 : 1);
+    // W, the query and the staged head factors: one arrival per softmax warp
+    for (int s = 0; s < kNumBars; ++s) {
+      const uint32_t bar = bar0 + 8 * s;
+      ptx::mbar_init(bar, (bar == bar_w || bar == bar_q || bar == bar_a) ? 4 : 1);
+    }
     *s_abort = 0;
     ptx::fence_barrier_init();
   }
@@ -271,10 +275,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::fence_proxy_async_smem();
       }
-      // all four softmax warps leave together if any of them timed out
-      if (ptx::named_barrier_or(1, 128, fail)) {
-        if (fail) atomicOr(p.err, kErrTimeout);
+      // rendezvous of the four softmax warps (a bounded wait): the staged A_K, A_V of this tile
+      // are visible afterwards; a warp that timed out raises the abort flag before arriving
+      if (fail) {
+        atomicOr(p.err, kErrTimeout);
         *s_abort = 1;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_a);
+      if (!ptx::mbar_wait_bounded(bar_a, j & 1)) {
+        atomicOr(p.err, kErrTimeout);
+        *s_abort = 1;
+      }
+      if (__any_sync(0xffffffffu, *s_abort != 0)) {
         ok = false;
         break;
       }
@@ -307,23 +320,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mx = fmaxf(mx, z[s]);
       }
-      // ---- online softmax with a lazily rescaled maximum
-      if (mx > m + 8.f || (m == -INFINITY && mx != -INFINITY)) {
-        const float m_new = mx;
-        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+      // ---- online softmax with a lazily rescaled maximum; the TMEM rescale of O is a
+      // warp-wide operation, so the whole warp runs it when any of its rows needs it
+      const bool grow = mx > m + 8.f || (m == -INFINITY && mx != -INFINITY);
+      const float alpha = !grow ? 1.f : (m == -INFINITY ? 0.f : exp2f(m - mx));
+      if (grow) {
         l *= alpha;
-        if (j > 0) {
+        m = mx;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            uint32_t ov[32];
-            ptx::tmem_ld32(t_o + lane_off + c4 * 32, ov);
-            ptx::tmem_wait_ld();
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t ov[32];
+          ptx::tmem_ld32(t_o + lane_off + c4 * 32, ov);
+          ptx::tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            ptx::tmem_st32(t_o + lane_off + c4 * 32, ov);
-          }
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          ptx::tmem_st32(t_o + lane_off + c4 * 32, ov);
         }
-        m = m_new;
       }
       // ---- W = p A_V / R_V as bf16 hi + lo, packed two rows per TMEM column
 #pragma unroll
@@ -353,7 +367,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ptx::mbar_arrive(bar_w);
     }
     // ---- epilogue: O / l to out[b][t][i][:]
-    if (ok && ptx::mbar_wait_bounded(bar_o, (nk - 1) & 1)) {
+    const bool o_ready = ok && ptx::mbar_wait_bounded(bar_o, (nk - 1) & 1);
+    if (__all_sync(0xffffffffu, o_ready)) {  // the TMEM loads below are warp-wide
       ptx::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       float* op = p.out + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + i) * kD;

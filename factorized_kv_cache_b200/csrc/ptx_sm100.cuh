@@ -107,12 +107,15 @@ __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v 
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
 // ---------------------------------------------------------------- named barrier, PDL
+// bar.sync is warp-aligned: reconverge the warp first.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
+  __syncwarp();
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // Named barrier that also ORs a predicate over the participating threads.
 __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t threads, bool pred) {
+  __syncwarp();
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"

@@ -58,6 +58,7 @@ class DecodeWorkload:
     seed: int
     min_length: int = 0    # >0: lengths drawn uniformly from [min_length, length]
     rope_base: float = 10000.0
+    b_std: float = 0.0     # std of the B factors; 0 means 1/sqrt(d_h)
 
     @property
     def capacity(self) -> int:
@@ -145,9 +146,10 @@ def decode_inputs(w: DecodeWorkload, batch: int | None = None, length: int | Non
     else:
         lengths = np.full(B, cap, dtype=np.int32)
     a_k = _normal(g, (B, cap, rk, h), 1.0)
-    b_k = _normal(g, (B, cap, rk, d), 1.0 / np.sqrt(d))
+    b_std = w.b_std if w.b_std > 0 else 1.0 / np.sqrt(d)
+    b_k = _normal(g, (B, cap, rk, d), b_std)
     a_v = _normal(g, (B, cap, rv, h), 1.0)
-    b_v = _normal(g, (B, cap, rv, d), 1.0 / np.sqrt(d))
+    b_v = _normal(g, (B, cap, rv, d), b_std)
     q = _normal(g, (B, h, d), 1.0)
     positions = np.broadcast_to(np.arange(cap, dtype=np.int32), (B, cap)).copy()
     return {

@@ -155,3 +155,14 @@ def test_workspace_contents_do_not_matter(kernel, grid):
     ws = torch.full((max(nbytes, 4) // 4,), float("nan"), dtype=torch.float32, device=DEV).view(torch.uint8)
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=600, num_splits=grid, kernel=kernel, workspace_buf=ws)
     _check(w, cache, x, q, q_pos, out, end_to_end=False)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("rank", [1, 2])
+def test_unit_variance_factors(kernel, rank):
+    """B factors ~ N(0, 1) (the prefill workload's scale): scores ~10x larger than the decode
+    workloads'.  A single bf16 rounding of the rotated query would exceed 2e-3 here."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="unit_var", r_k=rank, r_v=rank, b_std=1.0, seed=77)
+    cache, x, q, q_pos = build_decode_cache(w, batch=3, length=4000, min_length=1000)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=4000, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out)
