@@ -388,37 +388,15 @@ def add_cpu_baseline(res, x, w, lengths, target_s):
 
 def run_reference_prefill(args, w):
     """Reference arm for the prefill workload: the float64 oracle on sampled query rows."""
-    from factorized_kv_cache_b200 import synthetic as S
-    x = S.prefill_inputs(w)
-    host = {k: x[k].float().numpy() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v")}
     workers = max(1, min(os.cpu_count() or 1, 16))
     K, W = args.steps, args.warmup
     budget = 150.0 / max(1, K + W)
-    g = np.random.default_rng(0)
-    scale = 1.0 / math.sqrt(w.head_dim)
     rows_per_task = 8
-
-    def tasks(n):
-        return [(host["a_k"][t % w.batch], host["b_k"][t % w.batch], host["a_v"][t % w.batch],
-                 host["b_v"][t % w.batch], host["a_q"][t % w.batch], host["b_q"][t % w.batch],
-                 np.sort(g.integers(0, w.tokens, rows_per_task)), scale, w.rope_base) for t in range(n)]
-
-    t0 = time.perf_counter()
-    _prefill_oracle_task(tasks(1)[0])
-    per_task = time.perf_counter() - t0
-    tasks_per_step = max(1, min(workers, int(budget * workers / max(per_task, 1e-6))))
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(workers) as pool:
-        for _ in range(W):
-            pool.map(_prefill_oracle_task, tasks(tasks_per_step))
-        t0 = time.perf_counter()
-        done = 0
-        for _ in range(K):
-            done += sum(pool.map(_prefill_oracle_task, tasks(tasks_per_step)))
-        dt = time.perf_counter() - t0
+    n_fn = lambda per_task: max(1, min(workers, int(budget * workers / max(per_task, 1e-6))))
+    done, dt, n = _prefill_rate(w, workers, n_fn, rows_per_task, steps=K, warm_steps=W)
     value = done / dt
-    sample = (f"each step: {tasks_per_step} oracle prefills of {rows_per_task} random query rows (all heads, full "
-              f"causal prefix) of {w.name}, float64 oracle on {workers} spawned processes")
+    sample = (f"each step: {n} oracle prefills of {rows_per_task} random query rows of sequence 0 (all heads, "
+              f"full causal prefix) of {w.name}, float64 oracle on {workers} spawned processes")
     return {
         "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "tokens/s", "n_gpus": 1, "steps": K,
         "warmup": W, "ms_per_step": dt / max(1, K) * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -473,16 +451,49 @@ def run_reference(args, w):
 PREFILL_METRIC = "causal prefill query tokens/sec (TPA, R_Q-factorized queries) + tensor TFLOP/s vs peak, 1×B200"
 
 
-def _prefill_oracle_task(args):
-    """Oracle prefill of a few query rows of one sequence (runs in a spawned worker)."""
+_PF = {}
+
+
+def _prefill_worker_init(w):
+    """Spawned worker: regenerate sequence 0 of the prefill workload from its seed.
+
+    The hidden states and projections come from fixed Philox streams, so
+    batch=1 reproduces sequence 0 of the full batch exactly."""
+    from factorized_kv_cache_b200 import synthetic as S
+    x = S.prefill_inputs(w, batch=1)
+    _PF.update({k: x[k][0].double().numpy() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v")})
+    _PF["w"] = w
+
+
+def _prefill_oracle_task(rows):
+    """Oracle prefill of some query rows of sequence 0 (all heads, full causal prefix, RoPE)."""
     import oracle.tpa_oracle as O
-    a_k, b_k, a_v, b_v, a_q, b_q, rows, scale, base = args
-    f = lambda a: np.asarray(a, dtype=np.float64)
-    L = a_k.shape[0]
+    w = _PF["w"]
+    L = _PF["a_k"].shape[0]
     pos = np.arange(L)
-    O.prefill_attention(f(a_k), O.append_rope(f(b_k), pos, base), f(a_v), f(b_v), f(a_q), f(b_q), pos, scale, base,
-                        rows=rows)
+    O.prefill_attention(_PF["a_k"], O.append_rope(_PF["b_k"], pos, w.rope_base, "bf16"), _PF["a_v"], _PF["b_v"],
+                        _PF["a_q"], _PF["b_q"], pos, 1.0 / math.sqrt(w.head_dim), w.rope_base, rows=rows)
     return len(rows)
+
+
+def _prefill_rate(w, workers, n_tasks_fn, rows_per_task, steps=1, warm_steps=0):
+    """Run oracle prefill tasks on a spawned pool; returns (rows done, seconds, tasks per step)."""
+    g = np.random.default_rng(0)
+    draw = lambda n: [np.sort(g.integers(0, w.tokens, rows_per_task)) for _ in range(n)]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers, initializer=_prefill_worker_init, initargs=(w,)) as pool:
+        t0 = time.perf_counter()
+        pool.map(_prefill_oracle_task, draw(workers), chunksize=1)      # calibration, one task per worker
+        per_task = (time.perf_counter() - t0)
+        n = n_tasks_fn(per_task)
+        for _ in range(warm_steps):
+            pool.map(_prefill_oracle_task, draw(n), chunksize=1)
+        done = 0
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            done += sum(pool.map(_prefill_oracle_task, draw(n), chunksize=1))
+        dt = time.perf_counter() - t0
+    return done, dt, n
 
 
 def run_ours_prefill(args, w, rank, world, dev):
@@ -612,36 +623,14 @@ def run_ours_prefill(args, w, rank, world, dev):
 
 
 def add_prefill_cpu_baseline(res, x, w, target_s):
-    host = {k: x[k].float().numpy() for k in ("a_q", "b_q", "a_k", "b_k", "a_v", "b_v")}
     workers = max(1, min(os.cpu_count() or 1, 16))
     rows_per_task = 16
-    g = np.random.default_rng(0)
-    scale = 1.0 / math.sqrt(w.head_dim)
-
-    def tasks(n):
-        out = []
-        for t in range(n):
-            b = t % w.batch
-            rows = np.sort(g.integers(0, w.tokens, rows_per_task))
-            out.append((host["a_k"][b], host["b_k"][b], host["a_v"][b], host["b_v"][b], host["a_q"][b],
-                        host["b_q"][b], rows, scale, w.rope_base))
-        return out
-
-    t0 = time.perf_counter()
-    _prefill_oracle_task(tasks(1)[0])
-    per_task = time.perf_counter() - t0
-    n = max(workers, int(target_s * workers / max(per_task, 1e-6)))
-    n = (n + workers - 1) // workers * workers
-    ctx = mp.get_context("spawn")
-    with ctx.Pool(workers) as pool:
-        tl = tasks(n)
-        t0 = time.perf_counter()
-        done = sum(pool.map(_prefill_oracle_task, tl, chunksize=1))
-        dt = time.perf_counter() - t0
+    n_fn = lambda per_task: max(workers, int(target_s * workers / max(per_task, 1e-6)) // workers * workers)
+    done, dt, n = _prefill_rate(w, workers, n_fn, rows_per_task)
     res["cpu_baseline"] = {"value": done / dt, "unit": "tokens/s", "cores": workers, "kind": "oracle",
-                           "sample": f"{n} oracle prefills of {rows_per_task} random query rows (all heads, full "
-                                     f"causal prefix, RoPE included) of {w.name}; {dt:.1f} s on {workers} "
-                                     f"spawned processes"}
+                           "sample": f"{n} oracle prefills of {rows_per_task} random query rows of sequence 0 "
+                                     f"(all heads, full causal prefix, RoPE included) of {w.name}; {dt:.1f} s on "
+                                     f"{workers} spawned processes"}
 
 
 def main():
