@@ -62,7 +62,7 @@ constexpr int kStageBytes = 2 * kBTile + 2 * kATile;
 constexpr int kOffStages = 0;
 constexpr int kOffAf = kOffStages + kStages * kStageBytes;  // fp32 A_K, A_V of the head: [2 stages][2][128]
 constexpr int kOffBar = kOffAf + kStages * 2 * kKRows * 4;
-constexpr int kNumBars = 2 * kStages + 6;  // full[2], empty[2], q_ready, s_full, w_ready, o_done, final, staged
+constexpr int kNumBars = 2 * kStages + 7;  // full[2], empty[2], q_ready, s_full[2], w_ready, o_done, final, staged
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -98,8 +98,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar_full = [&](int s) { return bar0 + 8 * s; };
   auto bar_empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   const uint32_t bar_q = bar0 + 8 * (2 * kStages);
-  const uint32_t bar_s = bar_q + 8, bar_w = bar_q + 16, bar_o = bar_q + 24, bar_fin = bar_q + 32;
-  const uint32_t bar_a = bar_q + 40;  // the four softmax warps have staged this tile's A_K, A_V
+  auto bar_s = [&](int buf) { return bar_q + 8 + 8 * buf; };  // S buffer `buf` holds a tile's scores
+  const uint32_t bar_w = bar_q + 24, bar_o = bar_q + 32, bar_fin = bar_q + 40;
+  const uint32_t bar_a = bar_q + 48;  // the four softmax warps have staged this tile's A_K, A_V
   volatile uint32_t* s_taddr = reinterpret_cast<volatile uint32_t*>(gbase + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
 
@@ -136,9 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tbase = *s_taddr;
-  const uint32_t t_s = tbase;          // S, later W hi (cols 0..63) and W lo (64..127)
-  const uint32_t t_o = tbase + 128;    // O
-  const uint32_t t_q = tbase + 256;    // query hi (cols 256..319) and lo (320..383)
+  // S of tile j in columns [128 (j % 2), +128): scores, then W hi (first 64) and W lo (next 64)
+  auto t_s = [&](int j) { return tbase + 128u * static_cast<uint32_t>(j & 1); };
+  const uint32_t t_o = tbase + 256;    // O
+  const uint32_t t_q = tbase + 384;    // query hi (cols 384..447) and lo (448..511)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -172,40 +174,50 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Order: S(0); then for each tile j: S(j+1) into the other buffer (after the value MMA
+    // of tile j-1 has consumed the W stored there), then O += W(j) B_V once the softmax of
+    // tile j is done.  The score MMA of tile j+1 thus runs while the softmax works on tile j.
     if (lane == 0) {
-      bool ok = ptx::mbar_wait_bounded(bar_q, 0);
-      for (int j = 0; j < nk && ok; ++j) {
-        const int st = j % kStages;
-        if (*s_abort) break;
-        ok = ptx::mbar_wait_bounded(bar_full(st), (j / kStages) & 1);
-        // the previous value MMA must be done reading W (which lives where S goes) and writing O
-        if (ok && j > 0) ok = ptx::mbar_wait_bounded(bar_o, (j - 1) & 1);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        const uint32_t sb = sbase + kOffStages + st * kStageBytes;
+      auto scores = [&](int j) {
+        const uint32_t sb = sbase + kOffStages + (j % kStages) * kStageBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {  // query hi, then query lo
 #pragma unroll
           for (int k = 0; k < 8; ++k) {         // K = 128 features in steps of 16
             const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBox + (k & 3) * 32, 16, 1024);
-            ptx::umma_ts(t_s, t_q + half * 64 + k * 8, db, kIdescSS, (half > 0 || k > 0) ? 1u : 0u);
+            ptx::umma_ts(t_s(j), t_q + half * 64 + k * 8, db, kIdescSS, (half > 0 || k > 0) ? 1u : 0u);
           }
         }
-        ptx::umma_commit(bar_s);
+        ptx::umma_commit(bar_s(j & 1));
+      };
+      bool ok = ptx::mbar_wait_bounded(bar_q, 0) && ptx::mbar_wait_bounded(bar_full(0), 0);
+      if (ok) {
+        ptx::tc_fence_after();
+        scores(0);
+      }
+      for (int j = 0; j < nk && ok; ++j) {
+        if (*s_abort) break;
+        if (j + 1 < nk) {
+          ok = ptx::mbar_wait_bounded(bar_full((j + 1) % kStages), ((j + 1) / kStages) & 1);
+          if (ok && j > 0) ok = ptx::mbar_wait_bounded(bar_o, (j - 1) & 1);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          scores(j + 1);
+        }
         ok = ptx::mbar_wait_bounded(bar_w, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t bv = sb + kBTile;
+        const uint32_t bv = sbase + kOffStages + (j % kStages) * kStageBytes + kBTile;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {    // W hi, then W lo
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {        // K = 128 cache rows in steps of 16
             const uint64_t db = ptx::umma_desc_sw128(bv + kk * 2048, kBox, 1024);
-            ptx::umma_ts(t_o, t_s + half * 64 + kk * 8, db, kIdescTS, (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
+            ptx::umma_ts(t_o, t_s(j) + half * 64 + kk * 8, db, kIdescTS, (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
           }
         }
         ptx::umma_commit(bar_o);
-        ptx::umma_commit(bar_empty(st));
+        ptx::umma_commit(bar_empty(j % kStages));
       }
       if (!ok) {
         atomicOr(p.err, kErrTimeout);
@@ -250,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nk; ++j) {
       const int st = j % kStages;
       bool fail = *s_abort != 0;
-      if (!fail) fail = !ptx::mbar_wait_bounded(bar_full(st), (j / kStages) & 1) || !ptx::mbar_wait_bounded(bar_s, j & 1);
+      if (!fail) fail = !ptx::mbar_wait_bounded(bar_full(st), (j / kStages) & 1) || !ptx::mbar_wait_bounded(bar_s(j & 1), (j >> 1) & 1);
       ptx::tc_fence_after();
       const uint8_t* sb = gbase + kOffStages + st * kStageBytes;
       const int tok0 = j * TOK;
@@ -299,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t sv[32];
-        ptx::tmem_ld32(t_s + lane_off + c4 * 32, sv);
+        ptx::tmem_ld32(t_s(j) + lane_off + c4 * 32, sv);
         ptx::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32 / R; ++e) {
@@ -329,6 +341,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mx;
       }
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        // the value MMA of tile j-1 may still be accumulating into O
+        const bool o_prev = ptx::mbar_wait_bounded(bar_o, (j - 1) & 1);
+        if (!__all_sync(0xffffffffu, o_prev)) {
+          atomicOr(p.err, kErrTimeout);
+          *s_abort = 1;
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           uint32_t ov[32];
@@ -358,8 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           whi[e] = ptx::pack_bf16(w2[0], w2[1]);
           wlo[e] = ptx::pack_bf16(w2[0] - ptx::bf16_lo(whi[e]), w2[1] - ptx::bf16_hi(whi[e]));
         }
-        ptx::tmem_st32(t_s + lane_off + c2 * 32, whi);
-        ptx::tmem_st32(t_s + lane_off + 64 + c2 * 32, wlo);
+        ptx::tmem_st32(t_s(j) + lane_off + c2 * 32, whi);
+        ptx::tmem_st32(t_s(j) + lane_off + 64 + c2 * 32, wlo);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
