@@ -25,16 +25,17 @@
 // {B_K, B_V, A_K, A_V} tiles of 128 cache rows); warp 1 allocates 512 TMEM
 // columns and one of its threads issues the MMAs; warps 2-5 (one TMEM lane =
 // one query row per thread) stage the query and run the softmax.
-// Per key tile: S = (Q_hi + Q_lo) B_K^T (M = 128 queries, N = 128 rows,
-// K = 128; A from TMEM columns [256, 384)) into TMEM columns [0, 128); the
-// softmax reads S, applies A_K, the causal mask
+// Per key tile j: S = (Q_hi + Q_lo) B_K^T (M = 128 queries, N = 128 rows,
+// K = 128; A from TMEM columns [384, 512)) into TMEM columns
+// [128 (j % 2), +128), so the score MMA of tile j + 1 runs while the softmax
+// works on tile j; the softmax reads S, applies A_K, the causal mask
 // and the online softmax, rescales O in TMEM when the running maximum grows
-// by more than 2^8, and writes W as bf16 hi and lo halves into TMEM columns
-// [0, 64) and [64, 128) (over S); then O += W_hi B_V + W_lo B_V (A from TMEM,
-// B_V as an MN-major operand) into columns [128, 256).  Both the query and W
-// are split into two bf16 parts, which keeps them to ~16 bits: one bf16
-// rounding of either costs ~3.5e-3 relative error on the prefill workload,
-// above its 2e-3 budget.
+// by more than 2^8, and writes W as bf16 hi and lo halves into the first and
+// second 64 columns of the same buffer (over S); then O += W_hi B_V + W_lo B_V
+// (A from TMEM, B_V as an MN-major operand) into columns [256, 384).  Both the
+// query and W are split into two bf16 parts, which keeps them to ~16 bits: one
+// bf16 rounding of either costs ~3.5e-3 relative error on the prefill
+// workload, above its 2e-3 budget.
 #include <cuda.h>
 #include <math.h>
 
@@ -387,8 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar_w);
     }
-    // ---- epilogue: O / l to out[b][t][i][:]
-    const bool o_ready = ok && ptx::mbar_wait_bounded(bar_o, (nk - 1) & 1);
+    // ---- epilogue: O / l to out[b][t][i][:].  It waits on the issuer's final commit, not on
+    // the parity of the value barrier: with two score buffers that barrier can still be two
+    // phases behind here, where its parity alone cannot tell the last phase from an earlier one.
+    const bool o_ready = ok && ptx::mbar_wait_bounded(bar_fin, 0);
     if (__all_sync(0xffffffffu, o_ready)) {  // the TMEM loads below are warp-wide
       ptx::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
