@@ -192,7 +192,8 @@ def run_ours_decode(args, w, rank, world, dev):
     from factorized_kv_cache_b200 import synthetic as S
     from factorized_kv_cache_b200 import tpa as T
 
-    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR}[args.kernel]
+    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR,
+              "tensor_sync": T.TPA_KERNEL_TENSOR_SYNC}[args.kernel]
     dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
     esize = 4 if w.dtype == "f32" else 2
     x = decode_host_inputs(w, rank)
@@ -328,8 +329,12 @@ def run_ours_decode(args, w, rank, world, dev):
     mean_decode_s = statistics.mean(decode_ms) / 1e3
     peaks, kind = measured_peaks()
     achieved = bytes_per_decode / mean_decode_s / 1e9
-    kernel_src = ["factorized_kv_cache_b200/csrc/attention_simt.cu"] if (
-        kernel == T.TPA_KERNEL_SIMT or w.dtype == "f32") else ["factorized_kv_cache_b200/csrc/decode_tensor.cu"]
+    if kernel == T.TPA_KERNEL_SIMT or w.dtype == "f32":
+        kernel_src = ["factorized_kv_cache_b200/csrc/attention_simt.cu"]
+    elif kernel == T.TPA_KERNEL_TENSOR_SYNC:
+        kernel_src = ["factorized_kv_cache_b200/csrc/decode_tensor.cu"]
+    else:
+        kernel_src = ["factorized_kv_cache_b200/csrc/decode_umma.cu"]
     kernel_src = [p for p in kernel_src if os.path.exists(os.path.join(ROOT, p))]
     res = {
         "metric": METRIC,
@@ -502,7 +507,8 @@ def run_ours_prefill(args, w, rank, world, dev):
     from factorized_kv_cache_b200 import synthetic as S
     from factorized_kv_cache_b200 import tpa as T
 
-    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR}[args.kernel]
+    kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR,
+              "tensor_sync": T.TPA_KERNEL_TENSOR_SYNC}[args.kernel]
     ww = w.replace(seed=w.seed + 1000 * rank) if rank else w
     x = S.prefill_inputs(ww)
     B, Tn = w.batch, w.tokens
@@ -642,7 +648,7 @@ def main():
     ap.add_argument("--workload", default="decode_b8_l8k",
                     choices=["decode_tiny_f32", "decode_b8_l8k", "decode_b32_var32k", "prefill_b4_t4k",
                              "decode_long_512k"])
-    ap.add_argument("--kernel", choices=["auto", "simt", "tensor"], default="auto")
+    ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "tensor_sync"], default="auto")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")

@@ -40,6 +40,7 @@
 
 #include <mutex>
 
+#include "decode_common.cuh"
 #include "device_common.cuh"
 #include "ptx_sm100.cuh"
 #include "tma_host.h"
@@ -49,8 +50,12 @@
 namespace tpa {
 namespace {
 
-constexpr int kH = 32;
-constexpr int kD = 128;
+using dec::DecodeTcParams;
+using dec::kD;
+using dec::kH;
+using dec::kMaxBatch;
+using dec::owner_of;
+
 constexpr int kRows = 64;                          // cache-plane rows per tile
 constexpr int kStages = 2;
 constexpr int kConsumerWarps = 4;
@@ -59,7 +64,6 @@ constexpr int kBoxBytes = kRows * 128;             // 64 features x kRows rows, 
 constexpr int kBBytes = 2 * kBoxBytes;             // one B tile (128 features)
 constexpr int kABytes = kRows * kH * 2;            // one A tile
 constexpr int kStageBytes = 2 * kBBytes + 2 * kABytes;
-constexpr int kMaxBatch = 1024;
 // Per-segment scratch: the rotated query as bf16 high and low parts
 // ([2][32][128], 16 KB, swizzled for ldmatrix) while tiles are processed,
 // then the row-half merge buffers (O[2][16][128] and (m, l)[2][16]) at the
@@ -70,62 +74,6 @@ constexpr size_t kSmemBytes = 1024 + size_t(kStages) * kStageBytes + kMergeFloat
 static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
 static_assert(2 * kH * kD * 2 <= 2 * 16 * kD * 4, "query hi + lo fit in the merge buffer");
 constexpr unsigned kErrTimeout = 0x8u;
-
-struct DecodeTcParams {
-  const int32_t* seq_lens;
-  const __nv_bfloat16* q;
-  const int32_t* q_pos;
-  int batch, capacity, max_len, grid;
-  float zs;                // scale * log2(e) / R_K
-  float* out;              // [B][32][128]
-  int32_t* ws_prefix;      // [B + 1]
-  float* ws_ml;            // [2G][32][2]
-  float* ws_o;             // [2G][32][128]
-  unsigned int* err;
-  RopeTable rope;
-};
-
-__device__ __forceinline__ int owner_of(int t, int nt, int grid) {
-  return static_cast<int>((static_cast<long long>(t) * grid) / nt);
-}
-
-// Exclusive prefix of per-sequence tile counts into s_pref[0..B], lengths into s_len.
-template <int TOK>
-__device__ void build_prefix(const DecodeTcParams& p, int32_t* s_pref, int32_t* s_len, int32_t* s_tmp) {
-  const int B = p.batch;
-  const int tid = threadIdx.x;
-  const int per = (B + kThreads - 1) / kThreads;
-  const int b0 = tid * per;
-  int local = 0;
-  for (int b = b0; b < min(B, b0 + per); ++b) {
-    int L = p.seq_lens[b];
-    if (L < 0 || L > p.capacity || L > p.max_len) {
-      if (blockIdx.x == 0) atomicOr(p.err, TPA_DEVERR_LEN_RANGE);
-      L = min(max(L, 0), min(p.capacity, p.max_len));
-    }
-    s_len[b] = L;
-    local += (L + TOK - 1) / TOK;
-  }
-  // inclusive scan of `local` over the CTA
-  const int lane = tid & 31, warp = tid >> 5;
-  int incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) s_tmp[warp] = incl;
-  __syncthreads();
-  int warp_off = 0;
-  for (int w = 0; w < warp; ++w) warp_off += s_tmp[w];
-  int run = warp_off + incl - local;
-  for (int b = b0; b < min(B, b0 + per); ++b) {
-    s_pref[b] = run;
-    run += (s_len[b] + TOK - 1) / TOK;
-  }
-  if (tid == kThreads - 1) s_pref[B] = warp_off + incl;
-  __syncthreads();
-}
 
 template <int R>
 __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition: two CTAs per SM
@@ -162,27 +110,18 @@ __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition
     *s_abort = 0;
     ptx::fence_barrier_init();
   }
-  build_prefix<TOK>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
+  dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
   const int B = p.batch;
   const int NT = s_pref[B];
   if (blockIdx.x == 0)
     for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
   if (NT == 0) return;
   const int c = blockIdx.x;
-  const int t_begin = static_cast<int>((static_cast<long long>(c) * NT + p.grid - 1) / p.grid);
-  const int t_end = static_cast<int>((static_cast<long long>(c + 1) * NT + p.grid - 1) / p.grid);
+  const int t_begin = dec::first_tile(c, NT, p.grid);
+  const int t_end = dec::first_tile(c + 1, NT, p.grid);
   if (t_begin >= t_end) return;
   // first sequence with tiles in [t_begin, ...): largest b with s_pref[b] <= t_begin and s_pref[b+1] > t_begin
-  int b_first = 0;
-  {
-    int lo = 0, hi = B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (s_pref[mid] <= t_begin) lo = mid; else hi = mid - 1;
-    }
-    b_first = lo;
-    while (b_first < B && s_pref[b_first + 1] <= t_begin) ++b_first;
-  }
+  const int b_first = dec::sequence_of_tile(s_pref, B, t_begin);
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -247,7 +186,7 @@ __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition
     {
       // q~ = hi + lo, each as bf16 rows of 256 B with 16-byte chunks XOR-swizzled by (row & 7)
       // within each 128-byte half; the lo plane follows the hi plane (8 KB)
-      const __nv_bfloat16* qb = p.q + static_cast<size_t>(b) * kH * kD;
+      const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(p.q) + static_cast<size_t>(b) * kH * kD;
       uint8_t* sq = gbase + kStages * kStageBytes;
       for (int e = tid; e < kH * kD / 2; e += kConsumerWarps * 32) {
         const int head = e / (kD / 2), j = e % (kD / 2);  // RoPE pair j = features (2j, 2j+1)
@@ -539,8 +478,10 @@ __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition
 // (sequence, head).  The touched CTAs of sequence b are cs..ce; when every CTA
 // owns at least one tile (G <= NT) they all touched b, b is the first sequence
 // of each of them but possibly cs, and only cs needs a division.  The (m, l)
-// pairs are reduced across the CTA; the features are then summed with every
-// partial's float4 loads in flight at once (4 partial groups x 32 float4).
+// pairs are reduced across the CTA; the features are then summed by eight
+// partial groups of 32 threads (one float4 column per thread), each thread
+// with kMergeBatch partial loads in flight at once, so even the ~150 partials
+// of a single long sequence take only a few L2 round trips.
 struct TcMergeParams {
   int batch, grid;
   const int32_t* prefix;
@@ -549,7 +490,9 @@ struct TcMergeParams {
   float* out;
 };
 
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeGroups = kMergeThreads / 32;
+constexpr int kMergeBatch = 4;
 constexpr int kMergeMax = 1024;  // partials per pass
 
 __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red) {
@@ -567,34 +510,30 @@ __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red
   return v;
 }
 
-__device__ __forceinline__ int ceil_tile(int c, int nt, int grid) {
-  return static_cast<int>((static_cast<long long>(c) * nt + grid - 1) / grid);
-}
-
 __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __grid_constant__ TcMergeParams p) {
   ptx::pdl_wait();
   __shared__ float s_w[kMergeMax];
   __shared__ int s_slot[kMergeMax];
   __shared__ float s_red[kMergeThreads / 32];
-  __shared__ float4 s_acc[4][32];
+  __shared__ float4 s_acc[kMergeGroups][32];
   const int b = blockIdx.x, i = blockIdx.y, tid = threadIdx.x;
   const int NT = p.prefix[p.batch];
   const int t0 = p.prefix[b], t1 = p.prefix[b + 1];
   float* o = p.out + (static_cast<size_t>(b) * kH + i) * kD;
   if (t1 <= t0) {
-    o[tid] = 0.f;
+    if (tid < kD) o[tid] = 0.f;
     return;
   }
   const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
   if (cs == ce) return;  // written by the decode kernel
   const int n = ce - cs + 1;
   const bool dense = p.grid <= NT;
-  const bool cs_first = ceil_tile(cs, NT, p.grid) >= t0;
+  const bool cs_first = dec::first_tile(cs, NT, p.grid) >= t0;
   // slot (in units of [slot][head]) of CTA cs + u for this sequence, -1 if it did not touch it
   auto slot_of = [&](int u) -> int {
     const int cc = cs + u;
     if (dense) return (2 * cc + ((u > 0 || cs_first) ? 0 : 1)) * kH + i;
-    const int a = ceil_tile(cc, NT, p.grid), e = ceil_tile(cc + 1, NT, p.grid);
+    const int a = dec::first_tile(cc, NT, p.grid), e = dec::first_tile(cc + 1, NT, p.grid);
     if (!(a < e && a < t1 && e > t0)) return -1;
     return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
   };
@@ -622,15 +561,24 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       s_slot[u] = sl;
     }
     L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
-    for (int u = grp; u < cn; u += 4) {
-      const int sl = s_slot[u];
-      if (sl < 0) continue;  // never read a partial this sequence did not write
-      const float w = s_w[u];
-      const float4 v = reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4];
-      acc.x = fmaf(v.x, w, acc.x);
-      acc.y = fmaf(v.y, w, acc.y);
-      acc.z = fmaf(v.z, w, acc.z);
-      acc.w = fmaf(v.w, w, acc.w);
+    for (int u0 = grp; u0 < cn; u0 += kMergeGroups * kMergeBatch) {
+      float4 v[kMergeBatch];
+      float wv[kMergeBatch];
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        const int u = u0 + kMergeGroups * k;
+        const int sl = u < cn ? s_slot[u] : -1;  // never read a partial this sequence did not write
+        wv[k] = sl >= 0 ? s_w[u] : 0.f;
+        v[k] = sl >= 0 ? reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4]
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        acc.x = fmaf(v[k].x, wv[k], acc.x);
+        acc.y = fmaf(v[k].y, wv[k], acc.y);
+        acc.z = fmaf(v[k].z, wv[k], acc.z);
+        acc.w = fmaf(v[k].w, wv[k], acc.w);
+      }
     }
     __syncthreads();  // s_w, s_slot are rewritten by the next pass
   }
@@ -639,7 +587,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
   if (tid < 32) {
     float4 r = s_acc[0][tid];
 #pragma unroll
-    for (int g2 = 1; g2 < 4; ++g2) {
+    for (int g2 = 1; g2 < kMergeGroups; ++g2) {
       r.x += s_acc[g2][tid].x;
       r.y += s_acc[g2][tid].y;
       r.z += s_acc[g2][tid].z;
@@ -717,41 +665,48 @@ bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_
 
 bool tensor_decode_batch_ok(int batch) { return batch >= 1 && batch <= kMaxBatch; }
 
-// One wave: every resident CTA slot of the GPU.
-int tensor_decode_default_ctas(int sms) { return ctas_per_sm() * (sms > 0 ? sms : 148); }
+// One wave: every resident CTA slot of the GPU (the tcgen05 kernel holds one SM per CTA).
+int tensor_decode_default_ctas(int sms, int variant) {
+  return (variant == kDecodeUmma ? 1 : ctas_per_sm()) * (sms > 0 ? sms : 148);
+}
 
 size_t tensor_decode_workspace_bytes(int batch, int grid) { return carve(nullptr, batch, grid).bytes; }
 
 cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream) {
   const CacheView& cv = a.cache;
-  const uint64_t rows_k = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_k;
-  const uint64_t rows_v = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_v;
-  CUtensorMap tbk, tbv, tak, tav;
   cudaError_t e;
-  if ((e = encode_bf16_2d(&tbk, cv.b_k, kD, rows_k, 64, kRows, 128)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tbv, cv.b_v, kD, rows_v, 64, kRows, 128)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows_k, kH, kRows, 64)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows_v, kH, kRows, 64)) != cudaSuccess) return e;
   TcWorkspace ws = carve(a.workspace, cv.batch, a.grid);
   DecodeTcParams p;
   p.seq_lens = cv.seq_lens;
-  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.q = a.q;
   p.q_pos = a.q_pos;
   p.batch = cv.batch;
   p.capacity = cv.capacity;
   p.max_len = a.max_len;
   p.grid = a.grid;
   p.zs = a.scale * kLog2e / static_cast<float>(cv.r_k);
+  p.inv_rv = 1.f / static_cast<float>(cv.r_v);
   p.out = a.out;
   p.ws_prefix = ws.prefix;
   p.ws_ml = ws.ml;
   p.ws_o = ws.o;
   p.err = a.err;
   p.rope = a.rope;
-  auto kern = cv.r_k == 1 ? decode_tc_kernel<1> : decode_tc_kernel<2>;
-  if ((e = set_smem_once(cv.r_k)) != cudaSuccess) return e;
-  kern<<<a.grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
-  e = cudaGetLastError();
+  if (a.variant == kDecodeUmma) {
+    e = launch_decode_umma(p, cv, stream);
+  } else {
+    const uint64_t rows_k = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_k;
+    const uint64_t rows_v = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_v;
+    CUtensorMap tbk, tbv, tak, tav;
+    if ((e = encode_bf16_2d(&tbk, cv.b_k, kD, rows_k, 64, kRows, 128)) != cudaSuccess) return e;
+    if ((e = encode_bf16_2d(&tbv, cv.b_v, kD, rows_v, 64, kRows, 128)) != cudaSuccess) return e;
+    if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows_k, kH, kRows, 64)) != cudaSuccess) return e;
+    if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows_v, kH, kRows, 64)) != cudaSuccess) return e;
+    auto kern = cv.r_k == 1 ? decode_tc_kernel<1> : decode_tc_kernel<2>;
+    if ((e = set_smem_once(cv.r_k)) != cudaSuccess) return e;
+    kern<<<a.grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   TcMergeParams mp;
   mp.batch = cv.batch;
@@ -762,7 +717,7 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   mp.out = a.out;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cv.batch, kH);
-  cfg.blockDim = dim3(kD);
+  cfg.blockDim = dim3(kMergeThreads);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -113,6 +113,8 @@ bool use_tensor_decode(const tpa_cache* c, int kernel) {
          tensor_decode_batch_ok(c->batch);
 }
 
+int decode_variant(int kernel) { return kernel == TPA_KERNEL_TENSOR_SYNC ? kDecodeSync : kDecodeUmma; }
+
 // CUDA-core decode: split j of sequence b covers tokens [j*chunk, (j+1)*chunk).
 SplitPlan plan_splits(const tpa_cache* c, int max_len, int num_splits, int sms) {
   SplitPlan p;
@@ -241,7 +243,7 @@ int32_t tpa_decode_default_splits(const tpa_cache* cache, int32_t max_len, int32
   if (check_cache(cache) != TPA_OK || max_len < 0) return 0;
   int sms = 148;
   if (device_info(&sms, nullptr) != cudaSuccess) sms = 148;
-  if (use_tensor_decode(cache, kernel)) return tensor_decode_default_ctas(sms);
+  if (use_tensor_decode(cache, kernel)) return tensor_decode_default_ctas(sms, decode_variant(kernel));
   return plan_splits(cache, max_len, 0, sms).splits;
 }
 
@@ -250,7 +252,8 @@ size_t tpa_decode_workspace_size(const tpa_cache* cache, int32_t max_len, int32_
   int sms = 148;
   if (device_info(&sms, nullptr) != cudaSuccess) sms = 148;
   if (use_tensor_decode(cache, kernel))
-    return tensor_decode_workspace_bytes(cache->batch, num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms));
+    return tensor_decode_workspace_bytes(
+        cache->batch, num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms, decode_variant(kernel)));
   const SplitPlan p = plan_splits(cache, max_len, num_splits, sms);
   return carve_decode_ws(nullptr, cache->batch, cache->heads, cache->head_dim, p.splits).bytes;
 }
@@ -264,9 +267,10 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
   if (max_len < 0) return fail(TPA_ERR_SHAPE, "max_len = %d < 0", max_len);
   if (max_len > cache->capacity) return fail(TPA_ERR_CAPACITY, "max_len %d > capacity %d", max_len, cache->capacity);
   if (num_splits < 0) return fail(TPA_ERR_SHAPE, "num_splits = %d < 0", num_splits);
-  if (kernel != TPA_KERNEL_AUTO && kernel != TPA_KERNEL_SIMT && kernel != TPA_KERNEL_TENSOR)
+  if (kernel != TPA_KERNEL_AUTO && kernel != TPA_KERNEL_SIMT && kernel != TPA_KERNEL_TENSOR &&
+      kernel != TPA_KERNEL_TENSOR_SYNC)
     return fail(TPA_ERR_SHAPE, "kernel = %d", kernel);
-  if (kernel == TPA_KERNEL_TENSOR &&
+  if ((kernel == TPA_KERNEL_TENSOR || kernel == TPA_KERNEL_TENSOR_SYNC) &&
       !tensor_decode_supported(cache->dtype, cache->heads, cache->head_dim, cache->r_k, cache->r_v))
     return fail(TPA_ERR_UNSUPPORTED, "tensor-core decode needs bf16, heads 32, head_dim 128, r_k == r_v <= 2");
   if (!isfinite(scale)) return fail(TPA_ERR_SHAPE, "scale is not finite");
@@ -279,10 +283,11 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   RopeTable rope;
   make_rope_table(cache->rope_base, cache->head_dim, &rope);
-  if (kernel == TPA_KERNEL_TENSOR && !tensor_decode_batch_ok(cache->batch))
+  if ((kernel == TPA_KERNEL_TENSOR || kernel == TPA_KERNEL_TENSOR_SYNC) && !tensor_decode_batch_ok(cache->batch))
     return fail(TPA_ERR_UNSUPPORTED, "tensor-core decode takes at most 1024 sequences per call");
   if (use_tensor_decode(cache, kernel)) {
-    const int grid = num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms);
+    const int variant = decode_variant(kernel);
+    const int grid = num_splits > 0 ? num_splits : tensor_decode_default_ctas(sms, variant);
     const size_t need = tensor_decode_workspace_bytes(cache->batch, grid);
     if (!workspace) return fail(TPA_ERR_WORKSPACE, "workspace is NULL, %zu bytes needed", need);
     if (workspace_bytes < need)
@@ -299,6 +304,7 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
     a.workspace = workspace;
     a.rope = rope;
     a.err = err;
+    a.variant = variant;
     e = launch_tensor_decode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
     return TPA_OK;

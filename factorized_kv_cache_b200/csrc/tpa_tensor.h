@@ -10,9 +10,14 @@ namespace tpa {
 
 // ---- decode (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2}, batch <= 1024)
 // The grid is `grid` CTAs sharing the batch's tiles evenly (see decode_tensor.cu).
+// Two kernels share the partition, the workspace layout and the merge:
+// kDecodeUmma (tcgen05, TMEM accumulators, one CTA per SM) and kDecodeSync
+// (warp-level mma.sync, two CTAs per SM).
+constexpr int kDecodeUmma = 0;
+constexpr int kDecodeSync = 1;
 bool tensor_decode_supported(int dtype, int heads, int head_dim, int r_k, int r_v);
 bool tensor_decode_batch_ok(int batch);
-int tensor_decode_default_ctas(int sms);
+int tensor_decode_default_ctas(int sms, int variant);
 size_t tensor_decode_workspace_bytes(int batch, int grid);
 
 struct TensorDecodeArgs {
@@ -26,6 +31,7 @@ struct TensorDecodeArgs {
   void* workspace;  // tensor_decode_workspace_bytes(batch, grid) bytes, 256-byte aligned
   RopeTable rope;
   unsigned int* err;
+  int variant;  // kDecodeUmma or kDecodeSync
 };
 cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream);
 

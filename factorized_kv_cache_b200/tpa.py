@@ -21,7 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "tpa.h")
 
 TPA_OK = 0
 TPA_F32, TPA_BF16 = 0, 1
-TPA_KERNEL_AUTO, TPA_KERNEL_SIMT, TPA_KERNEL_TENSOR = 0, 1, 2
+TPA_KERNEL_AUTO, TPA_KERNEL_SIMT, TPA_KERNEL_TENSOR, TPA_KERNEL_TENSOR_SYNC = 0, 1, 2, 3
 TPA_DEVERR_APPEND_OVERFLOW = 0x1
 TPA_DEVERR_LEN_RANGE = 0x2
 TPA_DEVERR_PREFILL_LEN = 0x4

@@ -58,12 +58,16 @@ typedef enum tpa_dtype { TPA_F32 = 0, TPA_BF16 = 1 } tpa_dtype;
 /* Kernel choice for decode and prefill.  AUTO picks the fastest kernel that
  * supports the shape: the tensor-core kernels for bf16 at head_dim 128,
  * heads 32, r_k == r_v <= 2 (decode: batch <= 1024); the CUDA-core kernels
- * otherwise.  For the tensor-core decode, num_splits is the number of CTAs
- * that share the batch's token tiles evenly (default: two per SM). */
+ * otherwise.  For the tensor-core decodes, num_splits is the number of CTAs
+ * that share the batch's token tiles evenly (default: one wave, i.e. one
+ * CTA per SM for TPA_KERNEL_TENSOR and two for TPA_KERNEL_TENSOR_SYNC). */
 typedef enum tpa_kernel {
   TPA_KERNEL_AUTO = 0,
-  TPA_KERNEL_SIMT = 1,   /* CUDA-core fp32 FMA path (every supported shape) */
-  TPA_KERNEL_TENSOR = 2  /* tensor-core path (bf16 only; TPA_ERR_UNSUPPORTED otherwise) */
+  TPA_KERNEL_SIMT = 1,        /* CUDA-core fp32 FMA path (every supported shape) */
+  TPA_KERNEL_TENSOR = 2,      /* tensor-core path (bf16 only; TPA_ERR_UNSUPPORTED otherwise):
+                               * tcgen05 MMAs with TMEM accumulators */
+  TPA_KERNEL_TENSOR_SYNC = 3  /* decode only: the same shapes on warp-level mma.sync tensor-core
+                               * instructions, kept for comparison with TPA_KERNEL_TENSOR */
 } tpa_kernel;
 
 /* Device error word bits (tpa_read_device_error). */

@@ -16,7 +16,8 @@ from tests.parity_util import TOL, assert_rows_close, default_scale, f64, oracle
 
 pytestmark = pytest.mark.gpu
 
-KERNELS = [T.TPA_KERNEL_SIMT, T.TPA_KERNEL_AUTO]
+KERNELS = [T.TPA_KERNEL_SIMT, T.TPA_KERNEL_AUTO, T.TPA_KERNEL_TENSOR_SYNC]
+TENSOR_KERNELS = [T.TPA_KERNEL_TENSOR, T.TPA_KERNEL_TENSOR_SYNC]
 
 
 def _check(w, cache, x, q, q_pos, out, batches=None, heads=None, end_to_end=True):
@@ -46,7 +47,7 @@ def _check(w, cache, x, q, q_pos, out, batches=None, heads=None, end_to_end=True
     return worst
 
 
-@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("kernel", [T.TPA_KERNEL_SIMT, T.TPA_KERNEL_AUTO])
 def test_tiny_f32_workload(kernel):
     w = S.WORKLOADS["decode_tiny_f32"]
     cache, x, q, q_pos = build_decode_cache(w)
@@ -131,15 +132,16 @@ def test_long_512k_workload_full_size(kernel):
     assert T.tpa_read_device_error() == 0
 
 
+@pytest.mark.parametrize("kernel", TENSOR_KERNELS)
 @pytest.mark.parametrize("grid", [1, 2, 5, 37, 148, 300])
 @pytest.mark.parametrize("name", ["decode_b8_l8k", "decode_b32_var32k"])
-def test_tensor_kernel_partition_grids(grid, name):
+def test_tensor_kernel_partition_grids(kernel, grid, name):
     """The tensor-core kernel's even split of all tiles over `grid` CTAs: sequences spanning
     many CTAs, CTAs spanning many sequences, empty sequences, more CTAs than tiles."""
     w = S.WORKLOADS[name]
     lengths = [5000, 1, 0, 64, 65, 130, 3000, 7]
     cache, x, q, q_pos = build_decode_cache(w, batch=8, length=5000, lengths=lengths)
-    out = T.tpa_decode_attention(cache, q, q_pos, max_len=5000, num_splits=grid, kernel=T.TPA_KERNEL_TENSOR)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=5000, num_splits=grid, kernel=kernel)
     _check(w, cache, x, q, q_pos, out, end_to_end=False)
     assert torch.count_nonzero(out[2]) == 0
     assert T.tpa_read_device_error() == 0
@@ -166,3 +168,30 @@ def test_unit_variance_factors(kernel, rank):
     cache, x, q, q_pos = build_decode_cache(w, batch=3, length=4000, min_length=1000)
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=4000, kernel=kernel)
     _check(w, cache, x, q, q_pos, out)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("rank", [1, 2])
+@pytest.mark.parametrize("direction", [1, -1])
+def test_score_ramp(kernel, rank, direction):
+    """Scores that climb steadily along the sequence (direction 1: the running maximum grows on
+    almost every tile, so every rescale path runs) or fall (direction -1: the first tile holds
+    the maximum).  B_K is overwritten with multiples of the rotated query; the oracle reads the
+    cache back, so only the attention is compared."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="ramp", r_k=rank, r_v=rank, seed=91)
+    lengths = [4000, 2500, 129]
+    cache, x, q, q_pos = build_decode_cache(w, batch=3, length=4000, lengths=lengths)
+    for b, L in enumerate(lengths):
+        qr = O.rope(f64(q[b]).astype(np.float64), float(q_pos[b]), w.rope_base)  # [h, d]
+        u = qr.mean(axis=0)
+        u /= np.linalg.norm(u)
+        ramp = np.arange(L, dtype=np.float64) / L
+        if direction < 0:
+            ramp = ramp[::-1].copy()
+        # head-averaged query direction times a ramp: scores span ~60 natural-log units per head
+        bk = (60.0 * np.sqrt(w.head_dim) / np.abs(qr @ u).max()) * ramp[:, None, None] * u[None, None, :]
+        bk = np.repeat(bk, rank, axis=1)
+        cache.b_k[b, :L] = torch.from_numpy(bk).to(cache.b_k.dtype).to(DEV)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=4000, kernel=kernel)
+    _check(w, cache, x, q, q_pos, out, end_to_end=False)
+    assert T.tpa_read_device_error() == 0
