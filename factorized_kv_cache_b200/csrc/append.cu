@@ -12,6 +12,7 @@
 // over many CTAs and bump the lengths in a second one-CTA launch, so no CTA
 // ever reads a length another CTA has already advanced.
 #include "device_common.cuh"
+#include "ptx_sm100.cuh"
 #include "tpa_internal.h"
 
 namespace tpa {
@@ -21,15 +22,31 @@ constexpr int kAppendThreads = 256;
 constexpr int kTokensPerCta = 8;
 constexpr int kSingleCtaMaxTokens = 32;
 
+// cos, sin of every (token, RoPE pair) this CTA writes, one double-precision
+// evaluation per entry spread over the CTA: s_cs[jj][pair] for tokens
+// j0 + jj, jj < n_tok.  Ends with __syncthreads.
+__device__ void rope_table(const AppendArgs& a, int b, int j0, int n_tok, float2* s_cs) {
+  const int pairs = a.cache.head_dim / 2;
+  for (int e = threadIdx.x; e < n_tok * pairs; e += blockDim.x) {
+    const int jj = e / pairs, pr = e % pairs;
+    const int pos = a.positions[static_cast<size_t>(b) * a.n_new + j0 + jj];
+    float c, s;
+    rope_cos_sin(pos, a.rope.theta[pr], &c, &s);
+    s_cs[jj * kMaxPairs + pr] = make_float2(c, s);
+  }
+  __syncthreads();
+}
+
+// Copy (A_K, A_V, B_V) or rotate (B_K) every 16-byte vector of token j of
+// sequence b into `slot`, with 64 threads; cs = that token's cos/sin row.
 template <typename T>
-__device__ void append_token(const AppendArgs& a, int b, int j, int slot) {
+__device__ void append_token(const AppendArgs& a, int b, int j, int slot, const float2* cs) {
   constexpr int V = Vec16<T>::N;
   const int h = a.cache.heads, d = a.cache.head_dim;
   const int rk = a.cache.r_k, rv = a.cache.r_v;
   const size_t cap = a.cache.capacity;
   const size_t src_tok = static_cast<size_t>(b) * a.n_new + j;
   const size_t dst_tok = static_cast<size_t>(b) * cap + slot;
-  const int pos = a.positions[static_cast<size_t>(b) * a.n_new + j];
   // vectors per plane for this token
   const int n_ak = rk * h / V, n_bk = rk * d / V, n_av = rv * h / V, n_bv = rv * d / V;
   const int total = n_ak + n_bk + n_av + n_bv;
@@ -47,9 +64,8 @@ __device__ void append_token(const AppendArgs& a, int b, int j, int slot) {
       load16_f32(src, x);
 #pragma unroll
       for (int p = 0; p < V / 2; ++p) {
-        float c, s;
-        rope_cos_sin(pos, a.rope.theta[(e0 >> 1) + p], &c, &s);
-        rope_pair(x[2 * p], x[2 * p + 1], c, s);
+        const float2 r = cs[(e0 >> 1) + p];
+        rope_pair(x[2 * p], x[2 * p + 1], r.x, r.y);
       }
       store16_from_f32(dst, x);
     } else if (v < n_ak + n_bk + n_av) {
@@ -69,16 +85,20 @@ __device__ void append_token(const AppendArgs& a, int b, int j, int slot) {
 // One CTA per sequence: read the length, write every token, bump the length.
 template <typename T>
 __global__ void __launch_bounds__(kAppendThreads) append_single_kernel(const __grid_constant__ AppendArgs a) {
+  // a kernel launched after this one with programmatic dependent launch may start its own
+  // set-up now; it waits for this grid before it reads anything written here
+  ptx::pdl_launch_dependents();
   __shared__ int s_base;
+  __shared__ float2 s_cs[kSingleCtaMaxTokens * kMaxPairs];
   const int b = blockIdx.x;
   if (threadIdx.x == 0) s_base = a.seq_lens[b];
-  __syncthreads();
+  rope_table(a, b, 0, a.n_new, s_cs);  // ends with __syncthreads
   const int base = s_base;
   const bool fits = base >= 0 && base + a.n_new <= a.cache.capacity;
   for (int j = threadIdx.x / 64; j < a.n_new; j += kAppendThreads / 64) {
     const int slot = base + j;
     if (slot < 0 || slot >= a.cache.capacity) continue;
-    append_token<T>(a, b, j, slot);
+    append_token<T>(a, b, j, slot, s_cs + j * kMaxPairs);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -94,9 +114,12 @@ __global__ void __launch_bounds__(kAppendThreads) append_single_kernel(const __g
 // the lengths are not touched at all.
 template <typename T>
 __global__ void __launch_bounds__(kAppendThreads) append_multi_kernel(const __grid_constant__ AppendArgs a) {
+  ptx::pdl_launch_dependents();
+  __shared__ float2 s_cs[kTokensPerCta * kMaxPairs];
   const int b = blockIdx.y;
   const int base = a.slots ? 0 : a.seq_lens[b];
   const int j0 = blockIdx.x * kTokensPerCta;
+  rope_table(a, b, j0, min(kTokensPerCta, a.n_new - j0), s_cs);
   for (int jj = threadIdx.x / 64; jj < kTokensPerCta; jj += kAppendThreads / 64) {
     const int j = j0 + jj;
     if (j >= a.n_new) break;
@@ -105,7 +128,7 @@ __global__ void __launch_bounds__(kAppendThreads) append_multi_kernel(const __gr
       if (a.slots && (threadIdx.x & 63) == 0) atomicOr(a.err, TPA_DEVERR_APPEND_OVERFLOW);
       continue;
     }
-    append_token<T>(a, b, j, slot);
+    append_token<T>(a, b, j, slot, s_cs + jj * kMaxPairs);
   }
 }
 

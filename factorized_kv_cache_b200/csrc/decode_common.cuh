@@ -36,14 +36,18 @@ struct DecodeTcParams {
   RopeTable rope;
 };
 
-// CTA that owns tile t.
+// CTA that owns tile t: floor(t grid / nt).  The quotient is formed in
+// double precision, which is exact here: the product is an integer below
+// 2^53, and a quotient that is not an integer sits at least 1/nt away from
+// one, far above the 2^-53 relative rounding (64-bit integer division would
+// cost a long instruction sequence at kernel start).
 __device__ __forceinline__ int owner_of(int t, int nt, int grid) {
-  return static_cast<int>((static_cast<long long>(t) * grid) / nt);
+  return static_cast<int>(floor(static_cast<double>(t) * grid / nt));
 }
 
-// First tile of CTA c.
+// First tile of CTA c: ceil(c nt / grid), exact for the same reason.
 __device__ __forceinline__ int first_tile(int c, int nt, int grid) {
-  return static_cast<int>((static_cast<long long>(c) * nt + grid - 1) / grid);
+  return static_cast<int>(ceil(static_cast<double>(c) * nt / grid));
 }
 
 // Exclusive prefix of per-sequence tile counts into s_pref[0..B] and the

@@ -537,50 +537,79 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     if (!(a < e && a < t1 && e > t0)) return -1;
     return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
   };
-  float M = -INFINITY;
-  for (int u = tid; u < n; u += kMergeThreads) {
-    const int sl = slot_of(u);
-    if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
-  }
-  M = merge_reduce(M, true, s_red);
+  const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
-  for (int c0 = 0; c0 < n; c0 += kMergeMax) {
-    const int cn = min(kMergeMax, n - c0);
-    float lpart = 0.f;
-    for (int u = tid; u < cn; u += kMergeThreads) {
-      const int sl = slot_of(c0 + u);
-      float w = 0.f;
-      if (sl >= 0) {
-        const float mj = p.ws_ml[2 * static_cast<size_t>(sl)];
-        w = mj == -INFINITY ? 0.f : exp2f(mj - M);
-        lpart = fmaf(p.ws_ml[2 * static_cast<size_t>(sl) + 1], w, lpart);
-      }
-      s_w[u] = w;
-      s_slot[u] = sl;
-    }
-    L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
-    for (int u0 = grp; u0 < cn; u0 += kMergeGroups * kMergeBatch) {
-      float4 v[kMergeBatch];
-      float wv[kMergeBatch];
+  if (n <= kMergeGroups * kMergeBatch) {
+    // one pass: every partial's features and (m, l) are loaded at once, before the maximum is known
+    float4 v[kMergeBatch];
+    bool has[kMergeBatch];
 #pragma unroll
-      for (int k = 0; k < kMergeBatch; ++k) {
-        const int u = u0 + kMergeGroups * k;
-        const int sl = u < cn ? s_slot[u] : -1;  // never read a partial this sequence did not write
-        wv[k] = sl >= 0 ? s_w[u] : 0.f;
-        v[k] = sl >= 0 ? reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4]
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int k = 0; k < kMergeBatch; ++k) {
-        acc.x = fmaf(v[k].x, wv[k], acc.x);
-        acc.y = fmaf(v[k].y, wv[k], acc.y);
-        acc.z = fmaf(v[k].z, wv[k], acc.z);
-        acc.w = fmaf(v[k].w, wv[k], acc.w);
-      }
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const int u = grp + kMergeGroups * k;
+      const int sl = u < n ? slot_of(u) : -1;  // never read a partial this sequence did not write
+      has[k] = sl >= 0;
+      v[k] = has[k] ? reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4]
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();  // s_w, s_slot are rewritten by the next pass
+    const int my = tid < n ? slot_of(tid) : -1;
+    const float2 ml = my >= 0 ? *reinterpret_cast<const float2*>(p.ws_ml + 2 * static_cast<size_t>(my))
+                              : make_float2(-INFINITY, 0.f);
+    const float M = merge_reduce(ml.x, true, s_red);
+    const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
+    if (tid < n) s_w[tid] = w;
+    L = merge_reduce(ml.y * w, false, s_red);  // ends with a barrier: s_w visible
+#pragma unroll
+    for (int k = 0; k < kMergeBatch; ++k) {
+      const float wk = has[k] ? s_w[grp + kMergeGroups * k] : 0.f;
+      acc.x = fmaf(v[k].x, wk, acc.x);
+      acc.y = fmaf(v[k].y, wk, acc.y);
+      acc.z = fmaf(v[k].z, wk, acc.z);
+      acc.w = fmaf(v[k].w, wk, acc.w);
+    }
+  } else {
+    float M = -INFINITY;
+    for (int u = tid; u < n; u += kMergeThreads) {
+      const int sl = slot_of(u);
+      if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
+    }
+    M = merge_reduce(M, true, s_red);
+    for (int c0 = 0; c0 < n; c0 += kMergeMax) {
+      const int cn = min(kMergeMax, n - c0);
+      float lpart = 0.f;
+      for (int u = tid; u < cn; u += kMergeThreads) {
+        const int sl = slot_of(c0 + u);
+        float w = 0.f;
+        if (sl >= 0) {
+          const float mj = p.ws_ml[2 * static_cast<size_t>(sl)];
+          w = mj == -INFINITY ? 0.f : exp2f(mj - M);
+          lpart = fmaf(p.ws_ml[2 * static_cast<size_t>(sl) + 1], w, lpart);
+        }
+        s_w[u] = w;
+        s_slot[u] = sl;
+      }
+      L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
+      for (int u0 = grp; u0 < cn; u0 += kMergeGroups * kMergeBatch) {
+        float4 v[kMergeBatch];
+        float wv[kMergeBatch];
+#pragma unroll
+        for (int k = 0; k < kMergeBatch; ++k) {
+          const int u = u0 + kMergeGroups * k;
+          const int sl = u < cn ? s_slot[u] : -1;  // never read a partial this sequence did not write
+          wv[k] = sl >= 0 ? s_w[u] : 0.f;
+          v[k] = sl >= 0 ? reinterpret_cast<const float4*>(p.ws_o + static_cast<size_t>(sl) * kD)[f4]
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kMergeBatch; ++k) {
+          acc.x = fmaf(v[k].x, wv[k], acc.x);
+          acc.y = fmaf(v[k].y, wv[k], acc.y);
+          acc.z = fmaf(v[k].z, wv[k], acc.z);
+          acc.w = fmaf(v[k].w, wv[k], acc.w);
+        }
+      }
+      __syncthreads();  // s_w, s_slot are rewritten by the next pass
+    }
   }
   s_acc[grp][f4] = acc;
   __syncthreads();

@@ -18,26 +18,31 @@
 // splits keep ~16 bits: one bf16 rounding of W costs up to ~3e-3 relative
 // error on the decode workloads, above their 2e-3 budget.
 //
-// Roles (192 threads, one CTA per SM): warp 0 streams tiles with TMA
+// Roles (320 threads, one CTA per SM): warp 0 streams tiles with TMA
 // (no multicast) into a K ring {B_K, A_K} and a V ring {B_V, A_V}, two
-// 40 KB slots each; warp 1 owns 256 TMEM columns and one of its threads
-// issues the MMAs; warps 2-5 run the softmax, one thread per cache row
-// (TMEM lane) for the scores and one per feature (TMEM lane) for O^T.
+// 40 KB slots each, the K loads running one tile ahead of the V loads;
+// warp 1 owns 256 TMEM columns and one of its threads issues the MMAs;
+// warps 2-9 run the softmax.  TMEM lane quadrant q (warps q + 2 and q + 6)
+// holds cache rows 32q .. 32q + 31 of S and features 32q .. 32q + 31 of
+// O^T; warps 2-5 take heads 0-15 of their rows, warps 6-9 heads 16-31, so
+// every sub-partition runs two softmax warps.
 // Per tile j: S(j) goes to TMEM columns [64 (j % 2), +64), so the score MMA
 // of tile j + 1 overlaps the softmax of tile j; W(j) goes to one of two
 // shared-memory buffers; O^T sits in columns [128, 192).  The K slot is
 // released once the score MMA has completed and the softmax has read A_K;
 // the V slot once the value MMA has completed.
 //
-// Softmax: every thread holds its row's 32 scores.  The running maxima m_i
+// Softmax: every thread holds 16 scores of its row.  The running maxima m_i
 // are shared by the CTA and move lazily: one barrier-with-OR per tile asks
 // whether any score exceeds its head's maximum by more than 2^8; only then
-// is the tile maximum reduced (warp reduce-scatter plus a 4-warp exchange)
-// and O^T, l rescaled.  The row sums l_i stay per thread and are reduced at
-// the end of a sequence segment.
+// is the tile maximum reduced (warp reduce-scatter plus a 4-quadrant
+// exchange) and O^T, l rescaled.  The row sums l_i stay per thread and are
+// reduced at the end of a sequence segment.
 //
 // Scheduling, partials and the merge follow the balanced tile partition in
 // decode_common.cuh (shared with the warp-level kernel in decode_tensor.cu).
+// The kernel is launched with programmatic dependent launch: barriers, TMEM
+// and the tensor maps are set up before it waits for the preceding kernel.
 //
 // Every wait is bounded (2 s): on a timeout the waiting thread sets the error
 // word and an abort flag; the softmax warps leave their loop together at the
@@ -64,7 +69,10 @@ using dec::kH;
 using dec::kMaxBatch;
 
 constexpr int kRows = 128;                   // cache rows per tile
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kThreads = 64 + kSoftmaxThreads;
+constexpr int kHalf = kH / 2;                // heads per softmax thread
 constexpr int kBox = kRows * 128;            // 64 features x 128 rows, bf16: 16 KB
 constexpr int kBBytes = 2 * kBox;            // one B tile
 constexpr int kABytes = kRows * kH * 2;      // one A tile: 8 KB
@@ -75,7 +83,7 @@ constexpr int kOffK = 0;                     // K ring: 2 slots {B_K, A_K}
 constexpr int kOffV = kOffK + 2 * kSlotBytes;  // V ring: 2 slots {B_V, A_V}
 constexpr int kOffW = kOffV + 2 * kSlotBytes;  // two W buffers
 constexpr int kOffQ = kOffW + 2 * kWBytes;     // query hi/lo, two 64-feature boxes
-constexpr int kOffRed = kOffQ + 2 * kQBox;     // float [4][32]: per-warp head reductions
+constexpr int kOffRed = kOffQ + 2 * kQBox;     // float [4 quadrants][32 heads]
 constexpr int kOffCs = kOffRed + 4 * 32 * 4;   // float [64][2]: cos, sin of the query position
 constexpr int kOffBar = kOffCs + 64 * 2 * 4;
 // kfull[2], kempty[2], vfull[2], vempty[2], sfull[2], wready[2], wfree[2], qready, fin
@@ -96,12 +104,13 @@ constexpr uint32_t kIdescScore = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3
 // value MMA: A (B_V^T) and B (W) both MN-major
 constexpr uint32_t kIdescValue = kIdescScore | (1u << 15) | (1u << 16);
 
-// Reduce 32 per-head values over the 32 lanes of a warp; afterwards lane k
-// holds the result for head k (five halving exchange steps, 31 shuffles).
+// Reduce 16 per-head values over the 32 lanes of a warp; afterwards lanes k
+// and k + 16 hold the result for head k (four halving exchange steps, then
+// one across the two half-warps: 16 shuffles).
 template <bool kMax>
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+__device__ __forceinline__ float reduce_scatter16(float (&v)[kHalf], int lane) {
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
+  for (int o = 8; o >= 1; o >>= 1) {
     const bool up = (lane & o) != 0;
 #pragma unroll
     for (int i = 0; i < o; ++i) {
@@ -111,23 +120,48 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
       v[i] = kMax ? fmaxf(keep, got) : keep + got;
     }
   }
-  return v[0];
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
-__device__ __forceinline__ void unpack8(const uint4 v, float* f) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Heads 16 hh .. 16 hh + 15 of row `row` of a 128-row A tile (32 bf16 =
+// 64 bytes per row, 64-byte swizzle) as fp32.
+__device__ __forceinline__ void load_a_half(const uint8_t* tile, int row, int hh, float* f) {
+  const uint8_t* base = tile + row * 64;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    f[2 * k] = ptx::bf16_lo(w[k]);
-    f[2 * k + 1] = ptx::bf16_hi(w[k]);
+  for (int c = 0; c < 2; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(base + (((2 * hh + c) ^ ((row >> 1) & 3)) << 4));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[8 * c + 2 * k] = ptx::bf16_lo(w[k]);
+      f[8 * c + 2 * k + 1] = ptx::bf16_hi(w[k]);
+    }
   }
 }
 
-// Row `row` of a 128-row A tile (32 bf16 = 64 bytes, 64-byte swizzle) as fp32.
-__device__ __forceinline__ void load_a_row(const uint8_t* tile, int row, float* f) {
-  const uint8_t* base = tile + row * 64;
+// Sum over the four TMEM lane quadrants of the per-quadrant head values in
+// s_red[quad][32], for heads 16 hh .. 16 hh + 15.
+template <bool kMax>
+__device__ __forceinline__ void combine_quadrants(const float* s_red, int hh, float (&out)[kHalf]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) unpack8(*reinterpret_cast<const uint4*>(base + ((c ^ ((row >> 1) & 3)) << 4)), f + 8 * c);
+  for (int h4 = 0; h4 < kHalf / 4; ++h4) {
+    const float4 x0 = reinterpret_cast<const float4*>(s_red + 16 * hh)[h4];
+    const float4 x1 = reinterpret_cast<const float4*>(s_red + 32 + 16 * hh)[h4];
+    const float4 x2 = reinterpret_cast<const float4*>(s_red + 64 + 16 * hh)[h4];
+    const float4 x3 = reinterpret_cast<const float4*>(s_red + 96 + 16 * hh)[h4];
+    if (kMax) {
+      out[4 * h4] = fmaxf(fmaxf(x0.x, x1.x), fmaxf(x2.x, x3.x));
+      out[4 * h4 + 1] = fmaxf(fmaxf(x0.y, x1.y), fmaxf(x2.y, x3.y));
+      out[4 * h4 + 2] = fmaxf(fmaxf(x0.z, x1.z), fmaxf(x2.z, x3.z));
+      out[4 * h4 + 3] = fmaxf(fmaxf(x0.w, x1.w), fmaxf(x2.w, x3.w));
+    } else {
+      out[4 * h4] = (x0.x + x1.x) + (x2.x + x3.x);
+      out[4 * h4 + 1] = (x0.y + x1.y) + (x2.y + x3.y);
+      out[4 * h4 + 2] = (x0.z + x1.z) + (x2.z + x3.z);
+      out[4 * h4 + 3] = (x0.w + x1.w) + (x2.w + x3.w);
+    }
+  }
 }
 
 template <int R>
@@ -162,81 +196,100 @@ __global__ void __launch_bounds__(kThreads, 1)
   int32_t* s_len = reinterpret_cast<int32_t*>(gbase + kOffLen);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // Set-up that touches no global memory runs before the wait on the preceding kernel
+  // (programmatic dependent launch): barriers, TMEM, tensor-map prefetch.
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(kfull(s), 1);
-      ptx::mbar_init(kempty(s), 1 + 4);  // score-MMA commit + the four softmax warps (A_K read)
+      ptx::mbar_init(kempty(s), 1 + kSoftmaxWarps);  // score-MMA commit + the softmax warps (A_K read)
       ptx::mbar_init(vfull(s), 1);
       ptx::mbar_init(vempty(s), 1);
       ptx::mbar_init(sfull(s), 1);
-      ptx::mbar_init(wready(s), 4);
+      ptx::mbar_init(wready(s), kSoftmaxWarps);
       ptx::mbar_init(wfree(s), 1);
     }
-    ptx::mbar_init(qready, 4);
+    ptx::mbar_init(qready, kSoftmaxWarps);
     ptx::mbar_init(fin, 1);
     *s_abort = 0;
     ptx::fence_barrier_init();
   }
-  dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
-  const int B = p.batch;
-  const int NT = s_pref[B];
-  if (blockIdx.x == 0)
-    for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
-  if (NT == 0) return;
-  const int c = blockIdx.x;
-  const int t_begin = dec::first_tile(c, NT, p.grid);
-  const int t_end = dec::first_tile(c + 1, NT, p.grid);
-  if (t_begin >= t_end) return;  // uniform: before any TMEM is held
-  const int b_first = dec::sequence_of_tile(s_pref, B, t_begin);
-
   if (warp == 1) {
     ptx::tmem_alloc(sbase + kOffMisc, kTmemCols);
     ptx::tmem_relinquish();
+  }
+  if (tid == 0) {
+    ptx::prefetch_tmap(&tm_bk);
+    ptx::prefetch_tmap(&tm_bv);
+    ptx::prefetch_tmap(&tm_ak);
+    ptx::prefetch_tmap(&tm_av);
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tbase = *s_taddr;
+  ptx::pdl_wait();  // the cache, the lengths and the query are written by earlier work
+
+  dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
+  const int B = p.batch;
+  const int NT = s_pref[B];
+  if (blockIdx.x == 0)
+    for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
+  const int c = blockIdx.x;
+  const int t_begin = NT == 0 ? 0 : dec::first_tile(c, NT, p.grid);
+  const int t_end = NT == 0 ? 0 : dec::first_tile(c + 1, NT, p.grid);
+  if (t_begin >= t_end) {  // uniform: no tiles for this CTA
+    if (warp == 1) ptx::tmem_dealloc(tbase, kTmemCols);
+    return;
+  }
+  const int b_first = dec::sequence_of_tile(s_pref, B, t_begin);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // Load order K0, K1, V0, K2, V1, K3, ...: the score MMA of a tile needs only its K
+    // slot, and the softmax reaches for A_V (the V slot) last.
     if (lane == 0) {
-      ptx::prefetch_tmap(&tm_bk);
-      ptx::prefetch_tmap(&tm_bv);
-      ptx::prefetch_tmap(&tm_ak);
-      ptx::prefetch_tmap(&tm_av);
-      int it = 0, k_issued = 0, v_issued = 0;
+      const int n = t_end - t_begin;
+      int kb_seq = b_first, vb_seq = b_first;  // sequence cursors of the K and V streams
+      auto row_of = [&](int j, int& cur) {
+        const int t = t_begin + j;
+        while (s_pref[cur + 1] <= t) ++cur;
+        return (cur * p.capacity + (t - s_pref[cur]) * TOK) * R;
+      };
+      auto load_k = [&](int j) -> bool {
+        const int s = j & 1;
+        if (j >= 2 && !ptx::mbar_wait_bounded(kempty(s), ((j >> 1) & 1) ^ 1)) return false;
+        const int row0 = row_of(j, kb_seq);
+        const uint32_t kb = sbase + kOffK + s * kSlotBytes;
+        ptx::mbar_arrive_expect_tx(kfull(s), kSlotBytes);
+        ptx::tma_load_2d(kb, &tm_bk, 0, row0, kfull(s));
+        ptx::tma_load_2d(kb + kBox, &tm_bk, 64, row0, kfull(s));
+        ptx::tma_load_2d(kb + kBBytes, &tm_ak, 0, row0, kfull(s));
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int s = j & 1;
+        if (j >= 2 && !ptx::mbar_wait_bounded(vempty(s), ((j >> 1) & 1) ^ 1)) return false;
+        const int row0 = row_of(j, vb_seq);
+        const uint32_t vb = sbase + kOffV + s * kSlotBytes;
+        ptx::mbar_arrive_expect_tx(vfull(s), kSlotBytes);
+        ptx::tma_load_2d(vb, &tm_bv, 0, row0, vfull(s));
+        ptx::tma_load_2d(vb + kBox, &tm_bv, 64, row0, vfull(s));
+        ptx::tma_load_2d(vb + kBBytes, &tm_av, 0, row0, vfull(s));
+        return true;
+      };
+      int k_issued = 0, v_issued = 0;
       bool ok = true;
-      for (int b = b_first; b < B && s_pref[b] < t_end && ok; ++b) {
-        const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
-        for (int t = ta; t < tb; ++t, ++it) {
-          if (*s_abort) {
-            ok = false;
-            break;
-          }
-          const int s = it & 1;
-          const uint32_t par = ((it >> 1) & 1) ^ 1;
-          const int row0 = (b * p.capacity + (t - s_pref[b]) * TOK) * R;
-          if (!ptx::mbar_wait_bounded(kempty(s), par)) {
-            ok = false;
-            break;
-          }
-          const uint32_t kb = sbase + kOffK + s * kSlotBytes;
-          ptx::mbar_arrive_expect_tx(kfull(s), kSlotBytes);
-          ptx::tma_load_2d(kb, &tm_bk, 0, row0, kfull(s));
-          ptx::tma_load_2d(kb + kBox, &tm_bk, 64, row0, kfull(s));
-          ptx::tma_load_2d(kb + kBBytes, &tm_ak, 0, row0, kfull(s));
-          k_issued = it + 1;
-          if (!ptx::mbar_wait_bounded(vempty(s), par)) {
-            ok = false;
-            break;
-          }
-          const uint32_t vb = sbase + kOffV + s * kSlotBytes;
-          ptx::mbar_arrive_expect_tx(vfull(s), kSlotBytes);
-          ptx::tma_load_2d(vb, &tm_bv, 0, row0, vfull(s));
-          ptx::tma_load_2d(vb + kBox, &tm_bv, 64, row0, vfull(s));
-          ptx::tma_load_2d(vb + kBBytes, &tm_av, 0, row0, vfull(s));
-          v_issued = it + 1;
+      for (; k_issued < min(2, n); ++k_issued) load_k(k_issued);
+      while (ok && v_issued < n) {
+        if (*s_abort) {
+          ok = false;
+          break;
+        }
+        if (!(ok = load_v(v_issued))) break;
+        ++v_issued;
+        if (k_issued < n) {
+          if (!(ok = load_k(k_issued))) break;
+          ++k_issued;
         }
       }
       if (!ok) {
@@ -315,33 +368,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ---------------------------------------------------------------- softmax warps
     const int quad = warp & 3;                // TMEM lanes 32 quad .. 32 quad + 31
+    const int hh = (warp - 2) >> 2;           // heads 16 hh .. 16 hh + 15
     const int row = quad * 32 + lane;         // tile row for the scores, feature for O^T
-    const int wq = warp - 2;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int wt = tid - 64;                  // 0 .. 127
+    const int wt = tid - 64;                  // 0 .. 255
     int it = 0;
     bool aborted = false;
     for (int b = b_first; b < B && s_pref[b] < t_end; ++b) {
       const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
       if (ta >= tb) continue;
       const int len_b = s_len[b];
-      // ---- rotated query as bf16 hi (rows 0..31) and lo (rows 32..63), K-major, 128-byte swizzle
-      if (wt < kD / 2) {
-        float cs, sn;
-        rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
-        s_cs[2 * wt] = cs;
-        s_cs[2 * wt + 1] = sn;
-      }
-      ptx::named_barrier(1, 128);
+      // ---- rotated query as bf16 hi (rows 0..31) and lo (rows 32..63), K-major, 128-byte swizzle.
+      // This thread's 16 features of one head and the position are loaded together, first.
       {
-        const int head = wt >> 2, f0 = (wt & 3) * 32;
+        const int head = wt >> 3, f0 = (wt & 7) * 16;
         const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
                                                           (static_cast<size_t>(b) * kH + head) * kD + f0);
-        uint32_t hi[16], lo[16];
+        const uint4 qv[2] = {src[0], src[1]};
+        if (wt < kD / 2) {
+          float cs, sn;
+          rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
+          s_cs[2 * wt] = cs;
+          s_cs[2 * wt + 1] = sn;
+        }
+        ptx::named_barrier(1, kSoftmaxThreads);
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x4 = src[v];
-          const uint32_t w[4] = {x4.x, x4.y, x4.z, x4.w};
+        for (int v = 0; v < 2; ++v) {
+          const uint32_t w[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int e = 4 * v + k;
@@ -354,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         uint8_t* qb = gbase + kOffQ + (f0 >> 6) * kQBox;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           const int chunk = ((f0 & 63) >> 3) + cc;
           const int sw = (chunk ^ (head & 7)) << 4;  // rows head and 32 + head share (row & 7)
           *reinterpret_cast<uint4*>(qb + head * 128 + sw) =
@@ -367,20 +421,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(qready);
 
-      float m[32], lsum[32];
+      float m[kHalf], lsum[kHalf];
 #pragma unroll
-      for (int h = 0; h < 32; ++h) {
+      for (int h = 0; h < kHalf; ++h) {
         m[h] = -INFINITY;
         lsum[h] = 0.f;
       }
-      int t = ta;
-      for (; t < tb; ++t, ++it) {
+      for (int t = ta; t < tb; ++t, ++it) {
         const int j = it, s = j & 1;
-        bool fail = false;
-        fail = !ptx::mbar_wait_bounded(sfull(s), (j >> 1) & 1);
+        bool fail = !ptx::mbar_wait_bounded(sfull(s), (j >> 1) & 1);
         if (!fail) fail = !ptx::mbar_wait_bounded(kfull(s), (j >> 1) & 1);
-        if (!fail) fail = !ptx::mbar_wait_bounded(vfull(s), (j >> 1) & 1);
-        if (!fail && j >= 2) fail = !ptx::mbar_wait_bounded(wfree(s), ((j >> 1) - 1) & 1);  // value MMA of j - 2
         if (fail) {
           atomicOr(p.err, kErrTimeout);
           *s_abort = 1;
@@ -389,77 +439,69 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tok0 = (t - s_pref[b]) * TOK;
         const int valid_rows = min(kRows, (len_b - tok0) * R);
         const bool valid = row < valid_rows;
-        // ---- scores of this row: z[i] = (S_hi + S_lo) A_K scale/R_K, log2 units
-        float z[32];
+        // ---- 16 scores of this row: z[i] = (S_hi + S_lo) A_K scale/R_K, log2 units
+        float z[kHalf];
         {
-          uint32_t sh[32], sl[32];
-          ptx::tmem_ld32(tbase + lane_off + 64u * s, sh);
-          ptx::tmem_ld32(tbase + lane_off + 64u * s + 32, sl);
-          float ak[32];
-          load_a_row(gbase + kOffK + s * kSlotBytes + kBBytes, row, ak);
+          float ak[kHalf];
+          load_a_half(gbase + kOffK + s * kSlotBytes + kBBytes, row, hh, ak);
+          uint32_t sh[kHalf], sl[kHalf];
+          ptx::tmem_ld16(tbase + lane_off + 64u * s + kHalf * hh, sh);
+          ptx::tmem_ld16(tbase + lane_off + 64u * s + 32 + kHalf * hh, sl);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < 32; ++h) z[h] = (__uint_as_float(sh[h]) + __uint_as_float(sl[h])) * ak[h];
+          for (int h = 0; h < kHalf; ++h) z[h] = (__uint_as_float(sh[h]) + __uint_as_float(sl[h])) * ak[h];
         }
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(kempty(s));  // A_K read, S(j) read
         if (R == 2) {
 #pragma unroll
-          for (int h = 0; h < 32; ++h) z[h] += __shfl_xor_sync(0xffffffffu, z[h], 1);  // ranks of one token
+          for (int h = 0; h < kHalf; ++h) z[h] += __shfl_xor_sync(0xffffffffu, z[h], 1);  // ranks of one token
         }
         bool need = false;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
+        for (int h = 0; h < kHalf; ++h) {
           z[h] = valid ? z[h] * p.zs : -INFINITY;
           need |= z[h] > m[h] + kLazy;
         }
         const bool stop = fail || *s_abort != 0;
-        if (ptx::named_barrier_or(1, 128, need || stop)) {
-          if (ptx::named_barrier_or(2, 128, stop)) {
+        if (ptx::named_barrier_or(1, kSoftmaxThreads, need || stop)) {
+          if (ptx::named_barrier_or(2, kSoftmaxThreads, stop)) {
             aborted = true;
             break;  // every softmax thread leaves here together
           }
           // ---- new maxima: tile maximum per head over the CTA
-          float v[32];
+          float v[kHalf];
 #pragma unroll
-          for (int h = 0; h < 32; ++h) v[h] = z[h];
-          s_red[wq * 32 + lane] = reduce_scatter32<true>(v, lane);
-          ptx::named_barrier(2, 128);
-          float alpha[32];
+          for (int h = 0; h < kHalf; ++h) v[h] = z[h];
+          const float wmax = reduce_scatter16<true>(v, lane);
+          if (lane < kHalf) s_red[quad * 32 + kHalf * hh + lane] = wmax;
+          ptx::named_barrier(2, kSoftmaxThreads);
+          float tmax[kHalf];
+          combine_quadrants<true>(s_red, hh, tmax);
+          float alpha[kHalf];
 #pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            const float4 x0 = reinterpret_cast<const float4*>(s_red)[h4];
-            const float4 x1 = reinterpret_cast<const float4*>(s_red + 32)[h4];
-            const float4 x2 = reinterpret_cast<const float4*>(s_red + 64)[h4];
-            const float4 x3 = reinterpret_cast<const float4*>(s_red + 96)[h4];
-            const float tm[4] = {fmaxf(fmaxf(x0.x, x1.x), fmaxf(x2.x, x3.x)),
-                                 fmaxf(fmaxf(x0.y, x1.y), fmaxf(x2.y, x3.y)),
-                                 fmaxf(fmaxf(x0.z, x1.z), fmaxf(x2.z, x3.z)),
-                                 fmaxf(fmaxf(x0.w, x1.w), fmaxf(x2.w, x3.w))};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int h = 4 * h4 + e;
-              const float mn = fmaxf(m[h], tm[e]);
-              alpha[h] = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
-              m[h] = mn;
-              lsum[h] *= alpha[h];
-            }
+          for (int h = 0; h < kHalf; ++h) {
+            const float mn = fmaxf(m[h], tmax[h]);
+            alpha[h] = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
+            m[h] = mn;
+            lsum[h] *= alpha[h];
           }
           if (t > ta) {
-            // O^T (this thread's feature lane) by alpha per head column, once the value MMA
-            // of tile j - 1 has finished accumulating
+            // O^T (this thread's feature lane, its 16 head columns of each half) by alpha,
+            // once the value MMA of tile j - 1 has finished accumulating
             bool okw = ptx::mbar_wait_bounded(wfree((j - 1) & 1), ((j - 1) >> 1) & 1);
             if (__all_sync(0xffffffffu, okw)) {
               ptx::tc_fence_after();
 #pragma unroll
-              for (int half = 0; half < 2; ++half) {
-                uint32_t o[32];
-                ptx::tmem_ld32(tbase + lane_off + kColO + 32 * half, o);
+              for (int part = 0; part < 2; ++part) {
+                uint32_t o[kHalf];
+                const uint32_t col = tbase + lane_off + kColO + 32 * part + kHalf * hh;
+                ptx::tmem_ld16(col, o);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 32; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                ptx::tmem_st32(tbase + lane_off + kColO + 32 * half, o);
+                for (int h = 0; h < kHalf; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                ptx::tmem_st16(col, o);
               }
               ptx::tmem_wait_st();
             } else {
@@ -468,13 +510,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // ---- W = p A_V / R_V as bf16 hi | lo into this row of W buffer s (MN-major, 128-byte swizzle)
+        // ---- W = p A_V / R_V as bf16 hi | lo into this row of W buffer s (MN-major, 128-byte
+        // swizzle), once the V tile has landed and the value MMA of tile j - 2 has read the buffer
         {
-          float av[32];
-          load_a_row(gbase + kOffV + s * kSlotBytes + kBBytes, row, av);
-          uint32_t whi[16], wlo[16];
+          bool okv = ptx::mbar_wait_bounded(vfull(s), (j >> 1) & 1);
+          if (okv && j >= 2) okv = ptx::mbar_wait_bounded(wfree(s), ((j >> 1) - 1) & 1);
+          if (!okv) {
+            atomicOr(p.err, kErrTimeout);
+            *s_abort = 1;
+          }
+          float av[kHalf];
+          load_a_half(gbase + kOffV + s * kSlotBytes + kBBytes, row, hh, av);
+          uint32_t whi[kHalf / 2], wlo[kHalf / 2];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < kHalf / 2; ++e) {
             const int h0 = 2 * e, h1 = 2 * e + 1;
             const float p0 = exp2f(z[h0] - m[h0]);
             const float p1 = exp2f(z[h1] - m[h1]);
@@ -487,20 +536,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* wrow = gbase + kOffW + s * kWBytes + row * 128;
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            *reinterpret_cast<uint4*>(wrow + ((cc ^ (row & 7)) << 4)) =
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chi = 2 * hh + cc, clo = 4 + 2 * hh + cc;
+            *reinterpret_cast<uint4*>(wrow + ((chi ^ (row & 7)) << 4)) =
                 make_uint4(whi[4 * cc], whi[4 * cc + 1], whi[4 * cc + 2], whi[4 * cc + 3]);
-            *reinterpret_cast<uint4*>(wrow + (((4 + cc) ^ (row & 7)) << 4)) =
+            *reinterpret_cast<uint4*>(wrow + ((clo ^ (row & 7)) << 4)) =
                 make_uint4(wlo[4 * cc], wlo[4 * cc + 1], wlo[4 * cc + 2], wlo[4 * cc + 3]);
           }
           if (!valid) {
-            // a B_V row past the sequence end may hold NaN, and 0 * NaN would reach every feature
-            uint8_t* vrow = gbase + kOffV + s * kSlotBytes + row * 128;
+            // a B_V row past the sequence end may hold NaN, and 0 * NaN would reach every
+            // feature: each of the row's two threads zeroes one 64-feature box of it
+            uint8_t* vrow = gbase + kOffV + s * kSlotBytes + hh * kBox + row * 128;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-              *reinterpret_cast<uint4*>(vrow + cc * 16) = make_uint4(0, 0, 0, 0);
-              *reinterpret_cast<uint4*>(vrow + kBox + cc * 16) = make_uint4(0, 0, 0, 0);
-            }
+            for (int cc = 0; cc < 8; ++cc) *reinterpret_cast<uint4*>(vrow + cc * 16) = make_uint4(0, 0, 0, 0);
           }
         }
         ptx::fence_proxy_async_smem();
@@ -511,22 +559,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (aborted) break;
       // ---- end of the segment: l per head over the CTA, then O^T / l or the partial state
       const float inv_r = 1.f / static_cast<float>(R);  // each token's p was added once per rank row
-      const float lw = reduce_scatter32<false>(lsum, lane);
-      ptx::named_barrier(1, 128);  // the last tile's maxima exchange has finished reading s_red
-      s_red[wq * 32 + lane] = lw;
-      ptx::named_barrier(1, 128);
-      float l[32];
+      const float lw = reduce_scatter16<false>(lsum, lane);
+      ptx::named_barrier(1, kSoftmaxThreads);  // the last tile's maxima exchange has finished reading s_red
+      if (lane < kHalf) s_red[quad * 32 + kHalf * hh + lane] = lw;
+      ptx::named_barrier(1, kSoftmaxThreads);
+      float l[kHalf];
+      combine_quadrants<false>(s_red, hh, l);
 #pragma unroll
-      for (int h4 = 0; h4 < 8; ++h4) {
-        const float4 x0 = reinterpret_cast<const float4*>(s_red)[h4];
-        const float4 x1 = reinterpret_cast<const float4*>(s_red + 32)[h4];
-        const float4 x2 = reinterpret_cast<const float4*>(s_red + 64)[h4];
-        const float4 x3 = reinterpret_cast<const float4*>(s_red + 96)[h4];
-        l[4 * h4] = (x0.x + x1.x + x2.x + x3.x) * inv_r;
-        l[4 * h4 + 1] = (x0.y + x1.y + x2.y + x3.y) * inv_r;
-        l[4 * h4 + 2] = (x0.z + x1.z + x2.z + x3.z) * inv_r;
-        l[4 * h4 + 3] = (x0.w + x1.w + x2.w + x3.w) * inv_r;
-      }
+      for (int h = 0; h < kHalf; ++h) l[h] *= inv_r;
       const int jl = it - 1;  // last tile of the segment
       const bool okf = ptx::mbar_wait_bounded(wfree(jl & 1), (jl >> 1) & 1);
       if (!__all_sync(0xffffffffu, okf)) {
@@ -535,34 +575,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;  // the next tile barrier (or the kernel end) takes every warp out
       }
       ptx::tc_fence_after();
-      uint32_t o0[32], o1[32];
-      ptx::tmem_ld32(tbase + lane_off + kColO, o0);
-      ptx::tmem_ld32(tbase + lane_off + kColO + 32, o1);
+      uint32_t o0[kHalf], o1[kHalf];
+      ptx::tmem_ld16(tbase + lane_off + kColO + kHalf * hh, o0);
+      ptx::tmem_ld16(tbase + lane_off + kColO + 32 + kHalf * hh, o1);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       const bool whole = dec::owner_of(s_pref[b], NT, p.grid) == dec::owner_of(s_pref[b + 1] - 1, NT, p.grid);
       const int d = row;
       if (whole) {
-        float* op = p.out + static_cast<size_t>(b) * kH * kD + d;
+        float* op = p.out + (static_cast<size_t>(b) * kH + kHalf * hh) * kD + d;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
+        for (int h = 0; h < kHalf; ++h) {
           const float o = __uint_as_float(o0[h]) + __uint_as_float(o1[h]);
           op[h * kD] = l[h] > 0.f ? o / l[h] : 0.f;
         }
       } else {
         const int slot = 2 * c + (b == b_first ? 0 : 1);  // a shared sequence is the first or the last one
-        float* op = p.ws_o + static_cast<size_t>(slot) * kH * kD + d;
+        float* op = p.ws_o + (static_cast<size_t>(slot) * kH + kHalf * hh) * kD + d;
 #pragma unroll
-        for (int h = 0; h < 32; ++h) op[h * kD] = __uint_as_float(o0[h]) + __uint_as_float(o1[h]);
-        if (wq == 0) {
+        for (int h = 0; h < kHalf; ++h) op[h * kD] = __uint_as_float(o0[h]) + __uint_as_float(o1[h]);
+        if (quad == 0 && lane < kHalf) {
           float mk = m[0], lk = l[0];
 #pragma unroll
-          for (int h = 1; h < 32; ++h) {
+          for (int h = 1; h < kHalf; ++h) {
             mk = lane == h ? m[h] : mk;
             lk = lane == h ? l[h] : lk;
           }
-          p.ws_ml[(static_cast<size_t>(slot) * kH + lane) * 2] = mk;
-          p.ws_ml[(static_cast<size_t>(slot) * kH + lane) * 2 + 1] = lk;
+          const size_t e = (static_cast<size_t>(slot) * kH + kHalf * hh + lane) * 2;
+          p.ws_ml[e] = mk;
+          p.ws_ml[e + 1] = lk;
         }
       }
     }
@@ -604,8 +645,19 @@ cudaError_t launch_decode_umma(const dec::DecodeTcParams& p, const CacheView& cv
   if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows_v, kH, kRows, 64)) != cudaSuccess) return e;
   if ((e = set_smem_once(cv.r_k)) != cudaSuccess) return e;
   auto kern = cv.r_k == 1 ? decode_umma_kernel<1> : decode_umma_kernel<2>;
-  kern<<<p.grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
-  return cudaGetLastError();
+  // programmatic dependent launch: the CTAs start (barriers, TMEM, tensor maps) while the
+  // preceding kernel drains; the kernel waits for it before its first global access
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p, tbk, tbv, tak, tav);
 }
 
 }  // namespace tpa

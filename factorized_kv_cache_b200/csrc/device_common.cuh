@@ -52,13 +52,15 @@ __device__ __forceinline__ void store16_from_f32(T* __restrict__ p, const float*
   *reinterpret_cast<uint4*>(p) = raw;
 }
 
-// cos/sin of pos * theta, the angle formed and evaluated in double precision
-// (positions reach 2^19, where an fp32 angle would be off by ~0.03 rad).
-// The angle is first reduced by 2*pi (Cody-Waite: 2*pi split into a 32-bit
-// head, so k * head is exact for k < 2^21, and a double tail); the reduced
-// |r| <= pi then takes sincos' short-argument path, which keeps the large
-// positions of long contexts as cheap as small ones.  The reduction is exact
-// up to |pos * theta| < 2^21 * 2*pi (1.3e7 rad) and off by less than 1e-15 rad there.
+// cos/sin of pos * theta.  The angle is formed and reduced by 2*pi in double
+// precision (positions reach 2^19, where an fp32 angle would be off by
+// ~0.03 rad): Cody-Waite with 2*pi split into a 32-bit head, so k * head is
+// exact for k < 2^21, and a double tail.  The reduced |r| <= pi is then
+// rounded to fp32 (error <= 2^-24 pi ~ 1.9e-7 rad) and evaluated with fp32
+// sincosf (within 2 ulp), so the rotation is accurate to ~3e-7 relative: far
+// below one bf16 rounding (2^-9) and the fp32 workload's 1e-5 budget, at a
+// small fraction of a double-precision sincos.  The reduction is exact up
+// to |pos * theta| < 2^21 * 2*pi (1.3e7 rad) and off by less than 1e-15 rad there.
 __device__ __forceinline__ void rope_cos_sin(int pos, double theta, float* c, float* s) {
   const double kTwoPiHi = 0x1.921fb544p+2;             // 2*pi rounded to 32 significant bits
   const double kTwoPiLo = 0x1.0b4611a626331p-32;       // 2*pi - kTwoPiHi
@@ -67,10 +69,7 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double theta, float* c, fl
   const double k = rint(x * kInvTwoPi);
   double r = fma(-k, kTwoPiHi, x);
   r = fma(-k, kTwoPiLo, r);
-  double sd, cd;
-  sincos(r, &sd, &cd);
-  *c = static_cast<float>(cd);
-  *s = static_cast<float>(sd);
+  sincosf(static_cast<float>(r), s, c);
 }
 
 // Rotate the pair (x, y): (x c - y s, x s + y c), in fp32.

@@ -14,8 +14,9 @@
  * Readings where the page is silent (the CPU oracle uses the same ones):
  *   RoPE pairs are adjacent elements (2j, 2j+1), angle = pos * theta_j with
  *   theta_j = rope_base^(-2j/d_h), (x, y) -> (x cos a - y sin a, x sin a + y cos a);
- *   angles are formed and passed to sin/cos in double precision, the rotation
- *   itself runs in fp32 and is rounded once to the storage dtype.
+ *   angles are formed and reduced modulo 2*pi in double precision, the reduced
+ *   angle (|a| <= pi) is evaluated in fp32 (rotation error ~3e-7 relative),
+ *   the rotation itself runs in fp32 and is rounded once to the storage dtype.
  *   The softmax scale is given by the caller (1/sqrt(d_h) in the workloads).
  *
  * Conventions for every call:
