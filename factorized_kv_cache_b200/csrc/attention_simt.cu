@@ -311,32 +311,59 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Merg
 
 // Dense rotated prefill queries (fp32): Q[t][i] = (1/R_Q) sum_j A_Q[t,j,i] RoPE(B_Q[t,j], pos_t)
 // (section 解决思路 for the Q factorization, Theorem 3.1 for RoPE on B_Q).
+// kPrefillQTokens tokens per CTA: one cos/sin per (token, RoPE pair), the rotated B_Q rows and
+// A_Q of those tokens staged in shared memory, then every output float4 computed from them and
+// stored coalesced (the kernel is bound by writing the fp32 queries).
+constexpr int kPrefillQTokens = 4;
+constexpr int kPrefillQThreads = 256;
+
 template <typename T>
-__global__ void prefill_q_kernel(const __grid_constant__ PrefillQArgs a) {
-  extern __shared__ float s_bq[];  // [r_q][head_dim]
-  const int t = blockIdx.x, b = blockIdx.y;
+__global__ void __launch_bounds__(kPrefillQThreads) prefill_q_kernel(const __grid_constant__ PrefillQArgs a) {
+  extern __shared__ float s_q[];
   const int d = a.head_dim, h = a.heads, rq = a.r_q;
-  const size_t tok = static_cast<size_t>(b) * a.n_tokens + t;
-  const int pos = a.q_pos[tok];
-  const T* bq = static_cast<const T*>(a.b_q) + tok * rq * d;
-  for (int e = threadIdx.x; e < rq * d / 2; e += blockDim.x) {
-    const int j = e / (d / 2), p = e % (d / 2);
-    float x = to_f32(bq[j * d + 2 * p]), y = to_f32(bq[j * d + 2 * p + 1]);
-    float cs, sn;
-    rope_cos_sin(pos, a.rope.theta[p], &cs, &sn);
-    rope_pair(x, y, cs, sn);
-    s_bq[j * d + 2 * p] = x;
-    s_bq[j * d + 2 * p + 1] = y;
+  const int b = blockIdx.y;
+  const int t0 = blockIdx.x * kPrefillQTokens;
+  const int nt = min(kPrefillQTokens, a.n_tokens - t0);
+  float2* s_cs = reinterpret_cast<float2*>(s_q);                  // [tokens][d/2]
+  float* s_bq = s_q + kPrefillQTokens * d;                         // [tokens][r_q][d] rotated
+  float* s_aq = s_bq + kPrefillQTokens * rq * d;                   // [tokens][r_q][h]
+  const int pairs = d / 2;
+  for (int e = threadIdx.x; e < nt * pairs; e += blockDim.x) {
+    const int tt = e / pairs, pr = e % pairs;
+    float c, sn;
+    rope_cos_sin(a.q_pos[static_cast<size_t>(b) * a.n_tokens + t0 + tt], a.rope.theta[pr], &c, &sn);
+    s_cs[tt * pairs + pr] = make_float2(c, sn);
+  }
+  const size_t tok0 = static_cast<size_t>(b) * a.n_tokens + t0;
+  const T* aq = static_cast<const T*>(a.a_q) + tok0 * rq * h;
+  for (int e = threadIdx.x; e < nt * rq * h; e += blockDim.x) s_aq[e] = to_f32(aq[e]);
+  __syncthreads();
+  const T* bq = static_cast<const T*>(a.b_q) + tok0 * rq * d;
+  for (int e = threadIdx.x; e < nt * rq * pairs; e += blockDim.x) {
+    const int tt = e / (rq * pairs), pr = e % pairs;
+    float x = to_f32(bq[2 * e]), y = to_f32(bq[2 * e + 1]);
+    const float2 r = s_cs[tt * pairs + pr];
+    rope_pair(x, y, r.x, r.y);
+    s_bq[2 * e] = x;
+    s_bq[2 * e + 1] = y;
   }
   __syncthreads();
-  const T* aq = static_cast<const T*>(a.a_q) + tok * rq * h;
   const float inv_rq = 1.0f / static_cast<float>(rq);
-  float* qo = a.q_out + tok * h * d;
-  for (int e = threadIdx.x; e < h * d; e += blockDim.x) {
-    const int i = e / d, k = e % d;
-    float acc = 0.0f;
-    for (int j = 0; j < rq; ++j) acc = fmaf(to_f32(aq[j * h + i]), s_bq[j * d + k], acc);
-    qo[e] = acc * inv_rq;
+  float4* qo = reinterpret_cast<float4*>(a.q_out + tok0 * h * d);
+  const int per_tok = h * d / 4;
+  for (int e = threadIdx.x; e < nt * per_tok; e += blockDim.x) {
+    const int tt = e / per_tok, r4 = e % per_tok;
+    const int i = (4 * r4) / d, k = (4 * r4) % d;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < rq; ++j) {
+      const float w = s_aq[(tt * rq + j) * h + i];
+      const float4 v = *reinterpret_cast<const float4*>(s_bq + (tt * rq + j) * d + k);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    qo[e] = make_float4(acc.x * inv_rq, acc.y * inv_rq, acc.z * inv_rq, acc.w * inv_rq);
   }
 }
 
@@ -367,12 +394,13 @@ cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_prefill_q(const PrefillQArgs& a, cudaStream_t stream) {
-  dim3 grid(a.n_tokens, a.batch);
-  const size_t smem = static_cast<size_t>(a.r_q) * a.head_dim * sizeof(float);
+  dim3 grid((a.n_tokens + kPrefillQTokens - 1) / kPrefillQTokens, a.batch);
+  const size_t smem = sizeof(float) * kPrefillQTokens *
+                      (static_cast<size_t>(a.head_dim) + static_cast<size_t>(a.r_q) * (a.head_dim + a.heads));
   if (a.dtype == TPA_F32) {
-    prefill_q_kernel<float><<<grid, 128, smem, stream>>>(a);
+    prefill_q_kernel<float><<<grid, kPrefillQThreads, smem, stream>>>(a);
   } else {
-    prefill_q_kernel<__nv_bfloat16><<<grid, 128, smem, stream>>>(a);
+    prefill_q_kernel<__nv_bfloat16><<<grid, kPrefillQThreads, smem, stream>>>(a);
   }
   return cudaGetLastError();
 }

@@ -12,32 +12,34 @@
 //   O[t, i, :]  = sum_(s,r) W[t, (s,r)] B_V[s, r, :]         (tensor cores)
 // The dense per-head query is the only thing expanded: it is built once per
 // chunk in fp32 by prefill_q_kernel and split by the softmax threads into
-// bf16 high and low parts in shared memory.  Keys and values stay
-// factorized: the score MMA contracts the query with B_K rows, and the value
-// MMA contracts the softmax weights with B_V rows.  Putting the head factors
-// on the query side of the MMA (a dense Q tile per head) costs 2 h d_h R_K
-// tensor flops per (query, key) pair and little CUDA-core work; contracting
-// B_Q with B_K first would save tensor flops but needs ~h R_Q R_K CUDA-core
-// FMAs per pair to apply A_Q and A_K, which is slower on this machine.
+// bf16 high and low parts in TMEM.  Keys and values stay factorized: the
+// score MMA contracts the query with B_K rows, and the value MMA contracts
+// the softmax weights with B_V rows.  Putting the head factors on the query
+// side of the MMA (a dense Q tile per head) costs 2 h d_h R_K tensor flops
+// per (query, key) pair and little CUDA-core work; contracting B_Q with B_K
+// first would save tensor flops but needs ~h R_Q R_K CUDA-core FMAs per pair
+// to apply A_Q and A_K, which is slower on this machine.
 //
-// CTA = (sequence, pair of heads, tile of 128 queries); heavy (late) query
-// tiles are dispatched first.  The two heads share every key/value tile and
-// take turns on the tensor cores while the other one runs its softmax.
-// Roles (352 threads): warp 0 issues TMA loads of 64-row key tiles {B_K, the
-// 8-head slice of A_K holding both heads} into a 3-slot ring and value tiles
-// {B_V, A_V slice} into a 2-slot ring; warp 1 allocates all 512 TMEM columns
-// and one of its threads issues the MMAs; warps 2-5 (head 0) and 6-9
-// (head 1) own one query row each (one TMEM lane); warp 10 stages both
-// heads' A_K, A_V of a tile as fp32 (scale folded in) and zeroes B_V rows
-// past the sequence end, which may hold NaN.
-// TMEM per head h: S double-buffered in columns [256 h + 64 b, +64), then
-// overwritten in place by W as bf16 hi (first 32 columns) and lo (next 32);
-// O in [256 h + 128, +128).  Per key tile j and head:
-//   S = (Q_hi + Q_lo) B_K^T  (M = 128 queries, N = 64 rows, K = 128; both
-//       operands in shared memory, K-major, 128-byte swizzle);
+// CTA = (sequence, head, tile of 128 queries); heavy (late) query tiles are
+// dispatched first.  Both MMAs take their A operand from TMEM, so shared
+// memory only feeds their B operands (a 128-row B_K or B_V tile per 16 of K).
+// Roles (352 threads): warp 0 issues TMA loads of 128-row tiles {B_K, B_V,
+// the 8-head slices of A_K and A_V holding the head} into a 3-stage ring;
+// warp 1 allocates all 512 TMEM columns and one of its threads issues the
+// MMAs; warps 2-9 run the softmax, two threads per query row (TMEM lane):
+// warps 2-5 take the first 64 cache rows of a tile, warps 6-9 the last 64;
+// warp 10 stages A_K and A_V of the head as fp32 (scale folded in) and zeroes
+// B_V rows past the sequence end, which may hold NaN.
+// TMEM: S double-buffered in columns [128 b, +128) and overwritten in place by
+// W as bf16 hi (first 64 columns) and lo (next 64), O in [256, 384), the
+// query hi in [384, 448) and lo in [448, 512).  Per key tile j:
+//   S = (Q_hi + Q_lo) B_K^T  (M = 128 queries, N = 128 rows, K = 128), into
+//       the buffer that tile j - 1 does not use, so it overlaps the softmax
+//       of tile j - 1;
 //   softmax: A_K weighting, causal mask, online softmax with a lazily
-//       rescaled maximum (only when it grows by more than 2^8), W = p A_V;
-//   O += W_hi B_V + W_lo B_V  (A from TMEM, B_V MN-major).
+//       rescaled maximum (only when it grows by more than 2^8; the two
+//       threads of a row share their maxima through shared memory), W = p A_V;
+//   O += W_hi B_V + W_lo B_V  (B_V MN-major).
 // Both the query and W are split into two bf16 parts, which keeps them to
 // ~16 bits: one bf16 rounding of either costs ~3.5e-3 relative error on the
 // prefill workload, above its 2e-3 budget.  Every wait is bounded (2 s);
@@ -60,38 +62,36 @@ namespace {
 constexpr int kH = 32;
 constexpr int kD = 128;
 constexpr int kQ = 128;                 // queries per CTA
-constexpr int kRows = 64;               // cache rows per key tile
-constexpr int kKSlots = 3;
-constexpr int kVSlots = 2;
+constexpr int kRows = 128;              // cache rows per key tile
+constexpr int kHalfRows = kRows / 2;    // rows per softmax thread
+constexpr int kStages = 3;
 constexpr int kSoftmaxWarps = 8;
 constexpr int kThreads = (3 + kSoftmaxWarps) * 32;
 constexpr int kStagerWarp = 2 + kSoftmaxWarps;
-constexpr int kBBox = kRows * 128;        // 64 features x 64 rows, bf16: 8 KB
+constexpr int kBBox = kRows * 128;        // 64 features x 128 rows, bf16: 16 KB
 constexpr int kBBytes = 2 * kBBox;        // one B tile
 constexpr int kASlice = 8;                // heads in the A slice a tile carries (16 bytes per row)
 constexpr int kABytes = kRows * kASlice * 2;
-constexpr int kSlotBytes = kBBytes + kABytes;  // 17 KB
-constexpr int kQBox = kQ * 128;           // 128 queries x 64 features, bf16: 16 KB
-constexpr int kQHead = 4 * kQBox;         // hi (2 boxes) then lo (2 boxes)
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + kKSlots * kSlotBytes;
-constexpr int kOffQ = kOffV + kVSlots * kSlotBytes;
-constexpr int kOffA = kOffQ + 2 * kQHead;  // fp32 [2 buffers][4: A_K h0, A_K h1, A_V h0, A_V h1][64]
-constexpr int kOffBar = kOffA + 2 * 4 * kRows * 4;
-// kfull[3], kempty[3], vfull[2], vempty[2], sfull[2 heads][2], wready[2][2], odone[2], staged[2], qready, fin
-constexpr int kNumBars = 2 * kKSlots + 2 * kVSlots + 4 + 4 + 2 + 2 + 1 + 1;
+constexpr int kStageBytes = 2 * kBBytes + 2 * kABytes;  // B_K, B_V, A_K slice, A_V slice
+constexpr int kOffStages = 0;
+constexpr int kOffA = kOffStages + kStages * kStageBytes;  // fp32 [2 buffers][A_K, A_V][128]
+constexpr int kOffMx = kOffA + 2 * 2 * kRows * 4;          // fp32 [2 buffers][2 halves][128 rows]
+constexpr int kOffL = kOffMx + 2 * 2 * kQ * 4;             // fp32 [2 halves][128 rows]
+constexpr int kOffBar = kOffL + 2 * kQ * 4;
+// full[3], empty[3], sfull[2], wready[2], odone, staged[2], qready, fin
+constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 1 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-static_assert(kSlotBytes % 1024 == 0 && kQBox % 1024 == 0 && kOffQ % 1024 == 0, "swizzle atoms stay aligned");
+static_assert(kStageBytes % 1024 == 0 && kBBox % 1024 == 0, "swizzle atoms stay aligned");
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256, kColQ = 384;
 constexpr unsigned kErrTimeout = 0x8u;
 
-// kind::f16 instruction descriptors, D fp32, A and B bf16, M = 128:
-// score MMA N = 64 (both K-major); value MMA N = 128 with B (the B_V tile) MN-major.
-constexpr uint32_t kIdescScore = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescValue =
-    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// kind::f16 instruction descriptors, D fp32, A (TMEM) and B bf16, M = 128, N = 128;
+// the value MMA's B (the B_V tile) is MN-major.
+constexpr uint32_t kIdescScore = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescValue = kIdescScore | (1u << 16);
 
 struct PrefillTcParams {
   const int32_t* seq_lens;
@@ -108,62 +108,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ PrefillTcParams p,
                       const __grid_constant__ CUtensorMap tm_bk, const __grid_constant__ CUtensorMap tm_bv,
                       const __grid_constant__ CUtensorMap tm_ak, const __grid_constant__ CUtensorMap tm_av) {
-  constexpr int TOK = kRows / R;  // tokens per key tile
+  constexpr int TOK = kRows / R;           // tokens per key tile
+  constexpr int TOKH = kHalfRows / R;      // tokens per softmax thread
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (sbase - raw);
   float* s_a = reinterpret_cast<float*>(gbase + kOffA);
+  float* s_mx = reinterpret_cast<float*>(gbase + kOffMx);
+  float* s_l = reinterpret_cast<float*>(gbase + kOffL);
   const uint32_t bar0 = sbase + kOffBar;
-  auto kfull = [&](int s) { return bar0 + 8 * s; };
-  auto kempty = [&](int s) { return bar0 + 8 * (kKSlots + s); };
-  auto vfull = [&](int s) { return bar0 + 8 * (2 * kKSlots + s); };
-  auto vempty = [&](int s) { return bar0 + 8 * (2 * kKSlots + kVSlots + s); };
-  constexpr int kB1 = 2 * kKSlots + 2 * kVSlots;
-  auto sfull = [&](int h, int b) { return bar0 + 8 * (kB1 + 2 * h + b); };
-  auto wready = [&](int h, int b) { return bar0 + 8 * (kB1 + 4 + 2 * h + b); };
-  auto odone = [&](int h) { return bar0 + 8 * (kB1 + 8 + h); };
-  auto staged = [&](int b) { return bar0 + 8 * (kB1 + 10 + b); };
-  const uint32_t qready = bar0 + 8 * (kB1 + 12);
-  const uint32_t fin = bar0 + 8 * (kB1 + 13);
+  auto full = [&](int s) { return bar0 + 8 * s; };
+  auto empty = [&](int s) { return bar0 + 8 * (kStages + s); };
+  auto sfull = [&](int b) { return bar0 + 8 * (2 * kStages + b); };
+  auto wready = [&](int b) { return bar0 + 8 * (2 * kStages + 2 + b); };
+  const uint32_t odone = bar0 + 8 * (2 * kStages + 4);
+  auto staged = [&](int b) { return bar0 + 8 * (2 * kStages + 5 + b); };
+  const uint32_t qready = bar0 + 8 * (2 * kStages + 7);
+  const uint32_t fin = bar0 + 8 * (2 * kStages + 8);
   volatile uint32_t* s_taddr = reinterpret_cast<volatile uint32_t*>(gbase + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // heavy query tiles first: blockIdx.y runs over query tiles from the last one down
   const int qt = p.n_qtiles - 1 - static_cast<int>(blockIdx.y);
-  const int hp = blockIdx.x % (kH / 2);  // heads 2 hp, 2 hp + 1
-  const int b = blockIdx.x / (kH / 2);
+  const int head = blockIdx.x % kH;
+  const int b = blockIdx.x / kH;
   const int q0 = qt * kQ;
   const int len = p.seq_lens[b];
   const int P = len - p.n_tokens;
   if (len > p.capacity || P < 0) {
-    if (tid == 0 && hp == 0 && qt == 0) atomicOr(p.err, TPA_DEVERR_PREFILL_LEN);
+    if (tid == 0 && head == 0 && qt == 0) atomicOr(p.err, TPA_DEVERR_PREFILL_LEN);
     return;
   }
   const int q_hi = min(q0 + kQ, p.n_tokens);  // queries [q0, q_hi) are real
   const int key_end = P + q_hi;                // keys [0, key_end) are needed
   const int nk = (key_end + TOK - 1) / TOK;
-  const int a_x = kASlice * ((2 * hp) / kASlice);  // first head of the A slice
-  const int a_off = 2 * hp - a_x;                   // heads 2 hp, 2 hp + 1 within the slice
+  const int a_x = kASlice * (head / kASlice);  // first head of the A slice
+  const int a_off = head - a_x;                 // the head within the slice
 
   if (tid == 0) {
-    for (int s = 0; s < kKSlots; ++s) {
-      ptx::mbar_init(kfull(s), 1);
-      ptx::mbar_init(kempty(s), 2);  // score-MMA commit + the stager (A_K read)
+    for (int s = 0; s < kStages; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), 2);  // value-MMA commit + the stager (A slices read, B_V rows zeroed)
     }
-    for (int s = 0; s < kVSlots; ++s) {
-      ptx::mbar_init(vfull(s), 1);
-      ptx::mbar_init(vempty(s), 2);  // value-MMA commit + the stager (A_V read, B_V rows zeroed)
+    for (int bf = 0; bf < 2; ++bf) {
+      ptx::mbar_init(sfull(bf), 1);
+      ptx::mbar_init(wready(bf), kSoftmaxWarps);
+      ptx::mbar_init(staged(bf), 1);
     }
-    for (int h = 0; h < 2; ++h) {
-      for (int bf = 0; bf < 2; ++bf) {
-        ptx::mbar_init(sfull(h, bf), 1);
-        ptx::mbar_init(wready(h, bf), 4);
-      }
-      ptx::mbar_init(odone(h), 1);
-      ptx::mbar_init(staged(h), 1);
-    }
+    ptx::mbar_init(odone, 1);
     ptx::mbar_init(qready, kSoftmaxWarps);
     ptx::mbar_init(fin, 1);
     *s_abort = 0;
@@ -185,103 +179,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_bv);
       ptx::prefetch_tmap(&tm_ak);
       ptx::prefetch_tmap(&tm_av);
-      int k_issued = 0, v_issued = 0;
+      int issued = 0;
       bool ok = true;
-      for (int j = 0; j < nk && ok; ++j) {
+      for (int j = 0; j < nk; ++j) {
         if (*s_abort) {
           ok = false;
           break;
         }
+        const int st = j % kStages;
+        if (j >= kStages && !(ok = ptx::mbar_wait_bounded(empty(st), ((j / kStages) & 1) ^ 1))) break;
         const int row0 = (b * p.capacity + j * TOK) * R;
-        const int ks = j % kKSlots, vs = j % kVSlots;
-        if (j >= kKSlots && !(ok = ptx::mbar_wait_bounded(kempty(ks), ((j / kKSlots) & 1) ^ 1))) break;
-        const uint32_t kb = sbase + kOffK + ks * kSlotBytes;
-        ptx::mbar_arrive_expect_tx(kfull(ks), kSlotBytes);
-        ptx::tma_load_2d(kb, &tm_bk, 0, row0, kfull(ks));
-        ptx::tma_load_2d(kb + kBBox, &tm_bk, 64, row0, kfull(ks));
-        ptx::tma_load_2d(kb + kBBytes, &tm_ak, a_x, row0, kfull(ks));
-        ++k_issued;
-        if (j >= kVSlots && !(ok = ptx::mbar_wait_bounded(vempty(vs), ((j / kVSlots) & 1) ^ 1))) break;
-        const uint32_t vb = sbase + kOffV + vs * kSlotBytes;
-        ptx::mbar_arrive_expect_tx(vfull(vs), kSlotBytes);
-        ptx::tma_load_2d(vb, &tm_bv, 0, row0, vfull(vs));
-        ptx::tma_load_2d(vb + kBBox, &tm_bv, 64, row0, vfull(vs));
-        ptx::tma_load_2d(vb + kBBytes, &tm_av, a_x, row0, vfull(vs));
-        ++v_issued;
+        const uint32_t sb = sbase + kOffStages + st * kStageBytes;
+        ptx::mbar_arrive_expect_tx(full(st), kStageBytes);
+        ptx::tma_load_2d(sb, &tm_bk, 0, row0, full(st));
+        ptx::tma_load_2d(sb + kBBox, &tm_bk, 64, row0, full(st));
+        ptx::tma_load_2d(sb + kBBytes, &tm_bv, 0, row0, full(st));
+        ptx::tma_load_2d(sb + kBBytes + kBBox, &tm_bv, 64, row0, full(st));
+        ptx::tma_load_2d(sb + 2 * kBBytes, &tm_ak, a_x, row0, full(st));
+        ptx::tma_load_2d(sb + 2 * kBBytes + kABytes, &tm_av, a_x, row0, full(st));
+        ++issued;
       }
       if (!ok) {
         if (!*s_abort) atomicOr(p.err, kErrTimeout);
         *s_abort = 1;
         // every load already issued lands before the CTA can exit
-        for (int k = max(0, k_issued - kKSlots); k < k_issued; ++k)
-          ptx::mbar_wait_bounded(kfull(k % kKSlots), (k / kKSlots) & 1);
-        for (int k = max(0, v_issued - kVSlots); k < v_issued; ++k)
-          ptx::mbar_wait_bounded(vfull(k % kVSlots), (k / kVSlots) & 1);
+        for (int k = max(0, issued - kStages); k < issued; ++k)
+          ptx::mbar_wait_bounded(full(k % kStages), (k / kStages) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Iteration j: the score MMAs of tile j for both heads, then the value MMAs of
-    // tile j - 1 (whose W the softmax warps are finishing meanwhile).
+    // Order: S(0); then for each tile j: S(j+1) into the other buffer (after the value MMA
+    // of tile j-1 has consumed the W stored there), then O += W(j) B_V once the softmax of
+    // tile j is done.  The score MMA of tile j+1 thus runs while the softmax works on tile j.
     if (lane == 0) {
-      auto score = [&](int h, int j) {
-        const uint32_t kb = sbase + kOffK + (j % kKSlots) * kSlotBytes;
-        const uint32_t qb = sbase + kOffQ + h * kQHead;
+      auto score = [&](int j) {
+        const uint32_t sb = sbase + kOffStages + (j % kStages) * kStageBytes;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {  // query hi, then query lo
 #pragma unroll
           for (int k = 0; k < 8; ++k) {         // K = 128 features in steps of 16
-            const uint64_t da =
-                ptx::umma_desc_sw128(qb + half * 2 * kQBox + (k >> 2) * kQBox + (k & 3) * 32, 16, 1024);
-            const uint64_t db = ptx::umma_desc_sw128(kb + (k >> 2) * kBBox + (k & 3) * 32, 16, 1024);
-            ptx::umma_ss(tbase + 256u * h + 64u * (j & 1), da, db, kIdescScore, (half > 0 || k > 0) ? 1u : 0u);
+            const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBBox + (k & 3) * 32, 16, 1024);
+            ptx::umma_ts(tbase + 128u * (j & 1), tbase + kColQ + half * 64 + k * 8, db, kIdescScore,
+                         (half > 0 || k > 0) ? 1u : 0u);
           }
         }
-        ptx::umma_commit(sfull(h, j & 1));
+        ptx::umma_commit(sfull(j & 1));
       };
-      auto value = [&](int h, int j) {
-        const uint32_t vb = sbase + kOffV + (j % kVSlots) * kSlotBytes;
-        const uint32_t ts = tbase + 256u * h + 64u * (j & 1);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {    // W hi, then W lo
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {        // K = 64 cache rows in steps of 16
-            const uint64_t db = ptx::umma_desc_sw128(vb + kk * 2048, kBBox, 1024);
-            ptx::umma_ts(tbase + 256u * h + 128u, ts + 32u * half + 8u * kk, db, kIdescValue,
-                         (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        ptx::umma_commit(odone(h));
-      };
-      bool ok = ptx::mbar_wait_bounded(qready, 0);
-      for (int j = 0; j <= nk && ok; ++j) {
+      bool ok = ptx::mbar_wait_bounded(qready, 0) && ptx::mbar_wait_bounded(full(0), 0);
+      if (ok) {
+        ptx::tc_fence_after();
+        score(0);
+      }
+      for (int j = 0; j < nk && ok; ++j) {
         if (*s_abort) {
           ok = false;
           break;
         }
-        if (j < nk) {
-          if (!(ok = ptx::mbar_wait_bounded(kfull(j % kKSlots), (j / kKSlots) & 1))) break;
-          for (int h = 0; h < 2 && ok; ++h) {
-            // S buffer (j & 1) is free once the value MMA of tile j - 2 has read its W
-            if (j >= 2) ok = ptx::mbar_wait_bounded(odone(h), (j - 2) & 1);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            score(h, j);
-          }
+        if (j + 1 < nk) {
+          ok = ptx::mbar_wait_bounded(full((j + 1) % kStages), ((j + 1) / kStages) & 1);
+          if (ok && j > 0) ok = ptx::mbar_wait_bounded(odone, (j - 1) & 1);
           if (!ok) break;
-          ptx::umma_commit(kempty(j % kKSlots));
+          ptx::tc_fence_after();
+          score(j + 1);
         }
-        if (j >= 1) {
-          const int jv = j - 1;
-          if (!(ok = ptx::mbar_wait_bounded(vfull(jv % kVSlots), (jv / kVSlots) & 1))) break;
-          for (int h = 0; h < 2 && ok; ++h) {
-            if (!(ok = ptx::mbar_wait_bounded(wready(h, jv & 1), (jv >> 1) & 1))) break;
-            ptx::tc_fence_after();
-            value(h, jv);
+        if (!(ok = ptx::mbar_wait_bounded(wready(j & 1), (j >> 1) & 1))) break;
+        ptx::tc_fence_after();
+        const uint32_t bv = sbase + kOffStages + (j % kStages) * kStageBytes + kBBytes;
+        const uint32_t ts = tbase + 128u * (j & 1);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {    // W hi, then W lo
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {        // K = 128 cache rows in steps of 16
+            const uint64_t db = ptx::umma_desc_sw128(bv + kk * 2048, kBBox, 1024);
+            ptx::umma_ts(tbase + kColO, ts + half * 64 + kk * 8, db, kIdescValue,
+                         (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
           }
-          if (!ok) break;
-          ptx::umma_commit(vempty(jv % kVSlots));
         }
+        ptx::umma_commit(odone);
+        ptx::umma_commit(empty(j % kStages));
       }
       if (!ok) {
         if (!*s_abort) atomicOr(p.err, kErrTimeout);
@@ -293,18 +269,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kStagerWarp) {
     // ------------------------------------------------------------ A stager
-    // Per tile: A_K (times scale log2(e)/R_K) and A_V (times 1/R_V) of both heads as fp32
-    // rows of 64, zero past the sequence end, where B_V rows are zeroed as well.
+    // Per tile: A_K (times scale log2(e)/R_K) and A_V (times 1/R_V) of the head as fp32
+    // rows of 128, zero past the sequence end, where B_V rows are zeroed as well.
     const int valid_rows_all = len * R;
     for (int j = 0; j < nk; ++j) {
       if (__any_sync(0xffffffffu, *s_abort != 0)) break;  // the whole warp leaves together
-      const int ks = j % kKSlots, vs = j % kVSlots, ab = j & 1;
-      bool ok = ptx::mbar_wait_bounded(kfull(ks), (j / kKSlots) & 1) &&
-                ptx::mbar_wait_bounded(vfull(vs), (j / kVSlots) & 1);
-      // the softmax warps of both heads are done with buffer ab (tile j - 2)
-      if (ok && j >= 2)
-        ok = ptx::mbar_wait_bounded(wready(0, ab), ((j - 2) >> 1) & 1) &&
-             ptx::mbar_wait_bounded(wready(1, ab), ((j - 2) >> 1) & 1);
+      const int st = j % kStages, ab = j & 1;
+      bool ok = ptx::mbar_wait_bounded(full(st), (j / kStages) & 1);
+      // both softmax halves are done with buffer ab (tile j - 2)
+      if (ok && j >= 2) ok = ptx::mbar_wait_bounded(wready(ab), ((j - 2) >> 1) & 1);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) {
           atomicOr(p.err, kErrTimeout);
@@ -312,27 +285,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         break;
       }
-      const uint8_t* ka = gbase + kOffK + ks * kSlotBytes + kBBytes;
-      uint8_t* vslot = gbase + kOffV + vs * kSlotBytes;
-      const uint8_t* va = vslot + kBBytes;
-      float* sa = s_a + ab * 4 * kRows;
+      uint8_t* sb = gbase + kOffStages + st * kStageBytes;
+      const uint8_t* ka = sb + 2 * kBBytes;
+      const uint8_t* va = ka + kABytes;
+      float* sa = s_a + ab * 2 * kRows;
       bool zeroed = false;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int r = lane + 32 * half;
+      for (int u = 0; u < kRows / 32; ++u) {
+        const int r = lane + 32 * u;
         const bool valid = j * kRows + r < valid_rows_all;
-        const uint32_t k2 = *reinterpret_cast<const uint32_t*>(ka + r * 16 + a_off * 2);
-        const uint32_t v2 = *reinterpret_cast<const uint32_t*>(va + r * 16 + a_off * 2);
-        sa[0 * kRows + r] = valid ? ptx::bf16_lo(k2) * p.zs : 0.f;
-        sa[1 * kRows + r] = valid ? ptx::bf16_hi(k2) * p.zs : 0.f;
-        sa[2 * kRows + r] = valid ? ptx::bf16_lo(v2) * p.inv_rv : 0.f;
-        sa[3 * kRows + r] = valid ? ptx::bf16_hi(v2) * p.inv_rv : 0.f;
+        const float ak = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(ka + r * 16 + a_off * 2));
+        const float av = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(va + r * 16 + a_off * 2));
+        sa[r] = valid ? ak * p.zs : 0.f;
+        sa[kRows + r] = valid ? av * p.inv_rv : 0.f;
         if (!valid) {
           // a B_V row past the sequence end may hold NaN; 0 * NaN would reach every O row
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4*>(vslot + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(vslot + kBBox + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sb + kBBytes + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sb + kBBytes + kBBox + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
           }
           zeroed = true;
         }
@@ -341,44 +312,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) {
         ptx::mbar_arrive(staged(ab));
-        ptx::mbar_arrive(kempty(ks));
-        ptx::mbar_arrive(vempty(vs));
+        ptx::mbar_arrive(empty(st));
       }
     }
   } else {
     // ------------------------------------------------------------ softmax warps
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
-    const int h = (warp - 2) >> 2;             // head 2 hp + h
-    const int head = 2 * hp + h;
-    const int row = quad * 32 + lane;          // query row within the tile
+    const int hf = (warp - 2) >> 2;            // this thread's half of each key tile
+    const int row = quad * 32 + lane;          // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int tq = q0 + row;                   // query index in the chunk
     const int qslot = P + tq;                  // its cache slot: keys s <= qslot
-    const uint32_t t_o = tbase + 256u * h + 128u;
-    // stage this thread's query row as bf16 hi + lo (K-major, 128-byte swizzle; zeros past the chunk)
+    const uint32_t pair_bar = 1 + quad;        // named barrier of warps (quad, half 0) and (quad, half 1)
+    // stage features [64 hf, +64) of this thread's query row as bf16 hi + lo in TMEM
     {
-      const float* qr = p.q + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD;
-      uint8_t* qh = gbase + kOffQ + h * kQHead;
+      const float* qr = p.q + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD + 64 * hf;
+      uint32_t hi[32], lo[32];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {           // 16 chunks of 8 features
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (tq < p.n_tokens) {
-          v0 = *reinterpret_cast<const float4*>(qr + 8 * c);
-          v1 = *reinterpret_cast<const float4*>(qr + 8 * c + 4);
-        }
-        const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hi[e] = ptx::pack_bf16(f[2 * e], f[2 * e + 1]);
-          lo[e] = ptx::pack_bf16(f[2 * e] - ptx::bf16_lo(hi[e]), f[2 * e + 1] - ptx::bf16_hi(hi[e]));
-        }
-        const int box = c >> 3, chunk = c & 7;
-        const int off = box * kQBox + row * 128 + ((chunk ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(qh + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(qh + 2 * kQBox + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      for (int c = 0; c < 16; ++c) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (tq < p.n_tokens) v = *reinterpret_cast<const float4*>(qr + 4 * c);
+        hi[2 * c] = ptx::pack_bf16(v.x, v.y);
+        hi[2 * c + 1] = ptx::pack_bf16(v.z, v.w);
+        lo[2 * c] = ptx::pack_bf16(v.x - ptx::bf16_lo(hi[2 * c]), v.y - ptx::bf16_hi(hi[2 * c]));
+        lo[2 * c + 1] = ptx::pack_bf16(v.z - ptx::bf16_lo(hi[2 * c + 1]), v.w - ptx::bf16_hi(hi[2 * c + 1]));
       }
-      ptx::fence_proxy_async_smem();
+      ptx::tmem_st32(tbase + lane_off + kColQ + 32 * hf, hi);
+      ptx::tmem_st32(tbase + lane_off + kColQ + 64 + 32 * hf, lo);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(qready);
     }
@@ -387,10 +349,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nk; ++j) {
       const int ab = j & 1;
       bool fail = *s_abort != 0;
-      if (!fail)
-        fail = !ptx::mbar_wait_bounded(sfull(h, ab), (j >> 1) & 1) ||
-               !ptx::mbar_wait_bounded(staged(ab), (j >> 1) & 1);
-      if (!__all_sync(0xffffffffu, !fail)) {  // warp-wide TMEM accesses follow: leave together
+      if (!fail) fail = !ptx::mbar_wait_bounded(sfull(ab), (j >> 1) & 1) || !ptx::mbar_wait_bounded(staged(ab), (j >> 1) & 1);
+      fail = !__all_sync(0xffffffffu, !fail);  // warp-uniform: warp-wide TMEM loads follow
+      ptx::tc_fence_after();
+      const float* ak = s_a + ab * 2 * kRows + kHalfRows * hf;          // scaled A_K of this thread's rows
+      const float* av = s_a + ab * 2 * kRows + kRows + kHalfRows * hf;  // A_V / R_V of this thread's rows
+      const uint32_t ts = tbase + 128u * ab + lane_off;
+      // ---- scores: z[s] for this thread's TOKH tokens (log2 units)
+      float z[TOKH];
+      float mx = -INFINITY;
+      if (!fail) {
+        uint32_t sv[2][32];
+        ptx::tmem_ld32(ts + kHalfRows * hf, sv[0]);
+        ptx::tmem_ld32(ts + kHalfRows * hf + 32, sv[1]);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 a4 = reinterpret_cast<const float4*>(ak + 32 * c2)[e4];
+            const float a[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int u = 0; u < 4; u += R) {
+              const int e = 4 * e4 + u;  // row within this 32-row chunk
+              float acc = __uint_as_float(sv[c2][e]) * a[u];
+              if (R == 2) acc = fmaf(__uint_as_float(sv[c2][e + 1]), a[u + 1], acc);
+              z[(32 * c2 + e) / R] = acc;
+            }
+          }
+        }
+        const int tok0 = j * TOK + TOKH * hf;  // first token of this thread's rows
+        const bool need_mask = j * TOK + TOK - 1 > P + q0;  // the tile reaches past some query's own slot
+#pragma unroll
+        for (int s = 0; s < TOKH; ++s) {
+          if (need_mask && tok0 + s > qslot) z[s] = -INFINITY;
+          mx = fmaxf(mx, z[s]);
+        }
+      }
+      // ---- the row maximum over both halves of the tile: exchange with the partner thread.
+      // The pair barrier also orders both threads' S loads before either writes W over S, and
+      // carries the abort decision, so that both warps of the pair leave at the same tile.
+      float* mxbuf = s_mx + ab * 2 * kQ;
+      mxbuf[hf * kQ + row] = mx;
+      if (ptx::named_barrier_or(pair_bar, 64, fail)) {
         if (lane == 0) {
           atomicOr(p.err, kErrTimeout);
           *s_abort = 1;
@@ -398,66 +399,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      ptx::tc_fence_after();
-      const float* ak = s_a + ab * 4 * kRows + h * kRows;        // scaled A_K of this head, per row
-      const float* av = s_a + ab * 4 * kRows + (2 + h) * kRows;  // A_V / R_V of this head, per row
-      const uint32_t ts = tbase + 256u * h + 64u * ab + lane_off;
-      // ---- scores: z[s] for the TOK tokens of the tile (log2 units)
-      float z[TOK];
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t sv[32];
-        ptx::tmem_ld32(ts + 32 * c2, sv);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 a4 = reinterpret_cast<const float4*>(ak + 32 * c2)[e4];
-          const float a[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-          for (int u = 0; u < 4; u += R) {
-            const int e = 4 * e4 + u;  // row within this 32-row chunk
-            float acc = __uint_as_float(sv[e]) * a[u];
-            if (R == 2) acc = fmaf(__uint_as_float(sv[e + 1]), a[u + 1], acc);
-            z[(32 * c2 + e) / R] = acc;
-          }
-        }
-      }
-      const int tok0 = j * TOK;
-      const bool need_mask = tok0 + TOK - 1 > P + q0;  // the tile reaches past some query's own slot
-      float mx = -INFINITY;
-#pragma unroll
-      for (int s = 0; s < TOK; ++s) {
-        if (need_mask && tok0 + s > qslot) z[s] = -INFINITY;
-        mx = fmaxf(mx, z[s]);
-      }
-      // ---- online softmax with a lazily rescaled maximum; the TMEM rescale of O is a
-      // warp-wide operation, so the whole warp runs it when any of its rows needs it
+      mx = fmaxf(mx, mxbuf[(1 - hf) * kQ + row]);
+      // ---- online softmax with a lazily rescaled maximum; both threads of a row take the same
+      // decision, and the warp-wide TMEM rescale of O runs when any row of the warp needs it
       const bool grow = mx > m + 8.f || (m == -INFINITY && mx != -INFINITY);
-      const float alpha = !grow ? 1.f : (m == -INFINITY ? 0.f : exp2f(m - mx));
+      const float alpha = !grow ? 1.f : (m == -INFINITY ? 0.f : ptx::ex2(m - mx));
       if (grow) {
         l *= alpha;
         m = mx;
       }
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        // the value MMA of tile j-1 may still be accumulating into O
-        const bool o_prev = ptx::mbar_wait_bounded(odone(h), (j - 1) & 1);
-        if (!__all_sync(0xffffffffu, o_prev)) {
-          if (lane == 0) {
-            atomicOr(p.err, kErrTimeout);
-            *s_abort = 1;
+        // the value MMA of tile j-1 may still be accumulating into O; a timeout here is
+        // acted on at the next pair barrier, which both warps of the pair reach
+        const bool o_prev = ptx::mbar_wait_bounded(odone, (j - 1) & 1);
+        if (__all_sync(0xffffffffu, o_prev)) {
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int c2 = 0; c2 < 2; ++c2) {  // this thread's 64 columns of O
+            uint32_t ov[32];
+            const uint32_t col = tbase + lane_off + kColO + 64 * hf + 32 * c2;
+            ptx::tmem_ld32(col, ov);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            ptx::tmem_st32(col, ov);
           }
-          ok = false;
-          break;
-        }
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t ov[32];
-          ptx::tmem_ld32(t_o + lane_off + c4 * 32, ov);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          ptx::tmem_st32(t_o + lane_off + c4 * 32, ov);
+        } else if (lane == 0) {
+          atomicOr(p.err, kErrTimeout);
+          *s_abort = 1;
         }
       }
       // ---- W = p A_V / R_V as bf16 hi + lo, two cache rows per TMEM column, over S
@@ -468,12 +437,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float a[4] = {a4.x, a4.y, a4.z, a4.w};
         float w[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int rr = 4 * e4 + u;
-          const int s = rr / R;
-          const float pz = exp2f(z[s] - m);  // 0 for masked keys (z = -inf, m finite)
-          w[u] = pz * a[u];
-          if (rr % R == 0) l += pz;
+        for (int u = 0; u < 4; u += R) {
+          const int s = (4 * e4 + u) / R;
+          const float pz = ptx::ex2(z[s] - m);  // 0 for masked keys (z = -inf, m finite)
+          l += pz;
+#pragma unroll
+          for (int r = 0; r < R; ++r) w[u + r] = pz * a[u + r];
         }
         whi[2 * e4] = ptx::pack_bf16(w[0], w[1]);
         whi[2 * e4 + 1] = ptx::pack_bf16(w[2], w[3]);
@@ -481,28 +450,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         wlo[2 * e4 + 1] =
             ptx::pack_bf16(w[2] - ptx::bf16_lo(whi[2 * e4 + 1]), w[3] - ptx::bf16_hi(whi[2 * e4 + 1]));
       }
-      ptx::tmem_st32(ts, whi);
-      ptx::tmem_st32(ts + 32, wlo);
+      ptx::tmem_st32(ts + 32 * hf, whi);
+      ptx::tmem_st32(ts + 64 + 32 * hf, wlo);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(wready(h, ab));
+      if (lane == 0) ptx::mbar_arrive(wready(ab));
     }
-    // ---- epilogue: O / l to out[b][t][head][:] once every MMA of this CTA has completed
+    // ---- epilogue: the row sum over both halves, then O / l to out[b][t][head][:]
+    // (this thread's 64 features) once every MMA of this CTA has completed
+    if (ok) {  // both warps of the pair finished the loop (they leave it only together)
+      s_l[hf * kQ + row] = l;
+      ptx::named_barrier(pair_bar, 64);
+      l += s_l[(1 - hf) * kQ + row];
+    }
     const bool o_ready = ok && ptx::mbar_wait_bounded(fin, 0);
     if (__all_sync(0xffffffffu, o_ready)) {  // the TMEM loads below are warp-wide
       ptx::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* op = p.out + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD;
+      float* op = p.out + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD + 64 * hf;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t ov[32];
-        ptx::tmem_ld32(t_o + lane_off + c4 * 32, ov);
+        ptx::tmem_ld32(tbase + lane_off + kColO + 64 * hf + 32 * c2, ov);
         ptx::tmem_wait_ld();
         if (tq < p.n_tokens) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            *reinterpret_cast<float4*>(op + c4 * 32 + e) =
+            *reinterpret_cast<float4*>(op + 32 * c2 + e) =
                 make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
                             __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
           }
@@ -587,7 +562,7 @@ cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t strea
   p.q = qws;
   p.out = a.out;
   p.err = a.err;
-  dim3 grid(cv.batch * (kH / 2), p.n_qtiles);
+  dim3 grid(cv.batch * kH, p.n_qtiles);
   auto kern = cv.r_k == 1 ? prefill_tc_kernel<1> : prefill_tc_kernel<2>;
   kern<<<grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
   return cudaGetLastError();
