@@ -180,10 +180,25 @@ def cpu_oracle_rate(host, w, target_s: float, workers: int):
 
 
 # --------------------------------------------------------------------------- decode bench
+def rank_workload(w, rank):
+    """The workload rank `rank` runs: the same shapes, its own seed (rank 0 keeps the workload's)."""
+    return w.replace(seed=w.seed + 1000 * rank) if rank else w
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    """Maximum of a per-rank number (a time) over all ranks; x itself on one rank."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def decode_host_inputs(w, rank):
     from factorized_kv_cache_b200 import synthetic as S
-    ww = w.replace(seed=w.seed + 1000 * rank) if rank else w
-    return S.decode_inputs(ww)
+    return S.decode_inputs(rank_workload(w, rank))
 
 
 def run_ours_decode(args, w, rank, world, dev):
@@ -286,10 +301,7 @@ def run_ours_decode(args, w, rank, world, dev):
     clk = clocks.stop() if clocks else None
     elapsed_ms = t_start.elapsed_time(t_end)
     decode_ms = [a.elapsed_time(b) / n_calls for a, b in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     if T.tpa_read_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
@@ -327,10 +339,7 @@ def run_ours_decode(args, w, rank, world, dev):
     for k in range(e2e_steps):
         e2e_step(k % copies)
     e2e_s = time.perf_counter() - t0
-    if world > 1:
-        t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
+    e2e_s = max_over_ranks(e2e_s, world, dev)
 
     launches_per_step = 1 + 1 + (1 if splits > 1 else 0)
     bytes_per_decode = tokens_per_step * per_tok + B * w.heads * w.head_dim * (esize + 4)
@@ -520,7 +529,7 @@ def run_ours_prefill(args, w, rank, world, dev):
 
     kernel = {"auto": T.TPA_KERNEL_AUTO, "simt": T.TPA_KERNEL_SIMT, "tensor": T.TPA_KERNEL_TENSOR,
               "tensor_sync": T.TPA_KERNEL_TENSOR_SYNC}[args.kernel]
-    ww = w.replace(seed=w.seed + 1000 * rank) if rank else w
+    ww = rank_workload(w, rank)
     x = S.prefill_inputs(ww)
     B, Tn = w.batch, w.tokens
     cache = T.TpaCache.allocate(B, Tn, w.heads, w.head_dim, w.r_k, w.r_v, dtype=torch.bfloat16,
@@ -578,10 +587,7 @@ def run_ours_prefill(args, w, rank, world, dev):
     clk = clocks.stop() if clocks else None
     elapsed_ms = t_start.elapsed_time(t_end)
     pre_ms = [a.elapsed_time(b) for a, b in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     if T.tpa_read_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
@@ -604,10 +610,12 @@ def run_ours_prefill(args, w, rank, world, dev):
         stream.synchronize()
 
     e2e_step()
+    if world > 1:
+        dist.barrier()
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
         e2e_step()
-    e2e_s = time.perf_counter() - t0
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
 
     pairs = B * Tn * (Tn + 1) // 2
     flops = pairs * w.heads * 2 * w.head_dim * (w.r_k + w.r_v)   # score + value contractions, per (query, key) pair
