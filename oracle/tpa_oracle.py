@@ -166,16 +166,31 @@ def decode_attention(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block: int =
       q~_i = RoPE(q_i, q_pos)
       K_s = (1/R_K) A_K[s]^T B~_K[s],  V_s = (1/R_V) A_V[s]^T B_V[s]
       z[i, s] = scale * q~_i . K_s[i],  o_i = sum_s softmax_s(z[i, :]) V_s[i]
-
-    K and V are expanded ``block`` tokens at a time only to bound memory: every
-    score is computed on its own, the softmax is taken over the full score row,
-    and the output sum is split into consecutive partial sums.
     """
+    return _attend_rotated_query(a_k, b_k_rot, a_v, b_v, rope(q, q_pos, base), scale, block)
+
+
+def decode_attention_factored_query(a_k, b_k_rot, a_v, b_v, a_q, b_q, q_pos, scale, base, block: int = 8192):
+    """Decode attention with the query in TPA form (section 解决思路:
+    Q = (1/R_Q) A_Q^T B_Q; RoPE on the B factor, Theorem 3.1).
+
+    a_q [R_Q, h], b_q [R_Q, d_h] unrotated at position q_pos; the cache as in
+    decode_attention.  q~_i = (1/R_Q) sum_j A_Q[j, i] RoPE(B_Q[j], q_pos), then
+    the same attention.  Returns o [h, d_h] (float64).
+    """
+    return _attend_rotated_query(a_k, b_k_rot, a_v, b_v, tensor_product(a_q, rope(b_q, q_pos, base)), scale, block)
+
+
+def _attend_rotated_query(a_k, b_k_rot, a_v, b_v, q_rot, scale, block):
+    """Softmax attention of rotated per-head queries q_rot [h, d_h] over the
+    cached tokens (see decode_attention).  K and V are expanded ``block``
+    tokens at a time only to bound memory: every score is computed on its own,
+    the softmax is taken over the full score row, and the output sum is split
+    into consecutive partial sums."""
     L = np.asarray(a_k).shape[0]
-    h, d_h = np.asarray(q).shape
+    h, d_h = np.asarray(q_rot).shape
     if L == 0:
         return np.zeros((h, d_h))
-    q_rot = rope(q, q_pos, base)
     z = np.empty((h, L))
     for s0 in range(0, L, block):
         s1 = min(L, s0 + block)

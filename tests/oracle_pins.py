@@ -348,6 +348,78 @@ def pin_storage_rounding(O):
     assert (np.abs(st - ex) <= 2.0 ** -8 * np.abs(ex) * (1 + 1e-12)).all()
 
 
+# --------------------------------------------------------------------------- factorized decode query
+def _rand_q_factors(seed, rq, h, d):
+    g = np.random.default_rng(seed)
+    return g.standard_normal((rq, h)), g.standard_normal((rq, d))
+
+
+def pin_factored_query_rank_one(O):
+    """R_Q = 1 with a unit head factor: every head's query is the one rotated B_Q row,
+    i.e. the dense decode with q_i = B_Q[0] for all i."""
+    c = _rand_case(31, 40, 4, 16, 2, 2)
+    _, b_q = _rand_q_factors(32, 1, 4, 16)
+    o1 = O.decode_attention_factored_query(c["a_k"], c["b_k"], c["a_v"], c["b_v"], np.ones((1, 4)), b_q, 41.0,
+                                           0.25, 10000.0)
+    o2 = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], np.repeat(b_q, 4, axis=0), 41.0, 0.25,
+                            10000.0)
+    assert np.allclose(o1, o2, rtol=1e-12, atol=1e-14)
+
+
+def pin_factored_query_linearity(O):
+    """RoPE is linear, so rotating each B_Q row and then forming (1/R_Q) A_Q^T B~_Q equals
+    rotating the summed dense query: the factored decode must equal the dense decode with
+    q_i = (1/R_Q) sum_j A_Q[j, i] B_Q[j] (summed here by explicit loops)."""
+    c = _rand_case(33, 37, 3, 8, 1, 2)
+    rq = 3
+    a_q, b_q = _rand_q_factors(34, rq, 3, 8)
+    q = np.zeros((3, 8))
+    for i in range(3):
+        for k in range(8):
+            q[i, k] = math.fsum(a_q[j, i] * b_q[j, k] for j in range(rq)) / rq
+    o1 = O.decode_attention_factored_query(c["a_k"], c["b_k"], c["a_v"], c["b_v"], a_q, b_q, 777.0, 0.3, 10000.0)
+    o2 = O.decode_attention(c["a_k"], c["b_k"], c["a_v"], c["b_v"], q, 777.0, 0.3, 10000.0)
+    assert np.allclose(o1, o2, rtol=1e-11, atol=1e-13)
+
+
+def pin_factored_query_duplicate_ranks(O):
+    """R_Q copies of one rank equal the single rank (the 1/R_Q sits in the product)."""
+    c = _rand_case(35, 20, 4, 8, 2, 1)
+    a_q, b_q = _rand_q_factors(36, 1, 4, 8)
+    o1 = O.decode_attention_factored_query(c["a_k"], c["b_k"], c["a_v"], c["b_v"], a_q, b_q, 20.0, 0.5, 10000.0)
+    for r in (2, 6):
+        o2 = O.decode_attention_factored_query(c["a_k"], c["b_k"], c["a_v"], c["b_v"], np.repeat(a_q, r, axis=0),
+                                               np.repeat(b_q, r, axis=0), 20.0, 0.5, 10000.0)
+        assert np.allclose(o1, o2, rtol=1e-12, atol=1e-14)
+
+
+def pin_factored_query_brute_force(O):
+    """Tiny case by scalar loops: rotate each B_Q row pair by pair, weight by A_Q / R_Q,
+    expand K and V token by token, softmax with math.fsum."""
+    c = _rand_case(37, 3, 2, 4, 2, 1)
+    rq, h, d, L, qp, scale, base = 2, 2, 4, 3, 5.0, 0.7, 100.0
+    a_q, b_q = _rand_q_factors(38, rq, h, d)
+    qr = np.zeros((h, d))
+    for j in range(rq):
+        rot = _brute_rot(b_q[j], qp, base)
+        for i in range(h):
+            for k in range(d):
+                qr[i, k] += a_q[j, i] * rot[k] / rq
+    want = np.zeros((h, d))
+    for i in range(h):
+        z = []
+        for s in range(L):
+            kk = [math.fsum(c["a_k"][s, r, i] * c["b_k"][s, r, k] for r in range(2)) / 2 for k in range(d)]
+            z.append(scale * math.fsum(qr[i, k] * kk[k] for k in range(d)))
+        mz = max(z)
+        e = [math.exp(v - mz) for v in z]
+        tot = math.fsum(e)
+        for k in range(d):
+            want[i, k] = math.fsum(e[s] / tot * c["a_v"][s, 0, i] * c["b_v"][s, 0, k] for s in range(L))
+    got = O.decode_attention_factored_query(c["a_k"], c["b_k"], c["a_v"], c["b_v"], a_q, b_q, qp, scale, base)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-13)
+
+
 ALL_PINS = [
     pin_storage_rounding,
     pin_cache_size,
@@ -365,4 +437,8 @@ ALL_PINS = [
     pin_brute_force_decode,
     pin_brute_force_prefill,
     pin_prefill_first_row,
+    pin_factored_query_rank_one,
+    pin_factored_query_linearity,
+    pin_factored_query_duplicate_ranks,
+    pin_factored_query_brute_force,
 ]

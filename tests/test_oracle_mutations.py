@@ -62,6 +62,18 @@ def _prefill_q_no_rope(a_q, b_q, q_pos, base):
     return _tp(a_q, b_q)
 
 
+_factored = O.decode_attention_factored_query
+
+
+def _factored_no_q_rope(a_k, b_k_rot, a_v, b_v, a_q, b_q, q_pos, scale, base, block=8192):
+    return _factored(a_k, b_k_rot, a_v, b_v, a_q, b_q, 0.0, scale, base, block)
+
+
+def _factored_no_rq_scale(a_k, b_k_rot, a_v, b_v, a_q, b_q, q_pos, scale, base, block=8192):
+    return _factored(a_k, b_k_rot, a_v, b_v, np.asarray(a_q) * np.asarray(a_q).shape[0], b_q, q_pos, scale, base,
+                     block)
+
+
 def _round_truncate(x, storage):               # truncation instead of round-to-nearest-even
     if storage != "bf16":
         return _round(x, storage)
@@ -91,6 +103,8 @@ MUTANTS = {
     "decode_no_query_rope": ("decode_attention", _decode_no_query_rope),
     "decode_scale_squared": ("decode_attention", _decode_scale_squared),
     "prefill_no_query_rope": ("prefill_queries", _prefill_q_no_rope),
+    "factored_no_query_rope": ("decode_attention_factored_query", _factored_no_q_rope),
+    "factored_no_rq_scale": ("decode_attention_factored_query", _factored_no_rq_scale),
 }
 
 
