@@ -23,9 +23,13 @@ constexpr int kMaxBatch = 1024;
 
 struct DecodeTcParams {
   const int32_t* seq_lens;
-  const void* q;           // [B][32][128] bf16, unrotated
+  const void* q;           // [B][32][128] bf16, unrotated; with r_q > 0: B_Q [B][r_q][128]
+  const void* a_q;         // A_Q [B][r_q][32] bf16 when the query is factorized (r_q > 0)
+  int r_q;                 // 0: dense query
+  float inv_rq;            // 1 / r_q
   const int32_t* q_pos;
   int batch, capacity, max_len, grid;
+  double inv_grid;         // 1 / grid
   float zs;                // scale * log2(e) / R_K
   float inv_rv;            // 1 / R_V
   float* out;              // [B][32][128]
@@ -48,6 +52,17 @@ __device__ __forceinline__ int owner_of(int t, int nt, int grid) {
 // First tile of CTA c: ceil(c nt / grid), exact for the same reason.
 __device__ __forceinline__ int first_tile(int c, int nt, int grid) {
   return static_cast<int>(ceil(static_cast<double>(c) * nt / grid));
+}
+
+// ceil(c nt / grid) from a precomputed 1/grid: the double product is within one
+// of the quotient, and one 64-bit integer step each way makes it exact (a
+// multiply instead of the division sequence at the start of every CTA).
+__device__ __forceinline__ int first_tile_fast(int c, int nt, int grid, double inv_grid) {
+  const long long num = static_cast<long long>(c) * nt;
+  long long q = static_cast<long long>(static_cast<double>(num) * inv_grid);
+  if (q * grid < num) ++q;                    // q >= num / grid
+  if ((q - 1) * grid >= num && q > 0) --q;    // q - 1 < num / grid
+  return static_cast<int>(q);
 }
 
 // Exclusive prefix of per-sequence tile counts into s_pref[0..B] and the

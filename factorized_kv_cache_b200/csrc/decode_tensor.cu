@@ -708,11 +708,15 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   DecodeTcParams p;
   p.seq_lens = cv.seq_lens;
   p.q = a.q;
+  p.a_q = a.a_q;
+  p.r_q = a.r_q;
+  p.inv_rq = a.r_q > 0 ? 1.f / static_cast<float>(a.r_q) : 1.f;
   p.q_pos = a.q_pos;
   p.batch = cv.batch;
   p.capacity = cv.capacity;
   p.max_len = a.max_len;
   p.grid = a.grid;
+  p.inv_grid = 1.0 / static_cast<double>(a.grid);
   p.zs = a.scale * kLog2e / static_cast<float>(cv.r_k);
   p.inv_rv = 1.f / static_cast<float>(cv.r_v);
   p.out = a.out;

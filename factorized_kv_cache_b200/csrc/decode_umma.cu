@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (blockIdx.x == 0)
     for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
   const int c = blockIdx.x;
-  const int t_begin = NT == 0 ? 0 : dec::first_tile(c, NT, p.grid);
-  const int t_end = NT == 0 ? 0 : dec::first_tile(c + 1, NT, p.grid);
+  const int t_begin = NT == 0 ? 0 : dec::first_tile_fast(c, NT, p.grid, p.inv_grid);
+  const int t_end = NT == 0 ? 0 : dec::first_tile_fast(c + 1, NT, p.grid, p.inv_grid);
   if (t_begin >= t_end) {  // uniform: no tiles for this CTA
     if (warp == 1) ptx::tmem_dealloc(tbase, kTmemCols);
     return;
@@ -379,12 +379,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ta >= tb) continue;
       const int len_b = s_len[b];
       // ---- rotated query as bf16 hi (rows 0..31) and lo (rows 32..63), K-major, 128-byte swizzle.
-      // This thread's 16 features of one head and the position are loaded together, first.
+      // This thread's 16 features of one head and the position are loaded together, first.  A
+      // factorized query (section 解决思路: q = (1/R_Q) A_Q^T B_Q) is formed here in fp32 from
+      // its rotated rank rows.
       {
         const int head = wt >> 3, f0 = (wt & 7) * 16;
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                          (static_cast<size_t>(b) * kH + head) * kD + f0);
-        const uint4 qv[2] = {src[0], src[1]};
+        const __nv_bfloat16* qsrc = static_cast<const __nv_bfloat16*>(p.q);
+        const __nv_bfloat16* aqsrc = static_cast<const __nv_bfloat16*>(p.a_q);
+        // row jq of the query: the dense query itself, or rank jq of B_Q and its weight A_Q / R_Q
+        auto row_src = [&](int jq) {
+          return reinterpret_cast<const uint4*>(p.r_q > 0 ? qsrc + (static_cast<size_t>(b) * p.r_q + jq) * kD + f0
+                                                          : qsrc + (static_cast<size_t>(b) * kH + head) * kD + f0);
+        };
+        auto row_weight = [&](int jq) {
+          return p.r_q > 0 ? __bfloat162float(aqsrc[(static_cast<size_t>(b) * p.r_q + jq) * kH + head]) * p.inv_rq
+                           : 1.f;
+        };
+        const uint4* src0 = row_src(0);
+        uint4 qv[2] = {src0[0], src0[1]};
+        float wq = row_weight(0);
         if (wt < kD / 2) {
           float cs, sn;
           rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
@@ -392,19 +405,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           s_cs[2 * wt + 1] = sn;
         }
         ptx::named_barrier(1, kSoftmaxThreads);
+        float acc[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+        const int nrow = p.r_q > 0 ? p.r_q : 1;
+        for (int jq = 0; jq < nrow; ++jq) {
+          if (jq > 0) {
+            const uint4* src = row_src(jq);
+            qv[0] = src[0];
+            qv[1] = src[1];
+            wq = row_weight(jq);
+          }
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const uint32_t w[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int e = 4 * v + k;
+              const int jp = f0 / 2 + e;  // RoPE pair (features 2 jp, 2 jp + 1)
+              float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
+              rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
+              acc[2 * e] = fmaf(wq, x, acc[2 * e]);
+              acc[2 * e + 1] = fmaf(wq, y, acc[2 * e + 1]);
+            }
+          }
+        }
         uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const uint32_t w[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int e = 4 * v + k;
-            const int jp = f0 / 2 + e;  // RoPE pair (features 2 jp, 2 jp + 1)
-            float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
-            rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
-            hi[e] = ptx::pack_bf16(x, y);
-            lo[e] = ptx::pack_bf16(x - ptx::bf16_lo(hi[e]), y - ptx::bf16_hi(hi[e]));
-          }
+        for (int e = 0; e < 8; ++e) {
+          hi[e] = ptx::pack_bf16(acc[2 * e], acc[2 * e + 1]);
+          lo[e] = ptx::pack_bf16(acc[2 * e] - ptx::bf16_lo(hi[e]), acc[2 * e + 1] - ptx::bf16_hi(hi[e]));
         }
         uint8_t* qb = gbase + kOffQ + (f0 >> 6) * kQBox;
 #pragma unroll

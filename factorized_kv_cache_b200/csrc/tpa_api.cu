@@ -258,9 +258,12 @@ size_t tpa_decode_workspace_size(const tpa_cache* cache, int32_t max_len, int32_
   return carve_decode_ws(nullptr, cache->batch, cache->heads, cache->head_dim, p.splits).bytes;
 }
 
-tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int32_t* q_pos, float scale, float* out,
-                                int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
-                                size_t workspace_bytes, void* stream) {
+namespace {
+
+// Decode with a dense query (r_q == 0) or a factorized one (a_q, q = B_Q, r_q >= 1).
+tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, int32_t r_q, const int32_t* q_pos,
+                       float scale, float* out, int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   tpa_status s = check_cache(cache);
   if (s != TPA_OK) return s;
   if (!q || !q_pos || !out) return fail(TPA_ERR_NULL, "q, q_pos or out is NULL");
@@ -276,6 +279,18 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
   if (!isfinite(scale)) return fail(TPA_ERR_SHAPE, "scale is not finite");
   if (!aligned16(q) || !aligned16(out) || (reinterpret_cast<uintptr_t>(q_pos) & 3u))
     return fail(TPA_ERR_ALIGNMENT, "q and out must be 16-byte aligned");
+  if (r_q > 0) {
+    // the factorized query is formed inside the tcgen05 kernel only
+    if (!a_q) return fail(TPA_ERR_NULL, "a_q is NULL");
+    if (r_q > 8) return fail(TPA_ERR_UNSUPPORTED, "r_q = %d not in [1,8]", r_q);
+    if (kernel == TPA_KERNEL_SIMT || kernel == TPA_KERNEL_TENSOR_SYNC ||
+        !tensor_decode_supported(cache->dtype, cache->heads, cache->head_dim, cache->r_k, cache->r_v) ||
+        !tensor_decode_batch_ok(cache->batch))
+      return fail(TPA_ERR_UNSUPPORTED,
+                  "a factorized decode query needs the tcgen05 kernel: bf16, heads 32, head_dim 128, "
+                  "r_k == r_v <= 2, batch <= 1024, kernel AUTO or TENSOR");
+    if (reinterpret_cast<uintptr_t>(a_q) & 1u) return fail(TPA_ERR_ALIGNMENT, "a_q must be 2-byte aligned");
+  }
   int sms = 0;
   unsigned int* err = nullptr;
   cudaError_t e = device_info(&sms, &err);
@@ -296,6 +311,8 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
     TensorDecodeArgs a;
     a.cache = view_of(cache);
     a.q = q;
+    a.a_q = a_q;
+    a.r_q = r_q;
     a.q_pos = q_pos;
     a.scale = scale;
     a.max_len = max_len;
@@ -348,6 +365,24 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
   return TPA_OK;
+}
+
+}  // namespace
+
+tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int32_t* q_pos, float scale, float* out,
+                                int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return decode_impl(cache, q, nullptr, 0, q_pos, scale, out, max_len, num_splits, kernel, workspace,
+                     workspace_bytes, stream);
+}
+
+tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, const void* a_q, const void* b_q,
+                                         const int32_t* q_pos, float scale, float* out, int32_t max_len,
+                                         int32_t num_splits, int32_t kernel, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (r_q < 1) return fail(TPA_ERR_SHAPE, "r_q = %d < 1", r_q);
+  return decode_impl(cache, b_q, a_q, r_q, q_pos, scale, out, max_len, num_splits, kernel, workspace,
+                     workspace_bytes, stream);
 }
 
 size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q, int32_t kernel) {

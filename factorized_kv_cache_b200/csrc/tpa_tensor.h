@@ -22,7 +22,9 @@ size_t tensor_decode_workspace_bytes(int batch, int grid);
 
 struct TensorDecodeArgs {
   CacheView cache;
-  const void* q;
+  const void* q;       // dense query [B][h][d_h], or B_Q [B][r_q][d_h] when r_q > 0
+  const void* a_q;     // A_Q [B][r_q][h] when r_q > 0 (tcgen05 kernel only)
+  int r_q;
   const int32_t* q_pos;
   float scale;
   int max_len;

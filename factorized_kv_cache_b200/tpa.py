@@ -81,6 +81,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_decode_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_decode_attention": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P, ctypes.c_size_t, P]),
         "tpa_decode_attention_noalloc": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P]),
+        "tpa_decode_attention_factored": (ctypes.c_int, [C, I32, P, P, P, ctypes.c_float, P, I32, I32, I32, P,
+                                                          ctypes.c_size_t, P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
@@ -278,6 +280,36 @@ def tpa_decode_attention(cache: TpaCache, q, q_pos, scale: float | None = None, 
     nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
     _check(lib.tpa_decode_attention(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out), max_len,
                                     num_splits, kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+    return out
+
+
+def tpa_decode_attention_factored(cache: TpaCache, a_q, b_q, q_pos, scale: float | None = None, out=None,
+                                  max_len: int | None = None, num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO,
+                                  workspace_buf=None, stream=None):
+    """Decode attention with the query in TPA form: a_q [B, R_Q, h], b_q [B, R_Q, d_h] (unrotated);
+    returns out [B, h, d_h] float32."""
+    lib = load_library()
+    B, h, d = cache.batch, cache.heads, cache.head_dim
+    dev = cache.a_k.device
+    r_q = a_q.shape[1]
+    _need(a_q, "a_q", cache.dtype, (B, r_q, h), dev)
+    _need(b_q, "b_q", cache.dtype, (B, r_q, d), dev)
+    _need(q_pos, "q_pos", torch.int32, (B,), dev)
+    if out is None:
+        out = torch.empty(B, h, d, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, (B, h, d), dev)
+    if max_len is None:
+        max_len = cache.capacity
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    need = int(lib.tpa_decode_workspace_size(ctypes.byref(s), max_len, num_splits, kernel))
+    if workspace_buf is None:
+        workspace_buf = workspace(need, dev)
+    nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+    _check(lib.tpa_decode_attention_factored(ctypes.byref(s), r_q, _ptr(a_q), _ptr(b_q), _ptr(q_pos), float(scale),
+                                             _ptr(out), max_len, num_splits, kernel, _ptr(workspace_buf), nbytes,
+                                             _stream(stream)))
     return out
 
 

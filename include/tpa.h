@@ -177,6 +177,27 @@ tpa_status tpa_decode_attention(const tpa_cache* cache, const void* q, const int
                                 void* stream);
 
 /*
+ * Decode with the query in TPA form (section 解决思路: Q = (1/R_Q) A_Q^T B_Q,
+ * RoPE on the B factor by Theorem 3.1), the full-TPA variant of
+ * tpa_decode_attention:
+ *   a_q [batch][r_q][heads] and b_q [batch][r_q][head_dim] (NOT rotated):
+ *     device, bf16, b_q 16-byte aligned; 1 <= r_q <= 8;
+ *   query of head i: q~_i = (1/r_q) sum_j a_q[b][j][i] RoPE(b_q[b][j], q_pos[b]),
+ *     formed in fp32 inside the kernel, then the same attention as
+ *     tpa_decode_attention (same out, max_len, num_splits, workspace: use
+ *     tpa_decode_workspace_size(cache, max_len, num_splits, TPA_KERNEL_TENSOR)).
+ * Runs on the tcgen05 kernel only: bf16, heads 32, head_dim 128,
+ * r_k == r_v <= 2, batch <= 1024, kernel TPA_KERNEL_AUTO or TPA_KERNEL_TENSOR;
+ * anything else returns TPA_ERR_UNSUPPORTED.
+ * Errors: those of tpa_decode_attention, SHAPE (r_q < 1), UNSUPPORTED.
+ */
+tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, const void* a_q,
+                                         const void* b_q, const int32_t* q_pos, float scale,
+                                         float* out, int32_t max_len, int32_t num_splits,
+                                         int32_t kernel, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/*
  * tpa_decode_attention for callers that cannot allocate device memory (no
  * counterpart on the page; this is a deployment convenience).  Same
  * arguments and result as tpa_decode_attention minus the workspace: the

@@ -75,6 +75,29 @@ def test_decode_rejects_bad_arguments():
     assert _decode(lib, _fake_cache(dtype=T.TPA_F32), kernel=T.TPA_KERNEL_TENSOR) == 3
 
 
+def test_factored_decode_rejects_bad_arguments():
+    lib = T.load_library()
+    P = 0x90000
+
+    def call(c=None, rq=6, a_q=P, b_q=P, kernel=0):
+        c = _fake_cache() if c is None else c
+        return lib.tpa_decode_attention_factored(ctypes.byref(c), rq, a_q, b_q, 0x70000, 0.1, 0x80000, 64, 0, kernel,
+                                                 None, 0, None)
+
+    assert call(rq=0) == 2
+    assert call(rq=9) == 3
+    assert call(a_q=None) == 1
+    assert call(b_q=None) == 1
+    assert call(b_q=P + 8) == 6
+    assert call(a_q=P + 1) == 6
+    assert call(c=_fake_cache(dtype=T.TPA_F32, heads=32, head_dim=128)) == 3   # tcgen05 kernel only
+    assert call(c=_fake_cache(heads=16)) == 3
+    assert call(c=_fake_cache(r_k=2, r_v=1)) == 3
+    assert call(kernel=T.TPA_KERNEL_SIMT) == 3
+    assert call(kernel=T.TPA_KERNEL_TENSOR_SYNC) == 3
+    assert lib.tpa_last_error_message().decode() != ""
+
+
 def test_append_rejects_bad_arguments():
     lib = T.load_library()
     c = _fake_cache()

@@ -195,3 +195,44 @@ def test_score_ramp(kernel, rank, direction):
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=4000, kernel=kernel)
     _check(w, cache, x, q, q_pos, out, end_to_end=False)
     assert T.tpa_read_device_error() == 0
+
+
+@pytest.mark.parametrize("rank", [1, 2])
+@pytest.mark.parametrize("r_q,q_scale", [(1, 1.0), (6, 1.0), (8, 1.0), (6, 3.0)])
+def test_factored_query_decode(rank, r_q, q_scale):
+    """Decode with the query in TPA form (A_Q, B_Q; the full-TPA variant) against the oracle's
+    factored decode, on ragged lengths (empty and one-token sequences included).  B_Q rows are
+    scaled so that the summed query has about unit (or q_scale^2) variance per element."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="factored", r_k=rank, r_v=rank, seed=60 + r_q)
+    lengths = [1000, 1, 0, 333, 4000, 129]
+    cache, x, q, q_pos = build_decode_cache(w, batch=6, length=4000, lengths=lengths)
+    g = S.rng(w.seed, 17)
+    a_q = S.to_storage(g.standard_normal((6, r_q, w.heads), dtype=np.float32), "bf16").to(DEV)
+    b_q = S.to_storage(g.standard_normal((6, r_q, w.head_dim), dtype=np.float32) *
+                       np.float32(q_scale * np.sqrt(r_q)), "bf16").to(DEV)
+    out = T.tpa_decode_attention_factored(cache, a_q, b_q, q_pos, max_len=4000)
+    cpu = readback(cache)
+    scale = default_scale(w.head_dim)
+    got = f64(out)
+    for b, L in enumerate(lengths):
+        ref = O.decode_attention_factored_query(cpu["a_k"][b, :L], cpu["b_k"][b, :L], cpu["a_v"][b, :L],
+                                                cpu["b_v"][b, :L], f64(a_q[b]), f64(b_q[b]), float(q_pos[b]),
+                                                scale, w.rope_base)
+        if L == 0:
+            assert torch.count_nonzero(out[b]) == 0
+            continue
+        assert_rows_close(got[b], ref, TOL[torch.bfloat16], f"factored r_q={r_q} b={b}")
+    assert T.tpa_read_device_error() == 0
+
+
+def test_factored_query_rank_one_matches_dense_decode():
+    """R_Q = 1 with A_Q = 1 is the dense decode with q = B_Q for every head (same kernel path
+    for the attention; only the query stage differs)."""
+    w = S.WORKLOADS["decode_b8_l8k"]
+    cache, x, q, q_pos = build_decode_cache(w, batch=3, length=2000, min_length=100)
+    b_q = q[:, :1, :].contiguous()
+    a_q = torch.ones(3, 1, w.heads, dtype=torch.bfloat16, device=DEV)
+    o_f = T.tpa_decode_attention_factored(cache, a_q, b_q, q_pos, max_len=2000)
+    o_d = T.tpa_decode_attention(cache, b_q.expand(3, w.heads, w.head_dim).contiguous(), q_pos, max_len=2000,
+                                 kernel=T.TPA_KERNEL_TENSOR)
+    assert torch.equal(o_f, o_d)
