@@ -233,6 +233,17 @@ def run_ours_decode(args, w, rank, world, dev):
              for k in ("a_k", "b_k", "a_v", "b_v")}
     q = x["q"].to(dev)
     q_pos = newest[:, 0].contiguous().to(dev)
+    rq = args.query_rank
+    if rq > 0:
+        # the query in TPA form: A_Q ~ N(0,1), B_Q ~ N(0, R_Q), so the summed query has unit variance
+        g = S.rng(rank_workload(w, rank).seed, 23)
+        host_aq = S.to_storage(g.standard_normal((B, rq, w.heads), dtype=np.float32), w.dtype)
+        host_bq = S.to_storage(g.standard_normal((B, rq, w.head_dim), dtype=np.float32) * np.float32(math.sqrt(rq)),
+                               w.dtype)
+        a_q, b_q = host_aq.to(dev), host_bq.to(dev)
+        query_bytes = B * rq * (w.heads + w.head_dim) * esize
+    else:
+        query_bytes = B * w.heads * w.head_dim * esize
     out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32, device=dev)
     splits = T.tpa_decode_default_splits(c0, cap, kernel)
     ws = T.workspace(T.tpa_decode_workspace_size(c0, cap, 0, kernel), dev)
@@ -242,7 +253,11 @@ def run_ours_decode(args, w, rank, world, dev):
         T.tpa_cache_write_slots(caches[c], slots, pos, new_f["a_k"], new_f["b_k"], new_f["a_v"], new_f["b_v"])
 
     def decode(c):
-        T.tpa_decode_attention(caches[c], q, q_pos, out=out, max_len=cap, kernel=kernel, workspace_buf=ws)
+        if rq > 0:
+            T.tpa_decode_attention_factored(caches[c], a_q, b_q, q_pos, out=out, max_len=cap, kernel=kernel,
+                                            workspace_buf=ws)
+        else:
+            T.tpa_decode_attention(caches[c], q, q_pos, out=out, max_len=cap, kernel=kernel, workspace_buf=ws)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
@@ -307,14 +322,14 @@ def run_ours_decode(args, w, rank, world, dev):
 
     # e2e through the public API with host buffers: H2D of the step's inputs, D2H of the output
     host_in = {k: v.cpu().pin_memory() for k, v in new_f.items()}
-    host_q = x["q"].pin_memory()
+    host_qs = {"q": x["q"].pin_memory()} if rq == 0 else {"a_q": host_aq.pin_memory(), "b_q": host_bq.pin_memory()}
     host_idx = newest.pin_memory()
     host_out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32).pin_memory()
     dev_in = {k: torch.empty_like(v) for k, v in new_f.items()}
-    dev_q = torch.empty_like(q)
+    dev_qs = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_qs.items()}
     dev_idx = torch.empty_like(slots)
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + host_q.numel() * host_q.element_size() + \
-        host_idx.numel() * 4
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + \
+        sum(v.numel() * v.element_size() for v in host_qs.values()) + host_idx.numel() * 4
     d2h = host_out.numel() * 4
     e2e_steps = max(1, min(K, 2000))
 
@@ -322,12 +337,17 @@ def run_ours_decode(args, w, rank, world, dev):
         with torch.cuda.stream(stream):
             for k2, v in host_in.items():
                 dev_in[k2].copy_(v, non_blocking=True)
-            dev_q.copy_(host_q, non_blocking=True)
+            for k2, v in host_qs.items():
+                dev_qs[k2].copy_(v, non_blocking=True)
             dev_idx.copy_(host_idx, non_blocking=True)
             T.tpa_cache_write_slots(caches[c], dev_idx, dev_idx, dev_in["a_k"], dev_in["b_k"], dev_in["a_v"],
                                     dev_in["b_v"], stream=stream)
-            T.tpa_decode_attention(caches[c], dev_q, dev_idx[:, 0], out=out, max_len=cap, kernel=kernel,
-                                   workspace_buf=ws, stream=stream)
+            if rq > 0:
+                T.tpa_decode_attention_factored(caches[c], dev_qs["a_q"], dev_qs["b_q"], dev_idx[:, 0], out=out,
+                                                max_len=cap, kernel=kernel, workspace_buf=ws, stream=stream)
+            else:
+                T.tpa_decode_attention(caches[c], dev_qs["q"], dev_idx[:, 0], out=out, max_len=cap, kernel=kernel,
+                                       workspace_buf=ws, stream=stream)
             host_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -342,7 +362,7 @@ def run_ours_decode(args, w, rank, world, dev):
     e2e_s = max_over_ranks(e2e_s, world, dev)
 
     launches_per_step = 1 + 1 + (1 if splits > 1 else 0)
-    bytes_per_decode = tokens_per_step * per_tok + B * w.heads * w.head_dim * (esize + 4)
+    bytes_per_decode = tokens_per_step * per_tok + query_bytes + B * w.heads * w.head_dim * 4
     mean_decode_s = statistics.mean(decode_ms) / 1e3
     peaks, kind = measured_peaks()
     achieved = bytes_per_decode / mean_decode_s / 1e9
@@ -370,6 +390,7 @@ def run_ours_decode(args, w, rank, world, dev):
             "workload": w.name, "batch": B, "seq_len": int(lengths.max()), "seq_len_min": int(lengths.min()),
             "heads": w.heads, "head_dim": w.head_dim, "r_k": w.r_k, "r_v": w.r_v,
             "tokens_attended_per_step": tokens_per_step, "kernel": args.kernel, "splits": splits,
+            "query": "dense" if rq == 0 else f"TPA factors, R_Q={rq}",
             "step": "write newest token (RoPE on B_K) + decode attention (+ LSE merge), one CUDA graph per step",
             "l2": (f"inputs larger than L2: {copies} cache copies rotated ({copies * cache_bytes / 2**20:.0f} MiB "
                    f"> 126 MiB L2)" if copies > 1 else f"inputs larger than L2 ({cache_bytes / 2**20:.0f} MiB)"),
@@ -668,6 +689,8 @@ def main():
                     choices=["decode_tiny_f32", "decode_b8_l8k", "decode_b32_var32k", "prefill_b4_t4k",
                              "decode_long_512k"])
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "tensor_sync"], default="auto")
+    ap.add_argument("--query-rank", type=int, default=0,
+                    help="decode workloads: 0 = dense query; R_Q > 0 = query given as TPA factors A_Q, B_Q")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")

@@ -317,10 +317,11 @@ __global__ void __launch_bounds__(128) merge_kernel(const __grid_constant__ Merg
 constexpr int kPrefillQTokens = 4;
 constexpr int kPrefillQThreads = 256;
 
-template <typename T>
+// kD, kHeads > 0: the shape fixed at compile time (index arithmetic by shifts); 0: taken from a.
+template <typename T, int kD, int kHeads>
 __global__ void __launch_bounds__(kPrefillQThreads) prefill_q_kernel(const __grid_constant__ PrefillQArgs a) {
   extern __shared__ float s_q[];
-  const int d = a.head_dim, h = a.heads, rq = a.r_q;
+  const int d = kD > 0 ? kD : a.head_dim, h = kHeads > 0 ? kHeads : a.heads, rq = a.r_q;
   const int b = blockIdx.y;
   const int t0 = blockIdx.x * kPrefillQTokens;
   const int nt = min(kPrefillQTokens, a.n_tokens - t0);
@@ -397,10 +398,17 @@ cudaError_t launch_prefill_q(const PrefillQArgs& a, cudaStream_t stream) {
   dim3 grid((a.n_tokens + kPrefillQTokens - 1) / kPrefillQTokens, a.batch);
   const size_t smem = sizeof(float) * kPrefillQTokens *
                       (static_cast<size_t>(a.head_dim) + static_cast<size_t>(a.r_q) * (a.head_dim + a.heads));
+  const bool fixed = a.head_dim == 128 && a.heads == 32;
   if (a.dtype == TPA_F32) {
-    prefill_q_kernel<float><<<grid, kPrefillQThreads, smem, stream>>>(a);
+    if (fixed)
+      prefill_q_kernel<float, 128, 32><<<grid, kPrefillQThreads, smem, stream>>>(a);
+    else
+      prefill_q_kernel<float, 0, 0><<<grid, kPrefillQThreads, smem, stream>>>(a);
   } else {
-    prefill_q_kernel<__nv_bfloat16><<<grid, kPrefillQThreads, smem, stream>>>(a);
+    if (fixed)
+      prefill_q_kernel<__nv_bfloat16, 128, 32><<<grid, kPrefillQThreads, smem, stream>>>(a);
+    else
+      prefill_q_kernel<__nv_bfloat16, 0, 0><<<grid, kPrefillQThreads, smem, stream>>>(a);
   }
   return cudaGetLastError();
 }

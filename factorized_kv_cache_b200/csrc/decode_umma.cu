@@ -384,38 +384,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // its rotated rank rows.
       {
         const int head = wt >> 3, f0 = (wt & 7) * 16;
-        const __nv_bfloat16* qsrc = static_cast<const __nv_bfloat16*>(p.q);
-        const __nv_bfloat16* aqsrc = static_cast<const __nv_bfloat16*>(p.a_q);
-        // row jq of the query: the dense query itself, or rank jq of B_Q and its weight A_Q / R_Q
-        auto row_src = [&](int jq) {
-          return reinterpret_cast<const uint4*>(p.r_q > 0 ? qsrc + (static_cast<size_t>(b) * p.r_q + jq) * kD + f0
-                                                          : qsrc + (static_cast<size_t>(b) * kH + head) * kD + f0);
-        };
-        auto row_weight = [&](int jq) {
-          return p.r_q > 0 ? __bfloat162float(aqsrc[(static_cast<size_t>(b) * p.r_q + jq) * kH + head]) * p.inv_rq
-                           : 1.f;
-        };
-        const uint4* src0 = row_src(0);
-        uint4 qv[2] = {src0[0], src0[1]};
-        float wq = row_weight(0);
-        if (wt < kD / 2) {
-          float cs, sn;
-          rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
-          s_cs[2 * wt] = cs;
-          s_cs[2 * wt + 1] = sn;
-        }
-        ptx::named_barrier(1, kSoftmaxThreads);
-        float acc[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-        const int nrow = p.r_q > 0 ? p.r_q : 1;
-        for (int jq = 0; jq < nrow; ++jq) {
-          if (jq > 0) {
-            const uint4* src = row_src(jq);
-            qv[0] = src[0];
-            qv[1] = src[1];
-            wq = row_weight(jq);
+        uint32_t hi[8], lo[8];
+        if (p.r_q == 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                            (static_cast<size_t>(b) * kH + head) * kD + f0);
+          const uint4 qv[2] = {src[0], src[1]};
+          if (wt < kD / 2) {
+            float cs, sn;
+            rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
+            s_cs[2 * wt] = cs;
+            s_cs[2 * wt + 1] = sn;
           }
+          ptx::named_barrier(1, kSoftmaxThreads);
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
             const uint32_t w[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
@@ -425,16 +405,70 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int jp = f0 / 2 + e;  // RoPE pair (features 2 jp, 2 jp + 1)
               float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
               rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
-              acc[2 * e] = fmaf(wq, x, acc[2 * e]);
-              acc[2 * e + 1] = fmaf(wq, y, acc[2 * e + 1]);
+              hi[e] = ptx::pack_bf16(x, y);
+              lo[e] = ptx::pack_bf16(x - ptx::bf16_lo(hi[e]), y - ptx::bf16_hi(hi[e]));
             }
           }
-        }
-        uint32_t hi[8], lo[8];
+        } else {
+          // The rank rows are shared by all heads: each is loaded and rotated once, by
+          // 16 threads, into fp32 scratch in the (idle) W buffers with A_Q / R_Q beside it.
+          // rows of 128 features, each 16-feature chunk padded by 4 floats so that the eight
+          // chunks one warp reads land in distinct banks
+          constexpr int kChunk = 20, kRowF = 8 * kChunk;
+          float* s_bq = reinterpret_cast<float*>(gbase + kOffW);  // [r_q][8 chunks][20] rotated B_Q
+          float* s_aq = s_bq + 8 * kRowF;                            // [r_q][32] A_Q / R_Q
+          const int jr = wt >> 4, c8 = (wt & 15) * 8;                // rank row, first feature of 8
+          uint4 bv = make_uint4(0, 0, 0, 0);
+          if (jr < p.r_q)
+            bv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                 (static_cast<size_t>(b) * p.r_q + jr) * kD + c8);
+          const int ja = wt >> 5;                                    // A_Q: rank row ja, head (wt & 31)
+          float av = 0.f;
+          if (ja < p.r_q)
+            av = __bfloat162float(static_cast<const __nv_bfloat16*>(p.a_q)[(static_cast<size_t>(b) * p.r_q + ja) * kH +
+                                                                           (wt & 31)]) * p.inv_rq;
+          if (wt < kD / 2) {
+            float cs, sn;
+            rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
+            s_cs[2 * wt] = cs;
+            s_cs[2 * wt + 1] = sn;
+          }
+          ptx::named_barrier(1, kSoftmaxThreads);
+          if (jr < p.r_q) {
+            const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          hi[e] = ptx::pack_bf16(acc[2 * e], acc[2 * e + 1]);
-          lo[e] = ptx::pack_bf16(acc[2 * e] - ptx::bf16_lo(hi[e]), acc[2 * e + 1] - ptx::bf16_hi(hi[e]));
+            for (int k = 0; k < 4; ++k) {
+              const int jp = c8 / 2 + k;
+              float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
+              rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
+              const int f = c8 + 2 * k;
+              s_bq[jr * kRowF + (f >> 4) * kChunk + (f & 15)] = x;
+              s_bq[jr * kRowF + (f >> 4) * kChunk + (f & 15) + 1] = y;
+            }
+          }
+          if (ja < p.r_q) s_aq[ja * kH + (wt & 31)] = av;
+          ptx::named_barrier(1, kSoftmaxThreads);
+          float acc[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+          for (int jq = 0; jq < 8; ++jq) {
+            if (jq >= p.r_q) break;
+            const float wq = s_aq[jq * kH + head];
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const float4 v4 = reinterpret_cast<const float4*>(s_bq + jq * kRowF + (f0 >> 4) * kChunk)[e4];
+              acc[4 * e4] = fmaf(wq, v4.x, acc[4 * e4]);
+              acc[4 * e4 + 1] = fmaf(wq, v4.y, acc[4 * e4 + 1]);
+              acc[4 * e4 + 2] = fmaf(wq, v4.z, acc[4 * e4 + 2]);
+              acc[4 * e4 + 3] = fmaf(wq, v4.w, acc[4 * e4 + 3]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            hi[e] = ptx::pack_bf16(acc[2 * e], acc[2 * e + 1]);
+            lo[e] = ptx::pack_bf16(acc[2 * e] - ptx::bf16_lo(hi[e]), acc[2 * e + 1] - ptx::bf16_hi(hi[e]));
+          }
         }
         uint8_t* qb = gbase + kOffQ + (f0 >> 6) * kQBox;
 #pragma unroll
