@@ -54,7 +54,9 @@ __all__ = [
     "tensor_product",
     "append_rope",
     "decode_attention",
+    "decode_attention_factored_query",
     "decode_attention_from_unrotated",
+    "decode_step",
     "prefill_queries",
     "prefill_attention",
     "softmax_attention",
@@ -211,6 +213,31 @@ def decode_attention_from_unrotated(a_k, b_k, a_v, b_v, positions, q, q_pos, sca
     """End-to-end decode: rotate B_K at each token's position (stored in the
     cache dtype when ``storage`` is given), then attend."""
     return decode_attention(a_k, append_rope(b_k, positions, base, storage), a_v, b_v, q, q_pos, scale, base)
+
+
+def decode_step(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos, scale, base, q=None, a_q=None,
+                b_q=None, storage=None):
+    """One generation step of token x_t: append its factors, then attend with its query.
+
+    Section 解决思路 derives Q_t, K_t and V_t from the same token x_t, and section
+    RoPE 兼容性 (Theorem 3.1) rotates every B factor at that token's position, so
+    the new key and the query are both rotated at ``pos``.  The cache (a_k ..
+    b_v, L tokens, B_K stored rotated) gains slot L: new_a_k [R_K, h],
+    new_b_k [R_K, d_h] (unrotated, stored as append_rope(..., storage) does),
+    new_a_v [R_V, h], new_b_v [R_V, d_h].  The query is dense (q [h, d_h]) or in
+    TPA form (a_q [R_Q, h], b_q [R_Q, d_h]); it attends slots 0 .. L, its own
+    token included.  Returns (o [h, d_h], the stored new B~_K row [R_K, d_h]).
+    """
+    new_rot = append_rope(np.asarray(new_b_k, dtype=np.float64)[None], np.array([pos], dtype=np.float64), base,
+                          storage)[0]
+    cat = lambda old, new: np.concatenate([np.asarray(old, dtype=np.float64).reshape((-1,) + np.shape(new)),
+                                           np.asarray(new, dtype=np.float64)[None]], axis=0)
+    ak, bk, av, bv = cat(a_k, new_a_k), cat(b_k_rot, new_rot), cat(a_v, new_a_v), cat(b_v, new_b_v)
+    if q is not None:
+        o = decode_attention(ak, bk, av, bv, q, pos, scale, base)
+    else:
+        o = decode_attention_factored_query(ak, bk, av, bv, a_q, b_q, pos, scale, base)
+    return o, new_rot
 
 
 def prefill_queries(a_q, b_q, q_pos, base):

@@ -420,6 +420,93 @@ def pin_factored_query_brute_force(O):
     assert np.allclose(got, want, rtol=1e-12, atol=1e-13)
 
 
+# --------------------------------------------------------------------------- decode step (append + attend)
+def _step_case(seed, L, h, d, rk, rv):
+    g = np.random.default_rng(seed)
+    c = _rand_case(seed, L, h, d, rk, rv)
+    c.update(new_a_k=g.standard_normal((rk, h)), new_b_k=g.standard_normal((rk, d)) / math.sqrt(d),
+             new_a_v=g.standard_normal((rv, h)), new_b_v=g.standard_normal((rv, d)) / math.sqrt(d))
+    return c
+
+
+def pin_step_empty_cache(O):
+    """With nothing cached the token attends only itself (softmax over one key is 1):
+    o_i = (1/R_V) sum_r A_V[r, i] B_V[r], summed here by explicit loops, whatever the query."""
+    for rk, rv in ((1, 1), (2, 3)):
+        c = _step_case(41 + rk, 0, 3, 8, rk, rv)
+        o, _ = O.decode_step(c["a_k"], c["b_k"], c["a_v"], c["b_v"], c["new_a_k"], c["new_b_k"], c["new_a_v"],
+                             c["new_b_v"], 12.0, 0.4, 10000.0, q=c["q"])
+        for i in range(3):
+            for k in range(8):
+                want = math.fsum(c["new_a_v"][r, i] * c["new_b_v"][r, k] for r in range(rv)) / rv
+                assert abs(o[i, k] - want) <= 1e-14 * (1 + abs(want))
+
+
+def pin_step_brute_force(O):
+    """Tiny steps by scalar loops: the old keys rotated at their own positions, the new key
+    and the query both rotated at the step's position, softmax over old + new with math.fsum;
+    dense and TPA-form queries.  The stored new row, when rounded to bf16, is a bf16 value
+    within half an ulp of the exact rotation."""
+    h, d, rk, rv, L = 2, 4, 2, 1, 3
+    c = _step_case(45, L, h, d, rk, rv)
+    kpos = [2.0, 5.0, 9.0]
+    pos, scale, base = 11.0, 0.6, 100.0
+    old_rot = O.append_rope(c["b_k"], np.array(kpos), base)
+    a_q, b_q = _rand_q_factors(46, 2, h, d)
+    for form in ("dense", "factored"):
+        if form == "dense":
+            o, row = O.decode_step(c["a_k"], old_rot, c["a_v"], c["b_v"], c["new_a_k"], c["new_b_k"], c["new_a_v"],
+                                   c["new_b_v"], pos, scale, base, q=c["q"])
+            qr = [_brute_rot(list(c["q"][i]), pos, base) for i in range(h)]
+        else:
+            o, row = O.decode_step(c["a_k"], old_rot, c["a_v"], c["b_v"], c["new_a_k"], c["new_b_k"], c["new_a_v"],
+                                   c["new_b_v"], pos, scale, base, a_q=a_q, b_q=b_q)
+            rots = [_brute_rot(list(b_q[j]), pos, base) for j in range(2)]
+            qr = [[math.fsum(a_q[j, i] * rots[j][k] for j in range(2)) / 2 for k in range(d)] for i in range(h)]
+        for i in range(h):
+            keys, vals = [], []
+            for s in range(L + 1):
+                ak = c["a_k"][s] if s < L else c["new_a_k"]
+                bk = c["b_k"][s] if s < L else c["new_b_k"]
+                av = c["a_v"][s] if s < L else c["new_a_v"]
+                bv = c["b_v"][s] if s < L else c["new_b_v"]
+                p_s = kpos[s] if s < L else pos
+                rot = [_brute_rot(list(bk[r]), p_s, base) for r in range(rk)]
+                keys.append([math.fsum(ak[r, i] * rot[r][k] for r in range(rk)) / rk for k in range(d)])
+                vals.append([math.fsum(av[r, i] * bv[r, k] for r in range(rv)) / rv for k in range(d)])
+            z = [scale * math.fsum(qr[i][k] * key[k] for k in range(d)) for key in keys]
+            m = max(z)
+            w = [math.exp(x - m) for x in z]
+            tot = math.fsum(w)
+            for k in range(d):
+                want = math.fsum(w[s] / tot * vals[s][k] for s in range(L + 1))
+                assert abs(o[i, k] - want) <= 1e-12 * (1 + abs(want)), (form, i, k)
+        exact = np.array([_brute_rot(list(c["new_b_k"][r]), pos, base) for r in range(rk)])
+        assert np.allclose(row, exact, rtol=1e-14, atol=1e-15)
+    _, st = O.decode_step(c["a_k"], old_rot, c["a_v"], c["b_v"], c["new_a_k"], c["new_b_k"], c["new_a_v"],
+                          c["new_b_v"], pos, scale, base, q=c["q"], storage="bf16")
+    assert np.array_equal(torch.from_numpy(st).to(torch.bfloat16).double().numpy(), st)
+    assert (np.abs(st - exact) <= 2.0 ** -8 * np.abs(exact) * (1 + 1e-12)).all()
+
+
+def pin_step_shift_invariance(O):
+    """Theorem 3.1: scores depend on position differences only, so moving every cached
+    token and the step's token by the same offset leaves the step's output unchanged."""
+    c = _step_case(47, 30, 4, 16, 2, 2)
+    kpos = np.arange(30, dtype=np.float64) * 3 + 1
+    a_q, b_q = _rand_q_factors(48, 3, 4, 16)
+    for shift in (0.0, 517.0):
+        rot = O.append_rope(c["b_k"], kpos + shift, 10000.0)
+        args = (c["a_k"], rot, c["a_v"], c["b_v"], c["new_a_k"], c["new_b_k"], c["new_a_v"], c["new_b_v"],
+                95.0 + shift, 0.5, 10000.0)
+        od, _ = O.decode_step(*args, q=c["q"])
+        of, _ = O.decode_step(*args, a_q=a_q, b_q=b_q)
+        if shift == 0.0:
+            ref_d, ref_f = od, of
+    assert np.allclose(od, ref_d, rtol=1e-9, atol=1e-12)
+    assert np.allclose(of, ref_f, rtol=1e-9, atol=1e-12)
+
+
 ALL_PINS = [
     pin_storage_rounding,
     pin_cache_size,
@@ -441,4 +528,7 @@ ALL_PINS = [
     pin_factored_query_linearity,
     pin_factored_query_duplicate_ranks,
     pin_factored_query_brute_force,
+    pin_step_empty_cache,
+    pin_step_brute_force,
+    pin_step_shift_invariance,
 ]

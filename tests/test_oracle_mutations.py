@@ -74,6 +74,38 @@ def _factored_no_rq_scale(a_k, b_k_rot, a_v, b_v, a_q, b_q, q_pos, scale, base, 
                      block)
 
 
+_step = O.decode_step
+
+
+def _step_parts(a_k, b_k_rot, a_v, b_v, new_a_k, new_rot, new_a_v, new_b_v):
+    cat = lambda old, new: np.concatenate([np.asarray(old, dtype=np.float64).reshape((-1,) + np.shape(new)),
+                                           np.asarray(new, dtype=np.float64)[None]], axis=0)
+    return cat(a_k, new_a_k), cat(b_k_rot, new_rot), cat(a_v, new_a_v), cat(b_v, new_b_v)
+
+
+def _step_new_key_unrotated(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos, scale, base, q=None,
+                            a_q=None, b_q=None, storage=None):
+    nb = O.round_to_storage(np.asarray(new_b_k, dtype=np.float64), storage)
+    ak, bk, av, bv = _step_parts(a_k, b_k_rot, a_v, b_v, new_a_k, nb, new_a_v, new_b_v)
+    if q is not None:
+        return O.decode_attention(ak, bk, av, bv, q, pos, scale, base), nb
+    return O.decode_attention_factored_query(ak, bk, av, bv, a_q, b_q, pos, scale, base), nb
+
+
+def _step_new_key_next_position(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos, scale, base,
+                                q=None, a_q=None, b_q=None, storage=None):
+    return _step(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos + 1, scale, base, q, a_q, b_q,
+                 storage)[0], O.append_rope(np.asarray(new_b_k)[None], np.array([pos]), base, storage)[0]
+
+
+def _step_without_new_token(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos, scale, base, q=None,
+                            a_q=None, b_q=None, storage=None):
+    _, row = _step(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, new_b_v, pos, scale, base, q, a_q, b_q, storage)
+    if q is not None:
+        return O.decode_attention(a_k, b_k_rot, a_v, b_v, q, pos, scale, base), row
+    return O.decode_attention_factored_query(a_k, b_k_rot, a_v, b_v, a_q, b_q, pos, scale, base), row
+
+
 def _round_truncate(x, storage):               # truncation instead of round-to-nearest-even
     if storage != "bf16":
         return _round(x, storage)
@@ -105,6 +137,9 @@ MUTANTS = {
     "prefill_no_query_rope": ("prefill_queries", _prefill_q_no_rope),
     "factored_no_query_rope": ("decode_attention_factored_query", _factored_no_q_rope),
     "factored_no_rq_scale": ("decode_attention_factored_query", _factored_no_rq_scale),
+    "step_new_key_unrotated": ("decode_step", _step_new_key_unrotated),
+    "step_new_key_next_position": ("decode_step", _step_new_key_next_position),
+    "step_without_new_token": ("decode_step", _step_without_new_token),
 }
 
 
