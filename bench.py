@@ -218,69 +218,93 @@ def run_ours_decode(args, w, rank, world, dev):
     cache_bytes = B * cap * per_tok
     copies = 1 if cache_bytes >= 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / cache_bytes)) + 1
 
+    # The step generates one token per sequence: its factors and query come from the workload's
+    # newest token (slot L_b - 1, position L_b - 1).  Fused (tpa_decode_step): the cache holds
+    # L_b - 1 tokens and the step stores the token and attends all L_b (advance=False, so every
+    # step rewrites the same slot).  Two calls: the cache holds L_b tokens, tpa_cache_write_slots
+    # rewrites slot L_b - 1, then tpa_decode_attention attends all L_b.
+    fused = args.step == "fused" and kernel in (T.TPA_KERNEL_AUTO, T.TPA_KERNEL_TENSOR) and w.dtype == "bf16"
+    if fused and lengths.min() < 1:
+        raise ValueError("the fused step needs every sequence to hold its newest token")
     # copy 0 from the seeded inputs through the product append path, the rest cloned
     c0 = T.TpaCache.allocate(B, cap, w.heads, w.head_dim, w.r_k, w.r_v, dtype=dt, rope_base=w.rope_base, device=dev)
     T.tpa_cache_append(c0, x["positions"].to(dev), x["a_k"].to(dev), x["b_k"].to(dev), x["a_v"].to(dev),
                        x["b_v"].to(dev))
-    c0.seq_lens.copy_(x["lengths"].to(dev))
+    c0.seq_lens.copy_(torch.from_numpy((lengths - 1 if fused else lengths).astype(np.int32)).to(dev))
     caches = [c0] + [T.TpaCache(c0.a_k.clone(), c0.b_k.clone(), c0.a_v.clone(), c0.b_v.clone(), c0.seq_lens.clone(),
                                 w.rope_base) for _ in range(copies - 1)]
-    # the newest token of every sequence is rewritten each step: slot L_b-1, position L_b-1
     newest = torch.from_numpy((lengths - 1).clip(min=0).astype(np.int32))[:, None]
-    slots = newest.to(dev)
-    pos = newest.to(dev)
-    new_f = {k: x[k][torch.arange(B), torch.from_numpy((lengths - 1).clip(min=0))][:, None].contiguous().to(dev)
-             for k in ("a_k", "b_k", "a_v", "b_v")}
-    q = x["q"].to(dev)
-    q_pos = newest[:, 0].contiguous().to(dev)
+    sel = (torch.arange(B), torch.from_numpy((lengths - 1).clip(min=0)))
+    inputs = {}   # the step's device inputs, by name; the e2e leg copies them from one pinned buffer
+    if fused:
+        for k in ("a_k", "b_k", "a_v", "b_v"):
+            inputs[k] = x[k][sel].contiguous().to(dev)                 # [B, R, h | d_h]
+    else:
+        for k in ("a_k", "b_k", "a_v", "b_v"):
+            inputs[k] = x[k][sel][:, None].contiguous().to(dev)        # [B, 1, R, h | d_h]
+        inputs["slots"] = newest.to(dev)
+        inputs["pos2"] = newest.to(dev)
+    inputs["q_pos"] = newest[:, 0].contiguous().to(dev)
     rq = args.query_rank
     if rq > 0:
         # the query in TPA form: A_Q ~ N(0,1), B_Q ~ N(0, R_Q), so the summed query has unit variance
         g = S.rng(rank_workload(w, rank).seed, 23)
-        host_aq = S.to_storage(g.standard_normal((B, rq, w.heads), dtype=np.float32), w.dtype)
-        host_bq = S.to_storage(g.standard_normal((B, rq, w.head_dim), dtype=np.float32) * np.float32(math.sqrt(rq)),
-                               w.dtype)
-        a_q, b_q = host_aq.to(dev), host_bq.to(dev)
+        inputs["a_q"] = S.to_storage(g.standard_normal((B, rq, w.heads), dtype=np.float32), w.dtype).to(dev)
+        inputs["b_q"] = S.to_storage(g.standard_normal((B, rq, w.head_dim), dtype=np.float32) *
+                                     np.float32(math.sqrt(rq)), w.dtype).to(dev)
         query_bytes = B * rq * (w.heads + w.head_dim) * esize
     else:
+        inputs["q"] = x["q"].to(dev)
         query_bytes = B * w.heads * w.head_dim * esize
     out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32, device=dev)
     splits = T.tpa_decode_default_splits(c0, cap, kernel)
     ws = T.workspace(T.tpa_decode_workspace_size(c0, cap, 0, kernel), dev)
     tokens_per_step = int(lengths.sum())
 
-    def write(c):
-        T.tpa_cache_write_slots(caches[c], slots, pos, new_f["a_k"], new_f["b_k"], new_f["a_v"], new_f["b_v"])
-
-    def decode(c):
+    def step(c, v=inputs):
+        qkw = {"a_q": v["a_q"], "b_q": v["b_q"]} if rq > 0 else {"q": v["q"]}
+        if fused:
+            T.tpa_decode_step(caches[c], v["q_pos"], v["a_k"], v["b_k"], v["a_v"], v["b_v"], **qkw, out=out,
+                              max_len=cap, advance=False, kernel=kernel, workspace_buf=ws)
+            return
+        T.tpa_cache_write_slots(caches[c], v["slots"], v["pos2"], v["a_k"], v["b_k"], v["a_v"], v["b_v"])
         if rq > 0:
-            T.tpa_decode_attention_factored(caches[c], a_q, b_q, q_pos, out=out, max_len=cap, kernel=kernel,
-                                            workspace_buf=ws)
+            T.tpa_decode_attention_factored(caches[c], v["a_q"], v["b_q"], v["q_pos"], out=out, max_len=cap,
+                                            kernel=kernel, workspace_buf=ws)
         else:
-            T.tpa_decode_attention(caches[c], q, q_pos, out=out, max_len=cap, kernel=kernel, workspace_buf=ws)
+            T.tpa_decode_attention(caches[c], v["q"], v["q_pos"], out=out, max_len=cap, kernel=kernel,
+                                   workspace_buf=ws)
+
+    def decode_call(c):
+        """The call the roofline times: the fused step, or the decode of the two-call step."""
+        if fused:
+            step(c)
+        elif rq > 0:
+            T.tpa_decode_attention_factored(caches[c], inputs["a_q"], inputs["b_q"], inputs["q_pos"], out=out,
+                                            max_len=cap, kernel=kernel, workspace_buf=ws)
+        else:
+            T.tpa_decode_attention(caches[c], inputs["q"], inputs["q_pos"], out=out, max_len=cap, kernel=kernel,
+                                   workspace_buf=ws)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
         for c in range(copies):     # eager run first (loads the module, checks arguments)
-            write(c)
-            decode(c)
+            step(c)
     torch.cuda.synchronize(dev)
-    # one graph per cache copy for the whole step (the cache write, then the decode launched
-    # with programmatic dependent launch); for the kernel roofline, one graph of n_calls decode
-    # calls cycling over the copies, so that the per-graph launch cost is not charged to the kernel
+    # one graph per cache copy for the whole step; for the kernel roofline, one graph of n_calls
+    # decode calls cycling over the copies, so that the per-graph launch cost is not charged to the kernel
     gs = []
     for c in range(copies):
         g1 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g1, stream=stream):
-            write(c)
-            decode(c)
+            step(c)
         gs.append(g1)
     n_calls = copies * max(1, math.ceil(4 / copies))
     gd = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gd, stream=stream):
         for k in range(n_calls):
-            decode(k % copies)
+            decode_call(k % copies)
     torch.cuda.synchronize(dev)
     if T.tpa_read_device_error() != 0:
         raise RuntimeError("device error word set after set-up")
@@ -305,7 +329,7 @@ def run_ours_decode(args, w, rank, world, dev):
         for k in range(K):
             gs[(W + k) % copies].replay()
         t_end.record(stream)
-        # the decode call alone (split kernel + merge), n_calls back to back per graph, for the roofline
+        # the decode call alone, n_calls back to back per graph, for the roofline
         for r in range(reps):
             ev[r][0].record(stream)
             gd.replay()
@@ -320,34 +344,37 @@ def run_ours_decode(args, w, rank, world, dev):
     if T.tpa_read_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
-    # e2e through the public API with host buffers: H2D of the step's inputs, D2H of the output
-    host_in = {k: v.cpu().pin_memory() for k, v in new_f.items()}
-    host_qs = {"q": x["q"].pin_memory()} if rq == 0 else {"a_q": host_aq.pin_memory(), "b_q": host_bq.pin_memory()}
-    host_idx = newest.pin_memory()
+    # e2e through the public API with host buffers: every step copies its inputs from one pinned
+    # host buffer (one H2D copy) and reads the output back (one D2H copy), then synchronises
+    layout, off = [], 0
+    for k2, v in inputs.items():
+        nb = v.numel() * v.element_size()
+        layout.append((k2, off, nb, v))
+        off += (nb + 255) // 256 * 256
+    host_in = torch.empty(off, dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty(off, dtype=torch.uint8, device=dev)
+    views = {}
+    for k2, o, nb, v in layout:
+        host_in[o:o + nb].copy_(v.cpu().contiguous().view(-1).view(torch.uint8))
+        views[k2] = dev_in[o:o + nb].view(v.dtype).view(v.shape)
     host_out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32).pin_memory()
-    dev_in = {k: torch.empty_like(v) for k, v in new_f.items()}
-    dev_qs = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_qs.items()}
-    dev_idx = torch.empty_like(slots)
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values()) + \
-        sum(v.numel() * v.element_size() for v in host_qs.values()) + host_idx.numel() * 4
+    h2d = sum(nb for _, _, nb, _ in layout)
     d2h = host_out.numel() * 4
     e2e_steps = max(1, min(K, 2000))
 
+    if fused:   # a generation loop binds its buffers once (T.DecodeStepPlan), then calls it every step
+        v = views
+        qkw = {"a_q": v["a_q"], "b_q": v["b_q"]} if rq > 0 else {"q": v["q"]}
+        plans = [T.DecodeStepPlan(caches[c], v["q_pos"], v["a_k"], v["b_k"], v["a_v"], v["b_v"], out, **qkw,
+                                  max_len=cap, advance=False, kernel=kernel, workspace_buf=ws) for c in range(copies)]
+
     def e2e_step(c):
         with torch.cuda.stream(stream):
-            for k2, v in host_in.items():
-                dev_in[k2].copy_(v, non_blocking=True)
-            for k2, v in host_qs.items():
-                dev_qs[k2].copy_(v, non_blocking=True)
-            dev_idx.copy_(host_idx, non_blocking=True)
-            T.tpa_cache_write_slots(caches[c], dev_idx, dev_idx, dev_in["a_k"], dev_in["b_k"], dev_in["a_v"],
-                                    dev_in["b_v"], stream=stream)
-            if rq > 0:
-                T.tpa_decode_attention_factored(caches[c], dev_qs["a_q"], dev_qs["b_q"], dev_idx[:, 0], out=out,
-                                                max_len=cap, kernel=kernel, workspace_buf=ws, stream=stream)
+            dev_in.copy_(host_in, non_blocking=True)
+            if fused:
+                plans[c](stream)
             else:
-                T.tpa_decode_attention(caches[c], dev_qs["q"], dev_idx[:, 0], out=out, max_len=cap, kernel=kernel,
-                                       workspace_buf=ws, stream=stream)
+                step(c, views)
             host_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -361,8 +388,11 @@ def run_ours_decode(args, w, rank, world, dev):
     e2e_s = time.perf_counter() - t0
     e2e_s = max_over_ranks(e2e_s, world, dev)
 
-    launches_per_step = 1 + 1 + (1 if splits > 1 else 0)
-    bytes_per_decode = tokens_per_step * per_tok + query_bytes + B * w.heads * w.head_dim * 4
+    launches_per_step = 2 if fused else 1 + 1 + (1 if splits > 1 else 0)
+    # factor bytes of every attended token (cached, or the step's own read from its inputs), the
+    # step's token stored (fused), the query and the fp32 output
+    bytes_per_decode = tokens_per_step * per_tok + (B * per_tok if fused else 0) + query_bytes + \
+        B * w.heads * w.head_dim * 4
     mean_decode_s = statistics.mean(decode_ms) / 1e3
     peaks, kind = measured_peaks()
     achieved = bytes_per_decode / mean_decode_s / 1e9
@@ -391,7 +421,9 @@ def run_ours_decode(args, w, rank, world, dev):
             "heads": w.heads, "head_dim": w.head_dim, "r_k": w.r_k, "r_v": w.r_v,
             "tokens_attended_per_step": tokens_per_step, "kernel": args.kernel, "splits": splits,
             "query": "dense" if rq == 0 else f"TPA factors, R_Q={rq}",
-            "step": "write newest token (RoPE on B_K) + decode attention (+ LSE merge), one CUDA graph per step",
+            "step": ("tpa_decode_step: split kernel over the L-1 cached tokens + merge that stores the newest "
+                     "token (RoPE on B_K) and joins it, one CUDA graph per step" if fused else
+                     "write newest token (RoPE on B_K) + decode attention (+ LSE merge), one CUDA graph per step"),
             "l2": (f"inputs larger than L2: {copies} cache copies rotated ({copies * cache_bytes / 2**20:.0f} MiB "
                    f"> 126 MiB L2)" if copies > 1 else f"inputs larger than L2 ({cache_bytes / 2**20:.0f} MiB)"),
             "parallelism": f"dp{world} (independent batches, no collective)",
@@ -399,7 +431,8 @@ def run_ours_decode(args, w, rank, world, dev):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(w.name, kernel_src) if kernel_src else None,
-            "peak_kind": kind, "kernel": "decode attention call (split kernel + merge), timed right after the K "
+            "peak_kind": kind, "kernel": ("fused step call" if fused else "decode attention call") +
+                                          " (split kernel + merge), timed right after the K "
                                           "timed steps on the same stream: graphs of back-to-back decode calls "
                                           "over the same cache copies, CUDA events around each graph",
             "calls_per_graph": n_calls,
@@ -691,6 +724,8 @@ def main():
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "tensor_sync"], default="auto")
     ap.add_argument("--query-rank", type=int, default=0,
                     help="decode workloads: 0 = dense query; R_Q > 0 = query given as TPA factors A_Q, B_Q")
+    ap.add_argument("--step", choices=["fused", "two_call"], default="fused",
+                    help="decode step: tpa_decode_step (tcgen05 path), or tpa_cache_write_slots + decode")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")

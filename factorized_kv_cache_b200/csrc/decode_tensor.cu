@@ -482,12 +482,53 @@ __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition
 // partial groups of 32 threads (one float4 column per thread), each thread
 // with kMergeBatch partial loads in flight at once, so even the ~150 partials
 // of a single long sequence take only a few L2 round trips.
+//
+// Decode step (kStep): the token being generated (its factors and its query,
+// section 解决思路: Q_t, K_t, V_t all come from x_t) is appended and attended
+// in the same two launches.  It enters the log-sum-exp as one more partial
+// state (m = its own score z_t, l = 1, o = V_t), so the split kernel reads only
+// the tokens cached before the step and never waits on the new slot.  Its score
+// and value are formed here before the wait on the split kernel, from inputs
+// that earlier work wrote (the split kernel lets this grid start only once all
+// of its CTAs are past their own wait): the new B_K row and the query are
+// rotated at the step's position (Theorem 3.1), the row rounded to bf16 exactly
+// as an append stores it.  After the wait the (sequence, head 0) CTA stores the
+// token in slot L = the length the split kernel saw and, if asked, sets the
+// length to L + 1.  These CTAs start as the split kernel's CTAs leave their SMs,
+// so the work before the wait mostly overlaps the split kernel's tail.
+struct TcStepParams {
+  const int32_t* pos;             // [B] position of the step's token (its key and its query)
+  const __nv_bfloat16* a_k;       // new token [B][R][32], B_K [B][R][128] unrotated, A_V, B_V
+  const __nv_bfloat16* b_k;
+  const __nv_bfloat16* a_v;
+  const __nv_bfloat16* b_v;
+  const __nv_bfloat16* q;         // dense query [B][32][128], or B_Q [B][r_q][128]
+  const __nv_bfloat16* a_q;       // A_Q [B][r_q][32] when r_q > 0
+  int r_q;
+  float inv_rq;
+  int r;                          // R_K = R_V
+  float zs;                       // scale * log2(e) / R_K
+  float inv_rv;
+  int capacity;
+  int advance;
+  const int32_t* ws_len;          // lengths the split kernel saw (-1: out of range)
+  const float* step_ml;           // (m, l) of the sequences it finished inside one CTA
+  __nv_bfloat16* c_ak;            // the cache planes and lengths
+  __nv_bfloat16* c_bk;
+  __nv_bfloat16* c_av;
+  __nv_bfloat16* c_bv;
+  int32_t* seq_lens;
+  unsigned int* err;
+  RopeTable rope;
+};
+
 struct TcMergeParams {
   int batch, grid;
   const int32_t* prefix;
   const float* ws_ml;
   const float* ws_o;
   float* out;
+  TcStepParams st;  // read only by the step variant
 };
 
 constexpr int kMergeThreads = 256;
@@ -510,22 +551,158 @@ __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red
   return v;
 }
 
+template <bool kStep>
 __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __grid_constant__ TcMergeParams p) {
-  ptx::pdl_wait();
+  // the next decode may start its set-up on SMs this grid frees; it waits for this grid to
+  // complete before it touches memory
+  ptx::pdl_launch_dependents();
   __shared__ float s_w[kMergeMax];
   __shared__ int s_slot[kMergeMax];
   __shared__ float s_red[kMergeThreads / 32];
   __shared__ float4 s_acc[kMergeGroups][32];
   const int b = blockIdx.x, i = blockIdx.y, tid = threadIdx.x;
+  const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
+
+  // ---- the step's token for head i: score z_t (log2 units) and value V_t (columns 4 f4 ..
+  // 4 f4 + 3), every input load issued before the first is used
+  float zn = 0.f;
+  float4 vn = make_float4(0.f, 0.f, 0.f, 0.f);
+  uint32_t bkr[2] = {0u, 0u};  // rotated B_K pair 2 tid, 2 tid + 1 of rank rows 0, 1 (bf16 x 2), tid < 64
+  uint32_t word = 0u;          // one 4-byte word of the token's A_K | A_V | B_V, head-0 CTA, tid >= 64
+  if constexpr (kStep) {
+    const TcStepParams& st = p.st;
+    const int R = st.r;
+    float ak[2] = {0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+      if (r < R) ak[r] = __bfloat162float(st.a_k[(static_cast<size_t>(b) * R + r) * kH + i]);
+    if (tid < 64) {
+      const int pos = st.pos[b];
+      __nv_bfloat162 kk[2], qq[8];
+      float aq[8];
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        if (r < R) kk[r] = reinterpret_cast<const __nv_bfloat162*>(st.b_k + (static_cast<size_t>(b) * R + r) * kD)[tid];
+      if (st.r_q == 0) {
+        qq[0] = reinterpret_cast<const __nv_bfloat162*>(st.q + (static_cast<size_t>(b) * kH + i) * kD)[tid];
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < st.r_q) {
+            const size_t row = static_cast<size_t>(b) * st.r_q + j;
+            qq[j] = reinterpret_cast<const __nv_bfloat162*>(st.q + row * kD)[tid];
+            aq[j] = __bfloat162float(st.a_q[row * kH + i]);
+          }
+        }
+      }
+      float c, sn;
+      rope_cos_sin(pos, st.rope.theta[tid], &c, &sn);
+      float qx = 0.f, qy = 0.f;
+      if (st.r_q == 0) {
+        qx = __low2float(qq[0]);
+        qy = __high2float(qq[0]);
+        rope_pair(qx, qy, c, sn);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < st.r_q) {
+            float x = __low2float(qq[j]), y = __high2float(qq[j]);
+            rope_pair(x, y, c, sn);
+            qx = fmaf(aq[j], x, qx);
+            qy = fmaf(aq[j], y, qy);
+          }
+        }
+        qx *= st.inv_rq;
+        qy *= st.inv_rq;
+      }
+      float dot = 0.f;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (r < R) {
+          float x = __low2float(kk[r]), y = __high2float(kk[r]);
+          rope_pair(x, y, c, sn);
+          __nv_bfloat162 kr = __floats2bfloat162_rn(x, y);  // the stored row
+          bkr[r] = *reinterpret_cast<uint32_t*>(&kr);
+          dot = fmaf(ak[r], fmaf(qx, __low2float(kr), qy * __high2float(kr)), dot);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if ((tid & 31) == 0) s_red[tid >> 5] = dot;
+    }
+    if (tid < 32) {
+      for (int r = 0; r < R; ++r) {
+        const size_t row = static_cast<size_t>(b) * R + r;
+        const float a = __bfloat162float(st.a_v[row * kH + i]) * st.inv_rv;
+        const uint2 raw = reinterpret_cast<const uint2*>(st.b_v + row * kD)[tid];
+        const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        vn.x = fmaf(a, __low2float(v01), vn.x);
+        vn.y = fmaf(a, __high2float(v01), vn.y);
+        vn.z = fmaf(a, __low2float(v23), vn.z);
+        vn.w = fmaf(a, __high2float(v23), vn.w);
+      }
+    }
+    if (blockIdx.y == 0 && tid >= 64) {
+      const int w = tid - 64, na = R * kH / 2, nb = R * kD / 2;  // 4-byte words per plane
+      if (w < na) word = reinterpret_cast<const uint32_t*>(st.a_k + static_cast<size_t>(b) * R * kH)[w];
+      else if (w < 2 * na) word = reinterpret_cast<const uint32_t*>(st.a_v + static_cast<size_t>(b) * R * kH)[w - na];
+      else if (w < 2 * na + nb)
+        word = reinterpret_cast<const uint32_t*>(st.b_v + static_cast<size_t>(b) * R * kD)[w - 2 * na];
+    }
+    __syncthreads();
+    zn = (s_red[0] + s_red[1]) * st.zs;
+    __syncthreads();  // s_red is reused by the merge below
+  }
+
+  ptx::pdl_wait();  // the split kernel's partials, outputs and recorded lengths
+
+  // everything the merge reads first, loaded together
   const int NT = p.prefix[p.batch];
   const int t0 = p.prefix[b], t1 = p.prefix[b + 1];
+  bool nv = false;  // the step's token is attended
+  if constexpr (kStep) {
+    const TcStepParams& st = p.st;
+    const int R = st.r;
+    const int L = st.ws_len[b];
+    nv = L >= 0 && L < st.capacity;
+    if (blockIdx.y == 0) {
+      if (nv) {
+        const size_t tok = (static_cast<size_t>(b) * st.capacity + L) * R;  // first rank row of slot L
+        if (tid < 64) {
+          for (int r = 0; r < R; ++r) reinterpret_cast<uint32_t*>(st.c_bk + (tok + r) * kD)[tid] = bkr[r];
+        } else {
+          const int w = tid - 64, na = R * kH / 2, nb = R * kD / 2;
+          if (w < na) reinterpret_cast<uint32_t*>(st.c_ak + tok * kH)[w] = word;
+          else if (w < 2 * na) reinterpret_cast<uint32_t*>(st.c_av + tok * kH)[w - na] = word;
+          else if (w < 2 * na + nb) reinterpret_cast<uint32_t*>(st.c_bv + tok * kD)[w - 2 * na] = word;
+        }
+        if (tid == 0 && st.advance) st.seq_lens[b] = L + 1;
+      } else if (tid == 0 && L >= 0) {
+        atomicOr(st.err, TPA_DEVERR_APPEND_OVERFLOW);  // the cache is full: the token is neither stored nor attended
+      }
+    }
+  }
+
   float* o = p.out + (static_cast<size_t>(b) * kH + i) * kD;
-  if (t1 <= t0) {
-    if (tid < kD) o[tid] = 0.f;
+  if (t1 <= t0) {  // nothing cached: the step's token alone, or zeros
+    if (tid < 32) reinterpret_cast<float4*>(o)[tid] = nv ? vn : make_float4(0.f, 0.f, 0.f, 0.f);
     return;
   }
   const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
-  if (cs == ce) return;  // written by the decode kernel
+  if (cs == ce) {  // finished by the split kernel
+    if (kStep && nv && tid < 32) {
+      const float2 ml = reinterpret_cast<const float2*>(p.st.step_ml)[static_cast<size_t>(b) * kH + i];
+      const float4 on = reinterpret_cast<const float4*>(o)[tid];
+      const float M = fmaxf(ml.x, zn);
+      const float wo = (ml.x == -INFINITY ? 0.f : exp2f(ml.x - M)) * ml.y;
+      const float wn = exp2f(zn - M);
+      const float inv = 1.f / (wo + wn);
+      reinterpret_cast<float4*>(o)[tid] = make_float4((on.x * wo + vn.x * wn) * inv, (on.y * wo + vn.y * wn) * inv,
+                                                      (on.z * wo + vn.z * wn) * inv, (on.w * wo + vn.w * wn) * inv);
+    }
+    return;
+  }
   const int n = ce - cs + 1;
   const bool dense = p.grid <= NT;
   const bool cs_first = dec::first_tile(cs, NT, p.grid) >= t0;
@@ -537,9 +714,9 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     if (!(a < e && a < t1 && e > t0)) return -1;
     return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
   };
-  const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float M;
   if (n <= kMergeGroups * kMergeBatch) {
     // one pass: every partial's features and (m, l) are loaded at once, before the maximum is known
     float4 v[kMergeBatch];
@@ -555,7 +732,8 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     const int my = tid < n ? slot_of(tid) : -1;
     const float2 ml = my >= 0 ? *reinterpret_cast<const float2*>(p.ws_ml + 2 * static_cast<size_t>(my))
                               : make_float2(-INFINITY, 0.f);
-    const float M = merge_reduce(ml.x, true, s_red);
+    M = merge_reduce(ml.x, true, s_red);
+    if (nv) M = fmaxf(M, zn);
     const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
     if (tid < n) s_w[tid] = w;
     L = merge_reduce(ml.y * w, false, s_red);  // ends with a barrier: s_w visible
@@ -568,12 +746,13 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       acc.w = fmaf(v[k].w, wk, acc.w);
     }
   } else {
-    float M = -INFINITY;
+    M = -INFINITY;
     for (int u = tid; u < n; u += kMergeThreads) {
       const int sl = slot_of(u);
       if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
     }
     M = merge_reduce(M, true, s_red);
+    if (nv) M = fmaxf(M, zn);
     for (int c0 = 0; c0 < n; c0 += kMergeMax) {
       const int cn = min(kMergeMax, n - c0);
       float lpart = 0.f;
@@ -609,6 +788,16 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
         }
       }
       __syncthreads();  // s_w, s_slot are rewritten by the next pass
+    }
+  }
+  if (nv) {  // the step's token: one more partial (z_t, 1, V_t), added once (group 0 holds V_t)
+    const float wn = exp2f(zn - M);
+    L += wn;
+    if (grp == 0) {
+      acc.x = fmaf(vn.x, wn, acc.x);
+      acc.y = fmaf(vn.y, wn, acc.y);
+      acc.z = fmaf(vn.z, wn, acc.z);
+      acc.w = fmaf(vn.w, wn, acc.w);
     }
   }
   s_acc[grp][f4] = acc;
@@ -669,20 +858,28 @@ struct TcWorkspace {
   int32_t* prefix;
   float* ml;
   float* o;
+  int32_t* len;     // decode step: lengths the split kernel saw
+  float* step_ml;   // decode step: (m, l) of sequences finished inside one CTA
   size_t bytes;
 };
 
+// [prefix: B + 1 int32][ml: 2G x 32 x 2 f32][o: 2G x 32 x 128 f32][len: B int32][step ml: B x 32 x 2 f32],
+// each section 256-byte aligned.
 TcWorkspace carve(void* base, int batch, int grid) {
   TcWorkspace w;
   const size_t slots = 2 * static_cast<size_t>(grid);
   const size_t pb = round256((static_cast<size_t>(batch) + 1) * 4);
   const size_t mlb = round256(slots * kH * 2 * 4);
   const size_t ob = round256(slots * kH * kD * 4);
+  const size_t lb = round256(static_cast<size_t>(batch) * 4);
+  const size_t sb = round256(static_cast<size_t>(batch) * kH * 2 * 4);
   char* c = static_cast<char*>(base);
   w.prefix = reinterpret_cast<int32_t*>(c);
   w.ml = reinterpret_cast<float*>(c ? c + pb : nullptr);
   w.o = reinterpret_cast<float*>(c ? c + pb + mlb : nullptr);
-  w.bytes = pb + mlb + ob;
+  w.len = reinterpret_cast<int32_t*>(c ? c + pb + mlb + ob : nullptr);
+  w.step_ml = reinterpret_cast<float*>(c ? c + pb + mlb + ob + lb : nullptr);
+  w.bytes = pb + mlb + ob + lb + sb;
   return w;
 }
 
@@ -723,6 +920,8 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   p.ws_prefix = ws.prefix;
   p.ws_ml = ws.ml;
   p.ws_o = ws.o;
+  p.ws_len = ws.len;
+  p.step_ml = a.step ? ws.step_ml : nullptr;
   p.err = a.err;
   p.rope = a.rope;
   if (a.variant == kDecodeUmma) {
@@ -748,6 +947,32 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   mp.ws_ml = ws.ml;
   mp.ws_o = ws.o;
   mp.out = a.out;
+  if (a.step) {
+    TcStepParams& st = mp.st;
+    st.pos = a.q_pos;
+    st.a_k = static_cast<const __nv_bfloat16*>(a.step->a_k);
+    st.b_k = static_cast<const __nv_bfloat16*>(a.step->b_k);
+    st.a_v = static_cast<const __nv_bfloat16*>(a.step->a_v);
+    st.b_v = static_cast<const __nv_bfloat16*>(a.step->b_v);
+    st.q = static_cast<const __nv_bfloat16*>(a.q);
+    st.a_q = static_cast<const __nv_bfloat16*>(a.a_q);
+    st.r_q = a.r_q;
+    st.inv_rq = p.inv_rq;
+    st.r = cv.r_k;
+    st.zs = p.zs;
+    st.inv_rv = p.inv_rv;
+    st.capacity = cv.capacity;
+    st.advance = a.step->advance;
+    st.ws_len = ws.len;
+    st.step_ml = ws.step_ml;
+    st.c_ak = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.a_k));
+    st.c_bk = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.b_k));
+    st.c_av = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.a_v));
+    st.c_bv = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.b_v));
+    st.seq_lens = const_cast<int32_t*>(cv.seq_lens);
+    st.err = a.err;
+    st.rope = a.rope;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cv.batch, kH);
   cfg.blockDim = dim3(kMergeThreads);
@@ -757,7 +982,8 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel, mp);
+  if (a.step) return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<true>, mp);
+  return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<false>, mp);
 }
 
 }  // namespace tpa

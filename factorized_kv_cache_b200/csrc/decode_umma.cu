@@ -171,8 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tm_av) {
   constexpr int TOK = kRows / R;  // tokens per tile
   extern __shared__ uint8_t smem_raw[];
-  // the merge kernel may be scheduled now; it waits for this grid before reading
-  ptx::pdl_launch_dependents();
 
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -228,6 +226,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tbase = *s_taddr;
   ptx::pdl_wait();  // the cache, the lengths and the query are written by earlier work
+  // The merge kernel may be scheduled from here on: every CTA has passed its wait, so all
+  // work before this grid is complete and the merge may read the step's inputs at once
+  // (it waits for this grid before it reads anything written here).
+  ptx::pdl_launch_dependents();
 
   dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
   const int B = p.batch;
@@ -237,7 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int c = blockIdx.x;
   const int t_begin = NT == 0 ? 0 : dec::first_tile_fast(c, NT, p.grid, p.inv_grid);
   const int t_end = NT == 0 ? 0 : dec::first_tile_fast(c + 1, NT, p.grid, p.inv_grid);
+  // the lengths this grid saw, -1 where out of range, for the merge of a decode step
+  auto record_lengths = [&](int first, int step) {
+    for (int b = first; b < B; b += step) p.ws_len[b] = p.seq_lens[b] == s_len[b] ? s_len[b] : -1;
+  };
   if (t_begin >= t_end) {  // uniform: no tiles for this CTA
+    if (warp == 1 && blockIdx.x == 0 && p.step_ml) record_lengths(lane, 32);
     if (warp == 1) ptx::tmem_dealloc(tbase, kTmemCols);
     return;
   }
@@ -364,6 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every MMA issued by this thread completes before TMEM can be released
       ptx::umma_commit(fin);
       ptx::mbar_wait_bounded(fin, 0);
+    } else if (blockIdx.x == 0 && p.step_ml) {
+      record_lengths(lane - 1, 31);  // the other lanes of the MMA warp are idle
     }
   } else {
     // ---------------------------------------------------------------- softmax warps
@@ -652,6 +661,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < kHalf; ++h) {
           const float o = __uint_as_float(o0[h]) + __uint_as_float(o1[h]);
           op[h * kD] = l[h] > 0.f ? o / l[h] : 0.f;
+        }
+        if (p.step_ml && quad == 0 && lane < kHalf) {  // the step's own token joins in the merge kernel
+          float mk = m[0], lk = l[0];
+#pragma unroll
+          for (int h = 1; h < kHalf; ++h) {
+            mk = lane == h ? m[h] : mk;
+            lk = lane == h ? l[h] : lk;
+          }
+          const size_t e = (static_cast<size_t>(b) * kH + kHalf * hh + lane) * 2;
+          p.step_ml[e] = mk;
+          p.step_ml[e + 1] = lk;
         }
       } else {
         const int slot = 2 * c + (b == b_first ? 0 : 1);  // a shared sequence is the first or the last one

@@ -72,10 +72,11 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double theta, float* c, fl
   sincosf(static_cast<float>(r), s, c);
 }
 
-// Rotate the pair (x, y): (x c - y s, x s + y c), in fp32.
+// Rotate the pair (x, y): (x c - y s, x s + y c), in fp32, with the roundings
+// spelled out so that every kernel that rotates the same pair gets the same bits.
 __device__ __forceinline__ void rope_pair(float& x, float& y, float c, float s) {
-  const float xr = x * c - y * s;
-  const float yr = x * s + y * c;
+  const float xr = __fmaf_rn(x, c, -__fmul_rn(y, s));
+  const float yr = __fmaf_rn(x, s, __fmul_rn(y, c));
   x = xr;
   y = yr;
 }

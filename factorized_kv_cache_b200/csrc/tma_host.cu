@@ -23,8 +23,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 }  // namespace
 
-cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
-                           uint32_t box_rows, int swizzle_bytes) {
+namespace {
+
+cudaError_t encode_uncached(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                            uint32_t box_rows, int swizzle_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return cudaErrorNotSupported;
   CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -39,6 +41,39 @@ cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, u
                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// The last kMapCache descriptions encoded on this host thread.  A map depends only on these
+// arguments (an address range and its tiling), so a hit is the map the driver would return.
+constexpr int kMapCache = 32;
+struct MapEntry {
+  const void* base;
+  uint64_t inner, rows;
+  uint32_t box_inner, box_rows;
+  int swizzle;
+  bool valid;
+  CUtensorMap map;
+};
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_next = 0;
+
+}  // namespace
+
+cudaError_t encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                           uint32_t box_rows, int swizzle_bytes) {
+  for (const MapEntry& e : t_maps) {
+    if (e.valid && e.base == base && e.inner == inner && e.rows == rows && e.box_inner == box_inner &&
+        e.box_rows == box_rows && e.swizzle == swizzle_bytes) {
+      *map = e.map;
+      return cudaSuccess;
+    }
+  }
+  const cudaError_t r = encode_uncached(map, base, inner, rows, box_inner, box_rows, swizzle_bytes);
+  if (r != cudaSuccess) return r;
+  MapEntry& e = t_maps[t_next];
+  t_next = (t_next + 1) % kMapCache;
+  e = MapEntry{base, inner, rows, box_inner, box_rows, swizzle_bytes, true, *map};
+  return cudaSuccess;
 }
 
 }  // namespace tpa

@@ -174,10 +174,19 @@ void set_last_error_message(const char* fmt, ...) {
   t_last_error = buf;
 }
 
+// theta_j = base^(-2j/d_h); the last table built on this host thread is reused.
 void make_rope_table(double base, int head_dim, RopeTable* t) {
-  memset(t, 0, sizeof(*t));
-  for (int j = 0; j < head_dim / 2 && j < kMaxPairs; ++j)
-    t->theta[j] = pow(base, -2.0 * static_cast<double>(j) / static_cast<double>(head_dim));
+  thread_local double t_base = 0.0;
+  thread_local int t_dim = 0;
+  thread_local RopeTable t_table;
+  if (t_dim != head_dim || t_base != base) {
+    memset(&t_table, 0, sizeof(t_table));
+    for (int j = 0; j < head_dim / 2 && j < kMaxPairs; ++j)
+      t_table.theta[j] = pow(base, -2.0 * static_cast<double>(j) / static_cast<double>(head_dim));
+    t_base = base;
+    t_dim = head_dim;
+  }
+  *t = t_table;
 }
 
 }  // namespace tpa
@@ -260,10 +269,11 @@ size_t tpa_decode_workspace_size(const tpa_cache* cache, int32_t max_len, int32_
 
 namespace {
 
-// Decode with a dense query (r_q == 0) or a factorized one (a_q, q = B_Q, r_q >= 1).
+// Decode with a dense query (r_q == 0) or a factorized one (a_q, q = B_Q, r_q >= 1); with
+// `step`, the query's own token is appended and attended in the same launches.
 tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, int32_t r_q, const int32_t* q_pos,
                        float scale, float* out, int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+                       size_t workspace_bytes, void* stream, const DecodeStepArgs* step = nullptr) {
   tpa_status s = check_cache(cache);
   if (s != TPA_OK) return s;
   if (!q || !q_pos || !out) return fail(TPA_ERR_NULL, "q, q_pos or out is NULL");
@@ -290,6 +300,19 @@ tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, i
                   "a factorized decode query needs the tcgen05 kernel: bf16, heads 32, head_dim 128, "
                   "r_k == r_v <= 2, batch <= 1024, kernel AUTO or TENSOR");
     if (reinterpret_cast<uintptr_t>(a_q) & 1u) return fail(TPA_ERR_ALIGNMENT, "a_q must be 2-byte aligned");
+  }
+  if (step) {
+    if (!step->a_k || !step->b_k || !step->a_v || !step->b_v)
+      return fail(TPA_ERR_NULL, "a factor of the step's token is NULL");
+    if (step->advance != 0 && step->advance != 1) return fail(TPA_ERR_SHAPE, "advance = %d", step->advance);
+    if (kernel == TPA_KERNEL_SIMT || kernel == TPA_KERNEL_TENSOR_SYNC ||
+        !tensor_decode_supported(cache->dtype, cache->heads, cache->head_dim, cache->r_k, cache->r_v) ||
+        !tensor_decode_batch_ok(cache->batch))
+      return fail(TPA_ERR_UNSUPPORTED,
+                  "a decode step needs the tcgen05 kernel: bf16, heads 32, head_dim 128, r_k == r_v <= 2, "
+                  "batch <= 1024, kernel AUTO or TENSOR");
+    if (!aligned16(step->a_k) || !aligned16(step->b_k) || !aligned16(step->a_v) || !aligned16(step->b_v))
+      return fail(TPA_ERR_ALIGNMENT, "the step's factors must be 16-byte aligned");
   }
   int sms = 0;
   unsigned int* err = nullptr;
@@ -322,6 +345,7 @@ tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, i
     a.rope = rope;
     a.err = err;
     a.variant = variant;
+    a.step = step;
     e = launch_tensor_decode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
     return TPA_OK;
@@ -383,6 +407,21 @@ tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, co
   if (r_q < 1) return fail(TPA_ERR_SHAPE, "r_q = %d < 1", r_q);
   return decode_impl(cache, b_q, a_q, r_q, q_pos, scale, out, max_len, num_splits, kernel, workspace,
                      workspace_bytes, stream);
+}
+
+tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, const void* a_k, const void* b_k,
+                           const void* a_v, const void* b_v, int32_t r_q, const void* a_q, const void* q, float scale,
+                           float* out, int32_t max_len, int32_t advance, int32_t num_splits, int32_t kernel,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (r_q < 0) return fail(TPA_ERR_SHAPE, "r_q = %d < 0", r_q);
+  DecodeStepArgs step;
+  step.a_k = a_k;
+  step.b_k = b_k;
+  step.a_v = a_v;
+  step.b_v = b_v;
+  step.advance = advance;
+  return decode_impl(cache, q, r_q > 0 ? a_q : nullptr, r_q, positions, scale, out, max_len, num_splits, kernel,
+                     workspace, workspace_bytes, stream, &step);
 }
 
 size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q, int32_t kernel) {

@@ -20,6 +20,16 @@ bool tensor_decode_batch_ok(int batch);
 int tensor_decode_default_ctas(int sms, int variant);
 size_t tensor_decode_workspace_bytes(int batch, int grid);
 
+// A decode step: the token being generated is stored at slot seq_lens[b] and attended by its
+// own query (tcgen05 kernel only; the query position is that token's position).
+struct DecodeStepArgs {
+  const void* a_k;  // [B][R_K][h] bf16
+  const void* b_k;  // [B][R_K][d_h] bf16, unrotated
+  const void* a_v;  // [B][R_V][h]
+  const void* b_v;  // [B][R_V][d_h]
+  int advance;      // 1: seq_lens[b] += 1 after the step
+};
+
 struct TensorDecodeArgs {
   CacheView cache;
   const void* q;       // dense query [B][h][d_h], or B_Q [B][r_q][d_h] when r_q > 0
@@ -34,6 +44,7 @@ struct TensorDecodeArgs {
   RopeTable rope;
   unsigned int* err;
   int variant;  // kDecodeUmma or kDecodeSync
+  const DecodeStepArgs* step;  // null for a plain decode
 };
 cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream);
 

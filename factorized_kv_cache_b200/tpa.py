@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_decode_attention_noalloc": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P]),
         "tpa_decode_attention_factored": (ctypes.c_int, [C, I32, P, P, P, ctypes.c_float, P, I32, I32, I32, P,
                                                           ctypes.c_size_t, P]),
+        "tpa_decode_step": (ctypes.c_int, [C, P, P, P, P, P, I32, P, P, ctypes.c_float, P, I32, I32, I32, I32, P,
+                                            ctypes.c_size_t, P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
@@ -114,9 +116,16 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream(stream, device=None) -> ctypes.c_void_p:
+    """The cudaStream_t to launch on: `stream`, else the current stream of `device`."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        if _raw_current_stream is not None:
+            idx = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+            return ctypes.c_void_p(_raw_current_stream(idx))
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -182,6 +191,17 @@ class TpaCache:
         return self.a_k.dtype
 
     def struct(self) -> tpa_cache:
+        """The C descriptor, rebuilt (and re-checked) only when a plane tensor or the base changed."""
+        planes = (self.a_k, self.b_k, self.a_v, self.b_v, self.seq_lens)
+        key = tuple((id(t), t.data_ptr(), t.shape) for t in planes) + (self.rope_base,)
+        hit = self.__dict__.get("_struct_cache")
+        if hit is not None and hit[0] == key:
+            return hit[1]
+        s = self._build_struct()
+        self.__dict__["_struct_cache"] = (key, s)
+        return s
+
+    def _build_struct(self) -> tpa_cache:
         B, cap, rk, h = self.a_k.shape
         d = self.b_k.shape[3]
         rv = self.a_v.shape[2]
@@ -220,7 +240,7 @@ def tpa_cache_append(cache: TpaCache, positions, a_k, b_k, a_v, b_v, stream=None
     _need(b_v, "b_v", dt, (B, n_new, cache.r_v, cache.head_dim), dev)
     s = cache.struct()
     _check(lib.tpa_cache_append(ctypes.byref(s), n_new, _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v),
-                                _ptr(b_v), _stream(stream)))
+                                _ptr(b_v), _stream(stream, dev)))
 
 
 def tpa_cache_write_slots(cache: TpaCache, slots, positions, a_k, b_k, a_v, b_v, stream=None):
@@ -237,7 +257,7 @@ def tpa_cache_write_slots(cache: TpaCache, slots, positions, a_k, b_k, a_v, b_v,
     _need(b_v, "b_v", dt, (B, n_new, cache.r_v, cache.head_dim), dev)
     s = cache.struct()
     _check(lib.tpa_cache_write_slots(ctypes.byref(s), n_new, _ptr(slots), _ptr(positions), _ptr(a_k), _ptr(b_k),
-                                     _ptr(a_v), _ptr(b_v), _stream(stream)))
+                                     _ptr(a_v), _ptr(b_v), _stream(stream, dev)))
 
 
 def tpa_decode_default_splits(cache: TpaCache, max_len: int, kernel: int = TPA_KERNEL_AUTO) -> int:
@@ -279,7 +299,7 @@ def tpa_decode_attention(cache: TpaCache, q, q_pos, scale: float | None = None, 
         workspace_buf = workspace(need, dev)
     nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
     _check(lib.tpa_decode_attention(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out), max_len,
-                                    num_splits, kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+                                    num_splits, kernel, _ptr(workspace_buf), nbytes, _stream(stream, dev)))
     return out
 
 
@@ -309,8 +329,105 @@ def tpa_decode_attention_factored(cache: TpaCache, a_q, b_q, q_pos, scale: float
     nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
     _check(lib.tpa_decode_attention_factored(ctypes.byref(s), r_q, _ptr(a_q), _ptr(b_q), _ptr(q_pos), float(scale),
                                              _ptr(out), max_len, num_splits, kernel, _ptr(workspace_buf), nbytes,
-                                             _stream(stream)))
+                                             _stream(stream, dev)))
     return out
+
+
+def tpa_decode_step(cache: TpaCache, positions, a_k, b_k, a_v, b_v, q=None, a_q=None, b_q=None,
+                    scale: float | None = None, out=None, max_len: int | None = None, advance: bool = True,
+                    num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO, workspace_buf=None, stream=None):
+    """One fused generation step: store the token's factors (a_k [B, R_K, h], b_k [B, R_K, d_h]
+    unrotated, a_v, b_v) at slot seq_lens[b] and attend with its query, dense (q [B, h, d_h]) or
+    in TPA form (a_q [B, R_Q, h], b_q [B, R_Q, d_h]), at positions [B]; returns out [B, h, d_h]
+    float32.  advance=False leaves seq_lens unchanged."""
+    lib = load_library()
+    B, h, d = cache.batch, cache.heads, cache.head_dim
+    dev, dt = cache.a_k.device, cache.dtype
+    _need(positions, "positions", torch.int32, (B,), dev)
+    _need(a_k, "a_k", dt, (B, cache.r_k, h), dev)
+    _need(b_k, "b_k", dt, (B, cache.r_k, d), dev)
+    _need(a_v, "a_v", dt, (B, cache.r_v, h), dev)
+    _need(b_v, "b_v", dt, (B, cache.r_v, d), dev)
+    if q is not None:
+        if a_q is not None or b_q is not None:
+            raise ValueError("pass either q or (a_q, b_q)")
+        _need(q, "q", dt, (B, h, d), dev)
+        r_q, qa, qb = 0, None, q
+    else:
+        if a_q is None or b_q is None:
+            raise ValueError("pass q or both a_q and b_q")
+        r_q = a_q.shape[1]
+        _need(a_q, "a_q", dt, (B, r_q, h), dev)
+        _need(b_q, "b_q", dt, (B, r_q, d), dev)
+        qa, qb = a_q, b_q
+    if out is None:
+        out = torch.empty(B, h, d, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, (B, h, d), dev)
+    if max_len is None:
+        max_len = cache.capacity
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(int(lib.tpa_decode_workspace_size(ctypes.byref(s), max_len, num_splits, kernel)),
+                                  dev)
+    nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+    _check(lib.tpa_decode_step(ctypes.byref(s), _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v), _ptr(b_v), r_q,
+                               _ptr(qa), _ptr(qb), float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits,
+                               kernel, _ptr(workspace_buf), nbytes, _stream(stream, dev)))
+    return out
+
+
+class DecodeStepPlan:
+    """tpa_decode_step bound to fixed buffers, for a generation loop: the arguments are checked
+    and marshalled once, and each call is a single C call with the stored pointers.  The
+    buffers' contents may change between calls (new factors, query, positions); the tensors
+    themselves, and the cache's planes, must stay the same objects."""
+
+    def __init__(self, cache: TpaCache, positions, a_k, b_k, a_v, b_v, out, q=None, a_q=None, b_q=None,
+                 scale: float | None = None, max_len: int | None = None, advance: bool = True, num_splits: int = 0,
+                 kernel: int = TPA_KERNEL_AUTO, workspace_buf=None):
+        lib = load_library()
+        B, h, d = cache.batch, cache.heads, cache.head_dim
+        dev, dt = cache.a_k.device, cache.dtype
+        _need(positions, "positions", torch.int32, (B,), dev)
+        _need(a_k, "a_k", dt, (B, cache.r_k, h), dev)
+        _need(b_k, "b_k", dt, (B, cache.r_k, d), dev)
+        _need(a_v, "a_v", dt, (B, cache.r_v, h), dev)
+        _need(b_v, "b_v", dt, (B, cache.r_v, d), dev)
+        _need(out, "out", torch.float32, (B, h, d), dev)
+        if q is not None:
+            if a_q is not None or b_q is not None:
+                raise ValueError("pass either q or (a_q, b_q)")
+            _need(q, "q", dt, (B, h, d), dev)
+            r_q, qa, qb = 0, None, q
+        else:
+            if a_q is None or b_q is None:
+                raise ValueError("pass q or both a_q and b_q")
+            r_q = a_q.shape[1]
+            _need(a_q, "a_q", dt, (B, r_q, h), dev)
+            _need(b_q, "b_q", dt, (B, r_q, d), dev)
+            qa, qb = a_q, b_q
+        if max_len is None:
+            max_len = cache.capacity
+        if scale is None:
+            scale = 1.0 / math.sqrt(d)
+        self._struct = cache.struct()
+        if workspace_buf is None:
+            workspace_buf = workspace(
+                int(lib.tpa_decode_workspace_size(ctypes.byref(self._struct), max_len, num_splits, kernel)), dev)
+        nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+        self.out = out
+        self._keep = (cache, positions, a_k, b_k, a_v, b_v, qa, qb, out, workspace_buf)
+        self._device = dev
+        self._fn = lib.tpa_decode_step
+        self._args = (ctypes.byref(self._struct), _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v), _ptr(b_v), r_q,
+                      _ptr(qa), _ptr(qb), float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits, kernel,
+                      _ptr(workspace_buf), nbytes)
+
+    def __call__(self, stream=None):
+        _check(self._fn(*self._args, _stream(stream, self._device)))
+        return self.out
 
 
 def tpa_decode_attention_noalloc(cache: TpaCache, q, q_pos, out, scale: float | None = None,
@@ -332,7 +449,7 @@ def tpa_decode_attention_noalloc(cache: TpaCache, q, q_pos, out, scale: float | 
         scale = 1.0 / math.sqrt(d)
     s = cache.struct()
     _check(lib.tpa_decode_attention_noalloc(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out),
-                                            max_len, num_splits, kernel, _stream(stream)))
+                                            max_len, num_splits, kernel, _stream(stream, dev)))
     return out
 
 
@@ -364,7 +481,7 @@ def tpa_prefill_attention(cache: TpaCache, a_q, b_q, q_pos, scale: float | None 
         workspace_buf = workspace(need, dev)
     nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
     _check(lib.tpa_prefill_attention(ctypes.byref(s), T, r_q, _ptr(a_q), _ptr(b_q), _ptr(q_pos), float(scale),
-                                     _ptr(out), kernel, _ptr(workspace_buf), nbytes, _stream(stream)))
+                                     _ptr(out), kernel, _ptr(workspace_buf), nbytes, _stream(stream, dev)))
     return out
 
 

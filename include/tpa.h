@@ -198,6 +198,41 @@ tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, co
                                          void* stream);
 
 /*
+ * One generation step of token x_t, fused: its factors are appended and its
+ * query attends the cache including x_t itself (section 解决思路: Q_t, K_t, V_t
+ * all come from x_t; Theorem 3.1: B_K and the query rotate at x_t's position).
+ *   positions [batch] int32, device: x_t's position (its key's and its query's);
+ *   a_k [batch][r_k][heads], b_k [batch][r_k][head_dim] (NOT rotated),
+ *   a_v [batch][r_v][heads], b_v [batch][r_v][head_dim]: device, bf16,
+ *     16-byte aligned: x_t's factors;
+ *   the query: r_q == 0: q [batch][heads][head_dim] dense, a_q unused;
+ *     r_q in [1, 8]: TPA form as in tpa_decode_attention_factored, a_q
+ *     [batch][r_q][heads] and q = b_q [batch][r_q][head_dim]; not rotated;
+ *   out [batch][heads][head_dim] float32: attention of the query over slots
+ *     0 .. L of sequence b, where L = seq_lens[b] on entry and slot L now
+ *     holds x_t (B_K stored rotated, exactly as tpa_cache_append stores it);
+ *   advance: 1 = seq_lens[b] becomes L + 1 (generation); 0 = seq_lens is left
+ *     at L, so the next call overwrites the same slot (a fixed-length cache,
+ *     or a token that may be rejected);
+ *   max_len: host upper bound on every seq_lens[b] on entry; num_splits,
+ *     kernel, workspace, workspace_bytes: as tpa_decode_attention
+ *     (tpa_decode_workspace_size(cache, max_len, num_splits, TPA_KERNEL_TENSOR)).
+ * Two launches (the split kernel over the tokens cached before the step and
+ * the merge, which forms x_t's own score and value, stores x_t and joins it
+ * to the log-sum-exp), against three for tpa_cache_append followed by
+ * tpa_decode_attention.  If L == capacity, x_t is neither stored nor
+ * attended, seq_lens is unchanged and TPA_DEVERR_APPEND_OVERFLOW is set.
+ * Runs on the tcgen05 kernel only (same shapes as
+ * tpa_decode_attention_factored); anything else returns TPA_ERR_UNSUPPORTED.
+ * Errors: those of tpa_decode_attention, SHAPE (r_q < 0 or advance not 0/1),
+ * NULL (a factor of x_t), UNSUPPORTED.
+ */
+tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, const void* a_k, const void* b_k,
+                           const void* a_v, const void* b_v, int32_t r_q, const void* a_q, const void* q,
+                           float scale, float* out, int32_t max_len, int32_t advance, int32_t num_splits,
+                           int32_t kernel, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * tpa_decode_attention for callers that cannot allocate device memory (no
  * counterpart on the page; this is a deployment convenience).  Same
  * arguments and result as tpa_decode_attention minus the workspace: the

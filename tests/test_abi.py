@@ -98,6 +98,32 @@ def test_factored_decode_rejects_bad_arguments():
     assert lib.tpa_last_error_message().decode() != ""
 
 
+def test_decode_step_rejects_bad_arguments():
+    lib = T.load_library()
+    P = 0x90000
+
+    def call(c=None, pos=0x70000, ak=P, bk=P, av=P, bv=P, rq=0, a_q=None, q=0x60000, advance=1, kernel=0):
+        c = _fake_cache() if c is None else c
+        return lib.tpa_decode_step(ctypes.byref(c), pos, ak, bk, av, bv, rq, a_q, q, 0.1, 0x80000, 64, advance, 0,
+                                   kernel, None, 0, None)
+
+    assert call(rq=-1) == 2
+    assert call(advance=2) == 2
+    assert call(pos=None) == 1
+    assert call(q=None) == 1
+    for k in ("ak", "bk", "av", "bv"):
+        assert call(**{k: None}) == 1
+        assert call(**{k: P + 4}) == 6
+    assert call(rq=3, a_q=None) == 1
+    assert call(rq=9, a_q=P) == 3
+    assert call(c=_fake_cache(dtype=T.TPA_F32)) == 3   # tcgen05 kernel only
+    assert call(c=_fake_cache(r_k=2, r_v=1)) == 3
+    assert call(c=_fake_cache(batch=1025)) == 3
+    assert call(kernel=T.TPA_KERNEL_SIMT) == 3
+    assert call(kernel=T.TPA_KERNEL_TENSOR_SYNC) == 3
+    assert lib.tpa_last_error_message().decode() != ""
+
+
 def test_append_rejects_bad_arguments():
     lib = T.load_library()
     c = _fake_cache()
