@@ -396,12 +396,17 @@ def run_ours_decode(args, w, rank, world, dev):
     mean_decode_s = statistics.mean(decode_ms) / 1e3
     peaks, kind = measured_peaks()
     achieved = bytes_per_decode / mean_decode_s / 1e9
+    # the dominant kernel's source and the headers it includes (the traffic figure is reused
+    # only while all of them are unchanged)
+    hdrs = ["factorized_kv_cache_b200/csrc/device_common.cuh", "factorized_kv_cache_b200/csrc/ptx_sm100.cuh"]
     if kernel == T.TPA_KERNEL_SIMT or w.dtype == "f32":
-        kernel_src = ["factorized_kv_cache_b200/csrc/attention_simt.cu"]
+        kernel_src = ["factorized_kv_cache_b200/csrc/attention_simt.cu"] + hdrs
     elif kernel == T.TPA_KERNEL_TENSOR_SYNC:
-        kernel_src = ["factorized_kv_cache_b200/csrc/decode_tensor.cu"]
+        kernel_src = ["factorized_kv_cache_b200/csrc/decode_tensor.cu",
+                      "factorized_kv_cache_b200/csrc/decode_common.cuh"] + hdrs
     else:
-        kernel_src = ["factorized_kv_cache_b200/csrc/decode_umma.cu"]
+        kernel_src = ["factorized_kv_cache_b200/csrc/decode_umma.cu",
+                      "factorized_kv_cache_b200/csrc/decode_common.cuh"] + hdrs
     kernel_src = [p for p in kernel_src if os.path.exists(os.path.join(ROOT, p))]
     res = {
         "metric": METRIC,
