@@ -451,6 +451,176 @@ def run_ours_decode(args, w, rank, world, dev):
     return res, x, lengths
 
 
+def run_ours_decode_sharded(args, w, rank, world, dev):
+    """Strong scaling of one batch: rank r holds, for every sequence, the token range
+    token_range(L_b, world, r) at the tokens' global positions, decodes it with
+    tpa_decode_attention_lse, and the ranks all-gather (out, lse) and merge them with
+    tpa_merge_lse, so every rank ends with the output of the whole range."""
+    import torch
+    import torch.distributed as dist
+    from factorized_kv_cache_b200 import sharded
+    from factorized_kv_cache_b200 import tpa as T
+
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    esize = 4 if w.dtype == "f32" else 2
+    x = decode_host_inputs(w, 0)                 # the same batch on every rank
+    B, cap = x["a_k"].shape[:2]
+    lengths = x["lengths"].numpy().astype(np.int64)
+    ranges = [sharded.token_range(int(L), world, rank) for L in lengths]
+    shard_lens = np.array([e - s for s, e in ranges], dtype=np.int64)
+    scap = max(1, int(shard_lens.max()))
+    # tokens [s_b, s_b + scap) of each sequence (indices past the sequence clamp to its last
+    # slot: they sit past the shard's length and are never attended)
+    idx = np.stack([np.minimum(np.arange(scap) + s, cap - 1) for s, _ in ranges])
+    rows = torch.arange(B)[:, None]
+    tix = torch.from_numpy(idx)
+    per_tok = (w.r_k + w.r_v) * (w.heads + w.head_dim) * esize
+    shard_bytes = B * scap * per_tok
+    copies = 1 if shard_bytes >= 2 * L2_BYTES else int(math.ceil(2 * L2_BYTES / shard_bytes)) + 1
+    c0 = T.TpaCache.allocate(B, scap, w.heads, w.head_dim, w.r_k, w.r_v, dtype=dt, rope_base=w.rope_base, device=dev)
+    T.tpa_cache_append(c0, x["positions"][rows, tix].contiguous().to(dev),
+                       *(x[k][rows, tix].contiguous().to(dev) for k in ("a_k", "b_k", "a_v", "b_v")))
+    c0.seq_lens.copy_(torch.from_numpy(shard_lens.astype(np.int32)).to(dev))
+    caches = [c0] + [T.TpaCache(c0.a_k.clone(), c0.b_k.clone(), c0.a_v.clone(), c0.b_v.clone(), c0.seq_lens.clone(),
+                                w.rope_base) for _ in range(copies - 1)]
+    q = x["q"].to(dev)
+    q_pos = x["q_pos"].to(dev)
+    out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, w.heads, dtype=torch.float32, device=dev)
+    res = torch.empty_like(out)
+    res_lse = torch.empty_like(lse)
+    ws = T.workspace(T.tpa_decode_workspace_size(c0, scap, 0, T.TPA_KERNEL_AUTO), dev)
+
+    def local(c, qv=q):
+        T.tpa_decode_attention_lse(caches[c], qv, q_pos, out=out, lse=lse, max_len=scap, workspace_buf=ws)
+
+    def exchange_merge():
+        if world > 1:
+            parts_out, parts_lse = sharded.all_gather_partials(out, lse)
+        else:
+            parts_out, parts_lse = out[None], lse[None]
+        T.tpa_merge_lse(parts_out, parts_lse, out=res, lse_out=res_lse)
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for c in range(copies):
+            local(c)
+            exchange_merge()
+    torch.cuda.synchronize(dev)
+    gl = []
+    for c in range(copies):
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            local(c)
+        gl.append(g1)
+    n_calls = copies * max(1, math.ceil(4 / copies))
+    gd = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gd, stream=stream):
+        for k in range(n_calls):
+            local(k % copies)
+    torch.cuda.synchronize(dev)
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for k in range(W):
+            gl[k % copies].replay()
+            exchange_merge()
+        gd.replay()
+    torch.cuda.synchronize(dev)
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set after set-up")
+    reps = max(1, K // n_calls)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for k in range(K):
+            gl[(W + k) % copies].replay()
+            exchange_merge()
+        t_end.record(stream)
+        for r in range(reps):
+            ev[r][0].record(stream)
+            gd.replay()
+            ev[r][1].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    local_s = statistics.mean(a.elapsed_time(b) / n_calls for a, b in ev) / 1e3
+    if T.tpa_read_device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    # e2e: the query from pinned host memory, the merged output back, every step
+    host_q = x["q"].pin_memory()
+    host_out = torch.empty(B, w.heads, w.head_dim, dtype=torch.float32).pin_memory()
+    dev_q = torch.empty_like(q)
+    e2e_steps = max(1, min(K, 500))
+
+    def e2e_step(c):
+        with torch.cuda.stream(stream):
+            dev_q.copy_(host_q, non_blocking=True)
+            local(c, dev_q)
+            exchange_merge()
+            host_out.copy_(res, non_blocking=True)
+        stream.synchronize()
+
+    for k in range(min(W, 10)):
+        e2e_step(k % copies)
+    if world > 1:
+        dist.barrier()
+    t0 = time.perf_counter()
+    for k in range(e2e_steps):
+        e2e_step(k % copies)
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
+
+    tokens = int(lengths.sum())
+    local_bytes = int(shard_lens.sum()) * per_tok + B * w.heads * w.head_dim * (esize + 4) + B * w.heads * 4
+    peaks, kind = measured_peaks()
+    achieved = local_bytes / local_s / 1e9
+    res_json = {
+        "metric": METRIC,
+        "value": tokens * K / (elapsed_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": elapsed_ms / K,
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded Philox normals; A~N(0,1), B~N(0,1/d_h), q~N(0,1))",
+        "config": {
+            "workload": w.name, "batch": B, "seq_len": int(lengths.max()), "heads": w.heads, "head_dim": w.head_dim,
+            "r_k": w.r_k, "r_v": w.r_v, "tokens_attended_per_step": tokens,
+            "shard": f"token ranges over {world} rank(s); this rank holds {int(shard_lens.sum())} tokens",
+            "step": "tpa_decode_attention_lse on the local range (one CUDA graph) + all-gather of (out, lse) + "
+                    "tpa_merge_lse",
+            "l2": (f"inputs larger than L2: {copies} cache copies rotated" if copies > 1 else
+                   f"inputs larger than L2 ({shard_bytes / 2**20:.0f} MiB)"),
+            "parallelism": f"token-sharded x{world} (one all-gather per step)",
+        },
+        "roofline": {
+            "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_kind": kind,
+            "kernel": "local decode call with lse (split kernel + merge), graphs of back-to-back calls",
+            "calls_per_graph": n_calls, "algorithmic_bytes_per_launch": local_bytes,
+            "mean_launch_us": local_s * 1e6,
+        },
+        "e2e": {"value": tokens * e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": q.numel() * esize,
+                "d2h_bytes_per_step": host_out.numel() * 4, "steps": e2e_steps},
+        "gpu_launches": K * 3,
+        "clocks": clk,
+    }
+    return res_json, x, lengths
+
+
 def _host_arrays(x, lengths):
     host = {k: x[k].float().numpy() for k in ("a_k", "b_k", "a_v", "b_v", "q")}
     host["lengths"] = lengths
@@ -731,6 +901,8 @@ def main():
                     help="decode workloads: 0 = dense query; R_Q > 0 = query given as TPA factors A_Q, B_Q")
     ap.add_argument("--step", choices=["fused", "two_call"], default="fused",
                     help="decode step: tpa_decode_step (tcgen05 path), or tpa_cache_write_slots + decode")
+    ap.add_argument("--shard-tokens", action="store_true",
+                    help="decode workloads: split every sequence's token range across the ranks (strong scaling)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")
@@ -768,6 +940,10 @@ def main():
             res, x = run_ours_prefill(args, w, rank, world, dev)
             if rank == 0 and args.cpu_seconds > 0:
                 add_prefill_cpu_baseline(res, x, w, args.cpu_seconds)
+        elif args.shard_tokens:
+            res, x, lengths = run_ours_decode_sharded(args, w, rank, world, dev)
+            if rank == 0 and args.cpu_seconds > 0:
+                add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
         else:
             res, x, lengths = run_ours_decode(args, w, rank, world, dev)
             if rank == 0 and args.cpu_seconds > 0:

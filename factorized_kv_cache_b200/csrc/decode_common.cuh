@@ -36,11 +36,12 @@ struct DecodeTcParams {
   int32_t* ws_prefix;      // [B + 1]
   float* ws_ml;            // [2G][32][2]
   float* ws_o;             // [2G][32][128]
-  // Set for a decode step (append + attend, see decode_tensor.cu): the merge kernel adds the
-  // step's own token.  CTA 0 records the lengths it saw (-1: out of range), and a sequence
-  // finished inside one CTA also leaves its (m, l) per head beside its normalised output.
-  int32_t* ws_len;         // [B]
-  float* step_ml;          // [B][32][2], or null for a plain decode
+  // A decode step (append + attend, see decode_tensor.cu): CTA 0 records the lengths it saw
+  // (-1: out of range) for the merge kernel, which adds the step's own token.
+  int32_t* ws_len;         // [B], or null when no step follows
+  // A decode step, or a decode that also returns each head's log-sum-exp: a sequence finished
+  // inside one CTA leaves its (m, l) per head beside its normalised output.
+  float* whole_ml;         // [B][32][2], or null
   unsigned int* err;
   RopeTable rope;
 };

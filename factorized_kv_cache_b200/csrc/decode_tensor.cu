@@ -512,7 +512,6 @@ struct TcStepParams {
   int capacity;
   int advance;
   const int32_t* ws_len;          // lengths the split kernel saw (-1: out of range)
-  const float* step_ml;           // (m, l) of the sequences it finished inside one CTA
   __nv_bfloat16* c_ak;            // the cache planes and lengths
   __nv_bfloat16* c_bk;
   __nv_bfloat16* c_av;
@@ -528,8 +527,12 @@ struct TcMergeParams {
   const float* ws_ml;
   const float* ws_o;
   float* out;
-  TcStepParams st;  // read only by the step variant
+  float* lse;              // [B][32] natural-log log-sum-exp of the scaled scores, or null
+  const float* whole_ml;   // (m, l) of the sequences the split kernel finished inside one CTA
+  TcStepParams st;         // read only by the step variant
 };
+
+constexpr float kLn2 = 0.6931471805599453f;
 
 constexpr int kMergeThreads = 256;
 constexpr int kMergeGroups = kMergeThreads / 32;
@@ -685,21 +688,30 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
   }
 
   float* o = p.out + (static_cast<size_t>(b) * kH + i) * kD;
+  float* lse = p.lse ? p.lse + static_cast<size_t>(b) * kH + i : nullptr;
+  // natural-log log-sum-exp from a maximum and a sum in log2 units
+  auto write_lse = [&](float m2, float l) {
+    if (lse && tid == 0) *lse = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
+  };
   if (t1 <= t0) {  // nothing cached: the step's token alone, or zeros
     if (tid < 32) reinterpret_cast<float4*>(o)[tid] = nv ? vn : make_float4(0.f, 0.f, 0.f, 0.f);
+    write_lse(nv ? zn : 0.f, nv ? 1.f : 0.f);
     return;
   }
   const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
   if (cs == ce) {  // finished by the split kernel
-    if (kStep && nv && tid < 32) {
-      const float2 ml = reinterpret_cast<const float2*>(p.st.step_ml)[static_cast<size_t>(b) * kH + i];
-      const float4 on = reinterpret_cast<const float4*>(o)[tid];
-      const float M = fmaxf(ml.x, zn);
+    if (nv || lse) {
+      const float2 ml = reinterpret_cast<const float2*>(p.whole_ml)[static_cast<size_t>(b) * kH + i];
+      const float M = nv ? fmaxf(ml.x, zn) : ml.x;
       const float wo = (ml.x == -INFINITY ? 0.f : exp2f(ml.x - M)) * ml.y;
-      const float wn = exp2f(zn - M);
-      const float inv = 1.f / (wo + wn);
-      reinterpret_cast<float4*>(o)[tid] = make_float4((on.x * wo + vn.x * wn) * inv, (on.y * wo + vn.y * wn) * inv,
-                                                      (on.z * wo + vn.z * wn) * inv, (on.w * wo + vn.w * wn) * inv);
+      const float wn = nv ? exp2f(zn - M) : 0.f;
+      if (nv && tid < 32) {
+        const float4 on = reinterpret_cast<const float4*>(o)[tid];
+        const float inv = 1.f / (wo + wn);
+        reinterpret_cast<float4*>(o)[tid] = make_float4((on.x * wo + vn.x * wn) * inv, (on.y * wo + vn.y * wn) * inv,
+                                                        (on.z * wo + vn.z * wn) * inv, (on.w * wo + vn.w * wn) * inv);
+      }
+      write_lse(M, wo + wn);
     }
     return;
   }
@@ -716,7 +728,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
   };
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float M;
+  float M;  // the maximum of the partials' maxima (and the step token's score), log2 units
   if (n <= kMergeGroups * kMergeBatch) {
     // one pass: every partial's features and (m, l) are loaded at once, before the maximum is known
     float4 v[kMergeBatch];
@@ -814,6 +826,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     const float inv = L > 0.f ? 1.f / L : 0.f;
     reinterpret_cast<float4*>(o)[tid] = make_float4(r.x * inv, r.y * inv, r.z * inv, r.w * inv);
   }
+  write_lse(M, L);
 }
 
 size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
@@ -920,8 +933,8 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   p.ws_prefix = ws.prefix;
   p.ws_ml = ws.ml;
   p.ws_o = ws.o;
-  p.ws_len = ws.len;
-  p.step_ml = a.step ? ws.step_ml : nullptr;
+  p.ws_len = a.step ? ws.len : nullptr;
+  p.whole_ml = (a.step || a.lse) ? ws.step_ml : nullptr;
   p.err = a.err;
   p.rope = a.rope;
   if (a.variant == kDecodeUmma) {
@@ -947,6 +960,8 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   mp.ws_ml = ws.ml;
   mp.ws_o = ws.o;
   mp.out = a.out;
+  mp.lse = a.lse;
+  mp.whole_ml = ws.step_ml;
   if (a.step) {
     TcStepParams& st = mp.st;
     st.pos = a.q_pos;
@@ -964,7 +979,6 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
     st.capacity = cv.capacity;
     st.advance = a.step->advance;
     st.ws_len = ws.len;
-    st.step_ml = ws.step_ml;
     st.c_ak = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.a_k));
     st.c_bk = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.b_k));
     st.c_av = static_cast<__nv_bfloat16*>(const_cast<void*>(cv.a_v));

@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = first; b < B; b += step) p.ws_len[b] = p.seq_lens[b] == s_len[b] ? s_len[b] : -1;
   };
   if (t_begin >= t_end) {  // uniform: no tiles for this CTA
-    if (warp == 1 && blockIdx.x == 0 && p.step_ml) record_lengths(lane, 32);
+    if (warp == 1 && blockIdx.x == 0 && p.ws_len) record_lengths(lane, 32);
     if (warp == 1) ptx::tmem_dealloc(tbase, kTmemCols);
     return;
   }
@@ -371,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every MMA issued by this thread completes before TMEM can be released
       ptx::umma_commit(fin);
       ptx::mbar_wait_bounded(fin, 0);
-    } else if (blockIdx.x == 0 && p.step_ml) {
+    } else if (blockIdx.x == 0 && p.ws_len) {
       record_lengths(lane - 1, 31);  // the other lanes of the MMA warp are idle
     }
   } else {
@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float o = __uint_as_float(o0[h]) + __uint_as_float(o1[h]);
           op[h * kD] = l[h] > 0.f ? o / l[h] : 0.f;
         }
-        if (p.step_ml && quad == 0 && lane < kHalf) {  // the step's own token joins in the merge kernel
+        if (p.whole_ml && quad == 0 && lane < kHalf) {  // for the merge kernel: a step's token, or the lse
           float mk = m[0], lk = l[0];
 #pragma unroll
           for (int h = 1; h < kHalf; ++h) {
@@ -670,8 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             lk = lane == h ? l[h] : lk;
           }
           const size_t e = (static_cast<size_t>(b) * kH + kHalf * hh + lane) * 2;
-          p.step_ml[e] = mk;
-          p.step_ml[e + 1] = lk;
+          p.whole_ml[e] = mk;
+          p.whole_ml[e + 1] = lk;
         }
       } else {
         const int slot = 2 * c + (b == b_first ? 0 : 1);  // a shared sequence is the first or the last one

@@ -273,7 +273,8 @@ namespace {
 // `step`, the query's own token is appended and attended in the same launches.
 tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, int32_t r_q, const int32_t* q_pos,
                        float scale, float* out, int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
-                       size_t workspace_bytes, void* stream, const DecodeStepArgs* step = nullptr) {
+                       size_t workspace_bytes, void* stream, const DecodeStepArgs* step = nullptr,
+                       float* lse = nullptr) {
   tpa_status s = check_cache(cache);
   if (s != TPA_OK) return s;
   if (!q || !q_pos || !out) return fail(TPA_ERR_NULL, "q, q_pos or out is NULL");
@@ -300,6 +301,15 @@ tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, i
                   "a factorized decode query needs the tcgen05 kernel: bf16, heads 32, head_dim 128, "
                   "r_k == r_v <= 2, batch <= 1024, kernel AUTO or TENSOR");
     if (reinterpret_cast<uintptr_t>(a_q) & 1u) return fail(TPA_ERR_ALIGNMENT, "a_q must be 2-byte aligned");
+  }
+  if (lse) {
+    if (kernel == TPA_KERNEL_SIMT || kernel == TPA_KERNEL_TENSOR_SYNC ||
+        !tensor_decode_supported(cache->dtype, cache->heads, cache->head_dim, cache->r_k, cache->r_v) ||
+        !tensor_decode_batch_ok(cache->batch))
+      return fail(TPA_ERR_UNSUPPORTED,
+                  "the log-sum-exp output needs the tcgen05 kernel: bf16, heads 32, head_dim 128, "
+                  "r_k == r_v <= 2, batch <= 1024, kernel AUTO or TENSOR");
+    if (reinterpret_cast<uintptr_t>(lse) & 3u) return fail(TPA_ERR_ALIGNMENT, "lse must be 4-byte aligned");
   }
   if (step) {
     if (!step->a_k || !step->b_k || !step->a_v || !step->b_v)
@@ -346,6 +356,7 @@ tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, i
     a.err = err;
     a.variant = variant;
     a.step = step;
+    a.lse = lse;
     e = launch_tensor_decode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
     return TPA_OK;
@@ -407,6 +418,30 @@ tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, co
   if (r_q < 1) return fail(TPA_ERR_SHAPE, "r_q = %d < 1", r_q);
   return decode_impl(cache, b_q, a_q, r_q, q_pos, scale, out, max_len, num_splits, kernel, workspace,
                      workspace_bytes, stream);
+}
+
+tpa_status tpa_decode_attention_lse(const tpa_cache* cache, const void* q, const int32_t* q_pos, float scale,
+                                    float* out, float* lse, int32_t max_len, int32_t num_splits, int32_t kernel,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lse) return fail(TPA_ERR_NULL, "lse is NULL");
+  return decode_impl(cache, q, nullptr, 0, q_pos, scale, out, max_len, num_splits, kernel, workspace,
+                     workspace_bytes, stream, nullptr, lse);
+}
+
+tpa_status tpa_merge_lse(int32_t n_parts, int32_t rows, int32_t head_dim, const float* parts_out,
+                         const float* parts_lse, float* out, float* lse_out, void* stream) {
+  if (n_parts < 1 || rows < 0) return fail(TPA_ERR_SHAPE, "n_parts = %d (>= 1), rows = %d (>= 0)", n_parts, rows);
+  if (head_dim < 4 || head_dim > 128 || head_dim % 4 != 0)
+    return fail(TPA_ERR_UNSUPPORTED, "head_dim %d: a multiple of 4 in [4, 128]", head_dim);
+  if (rows == 0) return TPA_OK;
+  if (!parts_out || !parts_lse || !out) return fail(TPA_ERR_NULL, "parts_out, parts_lse or out is NULL");
+  if (!aligned16(parts_out) || !aligned16(out) || (reinterpret_cast<uintptr_t>(parts_lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_out) & 3u))
+    return fail(TPA_ERR_ALIGNMENT, "parts_out and out must be 16-byte aligned, the lse arrays 4-byte aligned");
+  const cudaError_t e = launch_merge_lse(n_parts, rows, head_dim, parts_out, parts_lse, out, lse_out,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  return TPA_OK;
 }
 
 tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, const void* a_k, const void* b_k,

@@ -87,6 +87,12 @@ struct MergeArgs {
 };
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t stream);
 
+// Attention over disjoint token sets from each set's (o, lse) (lse_merge.cu): parts_out
+// [n_parts][rows][head_dim], parts_lse [n_parts][rows] -> out [rows][head_dim], lse_out [rows]
+// (may be null); head_dim a multiple of 4, at most 128.
+cudaError_t launch_merge_lse(int n_parts, int rows, int head_dim, const float* parts_out, const float* parts_lse,
+                             float* out, float* lse_out, cudaStream_t stream);
+
 // Dense rotated queries for the CUDA-core prefill: Q[b][t][i][:] (fp32).
 struct PrefillQArgs {
   int batch, n_tokens, heads, head_dim, r_q, dtype;

@@ -45,6 +45,7 @@ struct TensorDecodeArgs {
   unsigned int* err;
   int variant;  // kDecodeUmma or kDecodeSync
   const DecodeStepArgs* step;  // null for a plain decode
+  float* lse;                  // [B][h] natural-log log-sum-exp of the scaled scores, or null
 };
 cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream);
 

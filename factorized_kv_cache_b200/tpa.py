@@ -83,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_decode_attention_noalloc": (ctypes.c_int, [C, P, P, ctypes.c_float, P, I32, I32, I32, P]),
         "tpa_decode_attention_factored": (ctypes.c_int, [C, I32, P, P, P, ctypes.c_float, P, I32, I32, I32, P,
                                                           ctypes.c_size_t, P]),
+        "tpa_decode_attention_lse": (ctypes.c_int, [C, P, P, ctypes.c_float, P, P, I32, I32, I32, P, ctypes.c_size_t,
+                                                     P]),
+        "tpa_merge_lse": (ctypes.c_int, [I32, I32, I32, P, P, P, P, P]),
         "tpa_decode_step": (ctypes.c_int, [C, P, P, P, P, P, I32, P, P, ctypes.c_float, P, I32, I32, I32, I32, P,
                                             ctypes.c_size_t, P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
@@ -376,6 +379,58 @@ def tpa_decode_step(cache: TpaCache, positions, a_k, b_k, a_v, b_v, q=None, a_q=
                                _ptr(qa), _ptr(qb), float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits,
                                kernel, _ptr(workspace_buf), nbytes, _stream(stream, dev)))
     return out
+
+
+def tpa_decode_attention_lse(cache: TpaCache, q, q_pos, scale: float | None = None, out=None, lse=None,
+                             max_len: int | None = None, num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO,
+                             workspace_buf=None, stream=None):
+    """Decode attention plus each head's log-sum-exp of the scaled scores; returns (out [B, h, d_h],
+    lse [B, h]) float32."""
+    lib = load_library()
+    B, h, d = cache.batch, cache.heads, cache.head_dim
+    dev = cache.a_k.device
+    _need(q, "q", cache.dtype, (B, h, d), dev)
+    _need(q_pos, "q_pos", torch.int32, (B,), dev)
+    if out is None:
+        out = torch.empty(B, h, d, dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty(B, h, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, (B, h, d), dev)
+    _need(lse, "lse", torch.float32, (B, h), dev)
+    if max_len is None:
+        max_len = cache.capacity
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    s = cache.struct()
+    if workspace_buf is None:
+        workspace_buf = workspace(int(lib.tpa_decode_workspace_size(ctypes.byref(s), max_len, num_splits, kernel)),
+                                  dev)
+    nbytes = 0 if workspace_buf is None else workspace_buf.numel() * workspace_buf.element_size()
+    _check(lib.tpa_decode_attention_lse(ctypes.byref(s), _ptr(q), _ptr(q_pos), float(scale), _ptr(out), _ptr(lse),
+                                        max_len, num_splits, kernel, _ptr(workspace_buf), nbytes,
+                                        _stream(stream, dev)))
+    return out, lse
+
+
+def tpa_merge_lse(parts_out, parts_lse, out=None, lse_out=None, stream=None):
+    """Attention over disjoint token sets from each set's (out, lse): parts_out [n, ..., d_h],
+    parts_lse [n, ...] float32 -> (out [..., d_h], lse [...])."""
+    lib = load_library()
+    n, d = parts_out.shape[0], parts_out.shape[-1]
+    lead = tuple(parts_out.shape[1:-1])
+    dev = parts_out.device
+    _need(parts_out, "parts_out", torch.float32, None, dev)
+    _need(parts_lse, "parts_lse", torch.float32, (n,) + lead, dev)
+    if out is None:
+        out = torch.empty(lead + (d,), dtype=torch.float32, device=dev)
+    if lse_out is None:
+        lse_out = torch.empty(lead, dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, lead + (d,), dev)
+    _need(lse_out, "lse_out", torch.float32, lead, dev)
+    rows = math.prod(lead)
+    _check(lib.tpa_merge_lse(n, rows, d, _ptr(parts_out), _ptr(parts_lse), _ptr(out), _ptr(lse_out),
+                             _stream(stream, dev)))
+    return out, lse_out
 
 
 class DecodeStepPlan:

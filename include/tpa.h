@@ -198,6 +198,36 @@ tpa_status tpa_decode_attention_factored(const tpa_cache* cache, int32_t r_q, co
                                          void* stream);
 
 /*
+ * tpa_decode_attention that also returns, per (sequence, head), the natural
+ * log of the sum of exp(scaled score) over the attended tokens:
+ *   lse [batch][heads] float32, device, 4-byte aligned;
+ *   lse[b][i] = log sum_s exp(scale * q~_i . K_s[i]); -inf for an empty sequence.
+ * (out, lse) of disjoint token ranges of one sequence combine exactly with
+ * tpa_merge_lse, so a long sequence can be split across devices by token
+ * range (each device holds its range with the tokens' global positions).
+ * Runs on the tcgen05 kernel only (same shapes as tpa_decode_attention_factored).
+ * Errors: those of tpa_decode_attention, NULL (lse), UNSUPPORTED, ALIGNMENT.
+ */
+tpa_status tpa_decode_attention_lse(const tpa_cache* cache, const void* q, const int32_t* q_pos, float scale,
+                                    float* out, float* lse, int32_t max_len, int32_t num_splits, int32_t kernel,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Attention over the union of n_parts disjoint token sets, from each set's
+ * result (section FlashTPA: softmax over all cached tokens):
+ *   parts_out [n_parts][rows][head_dim] float32, parts_lse [n_parts][rows] float32
+ *   (device; the layout an all-gather of per-device (out, lse) produces);
+ *   out [rows][head_dim] float32 = sum_r exp(lse_r - lse) parts_out[r],
+ *   lse_out [rows] (device, may be NULL) = log sum_r exp(lse_r).
+ * A part with lse_r = -inf (no tokens) drops out; a row without any token gets
+ * out = 0, lse = -inf.  rows = batch * heads; head_dim a multiple of 4 in
+ * [4, 128]; parts_out and out 16-byte aligned.  rows == 0 is a no-op.
+ * Errors: SHAPE (n_parts < 1, rows < 0), UNSUPPORTED (head_dim), NULL, ALIGNMENT, CUDA.
+ */
+tpa_status tpa_merge_lse(int32_t n_parts, int32_t rows, int32_t head_dim, const float* parts_out,
+                         const float* parts_lse, float* out, float* lse_out, void* stream);
+
+/*
  * One generation step of token x_t, fused: its factors are appended and its
  * query attends the cache including x_t itself (section 解决思路: Q_t, K_t, V_t
  * all come from x_t; Theorem 3.1: B_K and the query rotate at x_t's position).

@@ -57,6 +57,8 @@ __all__ = [
     "decode_attention_factored_query",
     "decode_attention_from_unrotated",
     "decode_step",
+    "decode_attention_lse",
+    "merge_lse",
     "prefill_queries",
     "prefill_attention",
     "softmax_attention",
@@ -185,14 +187,19 @@ def decode_attention_factored_query(a_k, b_k_rot, a_v, b_v, a_q, b_q, q_pos, sca
 
 def _attend_rotated_query(a_k, b_k_rot, a_v, b_v, q_rot, scale, block):
     """Softmax attention of rotated per-head queries q_rot [h, d_h] over the
-    cached tokens (see decode_attention).  K and V are expanded ``block``
-    tokens at a time only to bound memory: every score is computed on its own,
-    the softmax is taken over the full score row, and the output sum is split
-    into consecutive partial sums."""
+    cached tokens (see decode_attention)."""
+    return _attend_rotated_query_lse(a_k, b_k_rot, a_v, b_v, q_rot, scale, block)[0]
+
+
+def _attend_rotated_query_lse(a_k, b_k_rot, a_v, b_v, q_rot, scale, block):
+    """(o [h, d_h], lse [h]): the attention of _attend_rotated_query and the natural log of
+    each head's sum of exp(score).  K and V are expanded ``block`` tokens at a time only to
+    bound memory: every score is computed on its own, the softmax is taken over the full
+    score row, and the output sum is split into consecutive partial sums."""
     L = np.asarray(a_k).shape[0]
     h, d_h = np.asarray(q_rot).shape
     if L == 0:
-        return np.zeros((h, d_h))
+        return np.zeros((h, d_h)), np.full(h, -np.inf)
     z = np.empty((h, L))
     for s0 in range(0, L, block):
         s1 = min(L, s0 + block)
@@ -200,13 +207,38 @@ def _attend_rotated_query(a_k, b_k_rot, a_v, b_v, q_rot, scale, block):
         z[:, s0:s1] = scale * np.einsum("ik,sik->is", q_rot, k)
     m = z.max(axis=1, keepdims=True)
     p = np.exp(z - m)
-    p /= p.sum(axis=1, keepdims=True)
+    total = p.sum(axis=1, keepdims=True)
+    p /= total
     o = np.zeros((h, d_h))
     for s0 in range(0, L, block):
         s1 = min(L, s0 + block)
         v = tensor_product(a_v[s0:s1], b_v[s0:s1])                # [n, h, d_h]
         o += np.einsum("is,sik->ik", p[:, s0:s1], v)
-    return o
+    return o, (m + np.log(total))[:, 0]
+
+
+def decode_attention_lse(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block: int = 8192):
+    """decode_attention plus lse [h] = log sum_s exp(scale q~_i . K_s[i]) (natural log; -inf
+    with nothing cached, where o = 0).  (o, lse) is the state a shard of the token range hands
+    to merge_lse when one sequence is split across devices (the split-KV reduction)."""
+    return _attend_rotated_query_lse(a_k, b_k_rot, a_v, b_v, rope(q, q_pos, base), scale, block)
+
+
+def merge_lse(outs, lses):
+    """Attention over the union of disjoint token sets from each set's (o_r, lse_r):
+    lse = log sum_r exp(lse_r), o = sum_r exp(lse_r - lse) o_r; parts with lse_r = -inf (no
+    tokens) drop out, and with no tokens at all o = 0, lse = -inf.  outs [n, h, d_h],
+    lses [n, h] -> (o [h, d_h], lse [h])."""
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    top = lses.max(axis=0)                                            # [h]
+    safe = np.where(np.isfinite(top), top, 0.0)
+    w = np.where(np.isfinite(lses), np.exp(lses - safe[None]), 0.0)   # [n, h]
+    tot = w.sum(axis=0)
+    o = np.einsum("rh,rhk->hk", w, outs)
+    o = np.divide(o, tot[:, None], out=np.zeros_like(o), where=tot[:, None] > 0)
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return o, lse
 
 
 def decode_attention_from_unrotated(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, storage=None):

@@ -507,6 +507,51 @@ def pin_step_shift_invariance(O):
     assert np.allclose(of, ref_f, rtol=1e-9, atol=1e-12)
 
 
+# --------------------------------------------------------------------------- token-sharded decode (lse merge)
+def pin_lse_brute_force(O):
+    """The log-sum-exp of each head's scaled scores by scalar loops (math.exp, math.fsum,
+    math.log), and -inf with nothing cached."""
+    c = _rand_case(51, 4, 2, 4, 2, 1)
+    kpos = [1.0, 4.0, 6.0, 9.0]
+    qpos, scale, base = 12.0, 0.8, 100.0
+    rot = O.append_rope(c["b_k"], np.array(kpos), base)
+    o, lse = O.decode_attention_lse(c["a_k"], rot, c["a_v"], c["b_v"], c["q"], qpos, scale, base)
+    for i in range(2):
+        qr = _brute_rot(list(c["q"][i]), qpos, base)
+        z = []
+        for s in range(4):
+            key = [math.fsum(c["a_k"][s, r, i] * _brute_rot(list(c["b_k"][s, r]), kpos[s], base)[k] for r in range(2)) / 2
+                   for k in range(4)]
+            z.append(scale * math.fsum(qr[k] * key[k] for k in range(4)))
+        want = math.log(math.fsum(math.exp(v) for v in z))
+        assert abs(lse[i] - want) <= 1e-13 * (1 + abs(want)), (i, lse[i], want)
+    o0, l0 = O.decode_attention_lse(c["a_k"][:0], rot[:0], c["a_v"][:0], c["b_v"][:0], c["q"], qpos, scale, base)
+    assert (o0 == 0).all() and np.isneginf(l0).all()
+
+
+def pin_merge_lse_union(O):
+    """Softmax over a disjoint union: decoding the token range in shards (global positions,
+    an empty shard among them) and merging (o, lse) gives the decode of the whole range,
+    and the lse of the whole."""
+    c = _rand_case(53, 61, 4, 16, 2, 2)
+    pos = np.arange(61, dtype=np.float64) * 2 + 3
+    rot = O.append_rope(c["b_k"], pos, 10000.0)
+    args = (200.0, 0.4, 10000.0)
+    whole, whole_lse = O.decode_attention_lse(c["a_k"], rot, c["a_v"], c["b_v"], c["q"], *args)
+    cuts = [0, 17, 17, 40, 61]
+    parts = [O.decode_attention_lse(c["a_k"][a:e], rot[a:e], c["a_v"][a:e], c["b_v"][a:e], c["q"], *args)
+             for a, e in zip(cuts[:-1], cuts[1:])]
+    o, lse = O.merge_lse([p[0] for p in parts], [p[1] for p in parts])
+    assert np.allclose(o, whole, rtol=1e-12, atol=1e-14)
+    assert np.allclose(lse, whole_lse, rtol=1e-13, atol=1e-13)
+    assert np.allclose(o, O.decode_attention(c["a_k"], rot, c["a_v"], c["b_v"], c["q"], *args), rtol=1e-12,
+                       atol=1e-14)
+    o1, l1 = O.merge_lse([whole], [whole_lse])                      # one part: itself
+    assert np.allclose(o1, whole, rtol=1e-15, atol=0) and np.allclose(l1, whole_lse, rtol=1e-15, atol=0)
+    oe, le = O.merge_lse([np.zeros_like(whole)] * 2, [np.full(4, -np.inf)] * 2)   # no tokens anywhere
+    assert (oe == 0).all() and np.isneginf(le).all()
+
+
 ALL_PINS = [
     pin_storage_rounding,
     pin_cache_size,
@@ -531,4 +576,6 @@ ALL_PINS = [
     pin_step_empty_cache,
     pin_step_brute_force,
     pin_step_shift_invariance,
+    pin_lse_brute_force,
+    pin_merge_lse_union,
 ]

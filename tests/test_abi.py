@@ -124,6 +124,28 @@ def test_decode_step_rejects_bad_arguments():
     assert lib.tpa_last_error_message().decode() != ""
 
 
+def test_lse_decode_and_merge_reject_bad_arguments():
+    lib = T.load_library()
+    P = 0x90000
+    c = _fake_cache()
+    lse = lambda cc=c, lse_p=P, kernel=0: lib.tpa_decode_attention_lse(ctypes.byref(cc), 0x60000, 0x70000, 0.1,
+                                                                        0x80000, lse_p, 64, 0, kernel, None, 0, None)
+    assert lse(lse_p=None) == 1
+    assert lse(lse_p=P + 2) == 6
+    assert lse(kernel=T.TPA_KERNEL_SIMT) == 3
+    assert lse(cc=_fake_cache(dtype=T.TPA_F32)) == 3
+    merge = lambda n=2, rows=8, d=128, po=P, pl=P, o=0xA0000, lo=None: lib.tpa_merge_lse(n, rows, d, po, pl, o, lo, None)
+    assert merge(n=0) == 2
+    assert merge(rows=-1) == 2
+    assert merge(d=130) == 3
+    assert merge(d=2) == 3
+    assert merge(rows=0, po=None, pl=None, o=None) == 0      # nothing to merge
+    assert merge(po=None) == 1
+    assert merge(o=None) == 1
+    assert merge(po=P + 8) == 6
+    assert merge(lo=P + 2) == 6
+
+
 def test_append_rejects_bad_arguments():
     lib = T.load_library()
     c = _fake_cache()

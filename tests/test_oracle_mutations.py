@@ -106,6 +106,27 @@ def _step_without_new_token(a_k, b_k_rot, a_v, b_v, new_a_k, new_b_k, new_a_v, n
     return O.decode_attention_factored_query(a_k, b_k_rot, a_v, b_v, a_q, b_q, pos, scale, base), row
 
 
+_merge = O.merge_lse
+_lse = O.decode_attention_lse
+
+
+def _merge_unnormalised(outs, lses):        # weights exp(lse_r - max) not divided by their sum
+    o, lse = _merge(outs, lses)
+    lses = np.asarray(lses, dtype=np.float64)
+    top = lses.max(axis=0)
+    w = np.where(np.isfinite(lses), np.exp(lses - np.where(np.isfinite(top), top, 0.0)[None]), 0.0)
+    return o * w.sum(axis=0)[:, None], lse
+
+
+def _merge_plain_mean(outs, lses):          # parts averaged, lse ignored
+    return np.asarray(outs, dtype=np.float64).mean(axis=0), _merge(outs, lses)[1]
+
+
+def _lse_log2(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block=8192):   # base-2 log-sum-exp
+    o, lse = _lse(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block)
+    return o, lse / np.log(2.0)
+
+
 def _round_truncate(x, storage):               # truncation instead of round-to-nearest-even
     if storage != "bf16":
         return _round(x, storage)
@@ -140,6 +161,9 @@ MUTANTS = {
     "step_new_key_unrotated": ("decode_step", _step_new_key_unrotated),
     "step_new_key_next_position": ("decode_step", _step_new_key_next_position),
     "step_without_new_token": ("decode_step", _step_without_new_token),
+    "merge_unnormalised": ("merge_lse", _merge_unnormalised),
+    "merge_plain_mean": ("merge_lse", _merge_plain_mean),
+    "lse_log2": ("decode_attention_lse", _lse_log2),
 }
 
 
