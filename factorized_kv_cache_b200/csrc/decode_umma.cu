@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tmap(&tm_av);
   }
   ptx::tc_fence_before();
+  __syncwarp();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tbase = *s_taddr;
@@ -693,6 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::tc_fence_before();
   }
+  // The TMA and MMA warps ran their loops on lane 0 alone: reconverge them first, so that the
+  // CTA barrier counts every thread and TMEM is released only after every role is done.
+  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     ptx::tc_fence_after();
