@@ -236,3 +236,21 @@ def test_factored_query_rank_one_matches_dense_decode():
     o_d = T.tpa_decode_attention(cache, b_q.expand(3, w.heads, w.head_dim).contiguous(), q_pos, max_len=2000,
                                  kernel=T.TPA_KERNEL_TENSOR)
     assert torch.equal(o_f, o_d)
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_maximum_batch(kernel):
+    """The largest batch the tensor-core decodes take (1024 sequences), short ragged lengths with
+    empty ones among them, so that CTAs span many sequences; the oracle on a sample of them."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="max_batch", seed=131)
+    g = np.random.default_rng(131)
+    lengths = g.integers(0, 300, size=1024)
+    lengths[::97] = 0
+    lengths[5] = 300
+    cache, x, q, q_pos = build_decode_cache(w, batch=1024, length=300, lengths=lengths.tolist(), nan_tail=False)
+    out = T.tpa_decode_attention(cache, q, q_pos, max_len=300, kernel=kernel)
+    assert T.tpa_read_device_error() == 0
+    sample = sorted(set(g.choice(1024, 48, replace=False).tolist()) | {0, 5, 97, 1023})
+    _check(w, cache, x, q, q_pos, out, batches=sample, end_to_end=False)
+    for b in np.nonzero(lengths == 0)[0]:
+        assert torch.count_nonzero(out[b]) == 0

@@ -235,3 +235,36 @@ def test_plan_matches_the_call():
     for name in ("a_k", "b_k", "a_v", "b_v"):
         for b, L in enumerate(lengths):
             assert torch.equal(getattr(cache, name)[b, :L + 3], getattr(twin, name)[b, :L + 3])
+
+
+def test_step_and_lse_at_maximum_batch():
+    """1024 sequences (empty ones among them): the fused step against the oracle on a sample,
+    and the lse decode of the stepped cache against the oracle's lse."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="step_max_batch", seed=132)
+    g = np.random.default_rng(132)
+    lengths = g.integers(0, 200, size=1024)
+    lengths[::101] = 0
+    cache, x, _, _ = build_decode_cache(w, batch=1024, length=201, lengths=lengths.tolist(), nan_tail=False)
+    before = [t.clone() for t in (cache.a_k, cache.b_k, cache.a_v, cache.b_v, cache.seq_lens)]
+    tok = _token(w, 1024, 133)
+    pos = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    out = _step(cache, tok, pos, max_len=201)
+    assert T.tpa_read_device_error() == 0
+    assert torch.equal(cache.seq_lens.cpu(), torch.tensor(lengths, dtype=torch.int32) + 1)
+    sample = sorted(set(g.choice(1024, 32, replace=False).tolist()) | {0, 101, 1023})
+    cpu = readback(T.TpaCache(*before, rope_base=cache.rope_base), sample)
+    for n, b in enumerate(sample):
+        L = int(lengths[b])
+        ref, _ = O.decode_step(cpu["a_k"][n, :L], cpu["b_k"][n, :L], cpu["a_v"][n, :L], cpu["b_v"][n, :L],
+                               f64(tok["a_k"][b]), f64(tok["b_k"][b]), f64(tok["a_v"][b]), f64(tok["b_v"][b]),
+                               float(pos[b]), default_scale(w.head_dim), w.rope_base, q=f64(tok["q"][b]),
+                               storage="bf16")
+        assert_rows_close(f64(out[b]), ref, BF16, f"max-batch step b={b}")
+    o2, lse = T.tpa_decode_attention_lse(cache, tok["q"], pos, max_len=201)
+    cpu2 = readback(cache, sample)
+    for n, b in enumerate(sample):
+        L = int(lengths[b]) + 1
+        o, l = O.decode_attention_lse(cpu2["a_k"][n, :L], cpu2["b_k"][n, :L], cpu2["a_v"][n, :L], cpu2["b_v"][n, :L],
+                                      f64(tok["q"][b]), float(pos[b]), default_scale(w.head_dim), w.rope_base)
+        assert np.abs(f64(lse[b]) - l).max() <= BF16, b
+        assert_rows_close(f64(o2[b]), o, BF16, f"max-batch lse decode b={b}")
