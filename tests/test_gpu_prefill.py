@@ -103,3 +103,18 @@ def test_prefill_workload_full_size(kernel):
         heads = [0, 9, 31]
         ref = _oracle(w, cache, x, 0, w.tokens, b, rows=rows, heads=heads)
         assert_rows_close(got[b][rows][:, heads], ref, TOL[cache.dtype], f"prefill full b={b}")
+
+
+@pytest.mark.parametrize("tokens,prior", [(200, 0), (130, 37), (1000, 3000)])
+def test_last_prefill_row_equals_factored_decode(tokens, prior):
+    """Two kernels, one quantity: the prefill's last query row (slot L - 1, attending slots
+    0 .. L - 1) is the decode of a query in TPA form (A_Q, B_Q of that token, at position L - 1)
+    over the same cache."""
+    w = S.WORKLOADS["prefill_b4_t4k"]
+    cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, tokens, prior)
+    out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos)
+    L = prior + tokens
+    dec = T.tpa_decode_attention_factored(cache, a_q[:, -1].contiguous(), b_q[:, -1].contiguous(),
+                                          q_pos[:, -1].contiguous(), max_len=L)
+    assert T.tpa_read_device_error() == 0
+    assert_rows_close(f64(dec), f64(out[:, -1]), 2e-4, "prefill last row vs factored decode")
