@@ -484,6 +484,29 @@ class DecodeStepPlan:
         _check(self._fn(*self._args, _stream(stream, self._device)))
         return self.out
 
+    def graph(self, host_in=None, dev_in=None, host_out=None, stream=None):
+        """One whole step as a CUDA graph: the copy of ``host_in`` (pinned host memory) into
+        ``dev_in`` (the device memory the bound inputs live in), the step, and the copy of the
+        output into ``host_out`` (pinned).  Each ``replay()`` runs all three with the buffers'
+        current contents, for one graph launch per step; like any CUDA graph it replays on the
+        current stream."""
+        stream = torch.cuda.Stream(device=self._device) if stream is None else stream
+        g = torch.cuda.CUDAGraph()
+
+        def body():
+            if host_in is not None:
+                dev_in.copy_(host_in, non_blocking=True)
+            self(stream)
+            if host_out is not None:
+                host_out.copy_(self.out, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            body()               # a first run outside the capture (the library's one-time set-up)
+        stream.synchronize()
+        with torch.cuda.graph(g, stream=stream):
+            body()
+        return g
+
 
 def tpa_decode_attention_noalloc(cache: TpaCache, q, q_pos, out, scale: float | None = None,
                                  max_len: int | None = None, num_splits: int = 0, kernel: int = TPA_KERNEL_AUTO,

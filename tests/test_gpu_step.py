@@ -268,3 +268,46 @@ def test_step_and_lse_at_maximum_batch():
                                       f64(tok["q"][b]), float(pos[b]), default_scale(w.head_dim), w.rope_base)
         assert np.abs(f64(lse[b]) - l).max() <= BF16, b
         assert_rows_close(f64(o2[b]), o, BF16, f"max-batch lse decode b={b}")
+
+
+def test_plan_graph_copies_in_steps_and_copies_out():
+    """DecodeStepPlan.graph(): each replay copies the host inputs in, steps (advancing the
+    lengths) and copies the output back; the same as the plain calls on a twin cache."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="step_graph", seed=79)
+    lengths = [500, 0, 1200]
+    cache, x, _, _ = build_decode_cache(w, batch=3, length=1300, lengths=lengths)
+    twin = T.TpaCache(*(t.clone() for t in (cache.a_k, cache.b_k, cache.a_v, cache.b_v, cache.seq_lens)),
+                      rope_base=cache.rope_base)
+    names = ("a_k", "b_k", "a_v", "b_v", "q")
+    toks = [_token(w, 3, 150 + k) for k in range(3)]
+    sizes = [toks[0][k].numel() for k in names] + [3]
+    host_in = torch.empty(sum(sizes) * 4, dtype=torch.uint8).pin_memory()
+    dev_in = torch.empty_like(host_in, device=DEV)
+    views, off = {}, 0
+    for k in names:
+        nb = toks[0][k].numel() * 2
+        views[k] = dev_in[off:off + nb].view(torch.bfloat16).view(toks[0][k].shape)
+        off += (nb + 255) // 256 * 256
+    views["pos"] = dev_in[off:off + 12].view(torch.int32)
+    out = torch.empty(3, w.heads, w.head_dim, dtype=torch.float32, device=DEV)
+    host_out = torch.empty(3, w.heads, w.head_dim, dtype=torch.float32).pin_memory()
+    plan = T.DecodeStepPlan(cache, views["pos"], views["a_k"], views["b_k"], views["a_v"], views["b_v"], out,
+                            q=views["q"], max_len=1300)
+    staging = torch.empty_like(dev_in)
+    g = None
+    for k, tok in enumerate(toks):
+        pos = twin.seq_lens.clone()
+        for name in names:                      # the step's inputs, laid out in the staging buffer
+            staging_view = staging[views[name].data_ptr() - dev_in.data_ptr():][:tok[name].numel() * 2]
+            staging_view.copy_(tok[name].view(-1).view(torch.uint8))
+        staging[views["pos"].data_ptr() - dev_in.data_ptr():][:12].copy_(pos.view(torch.uint8))
+        host_in.copy_(staging.cpu())
+        if g is None:
+            g = plan.graph(host_in, dev_in, host_out)   # the capture's first run is step 0
+        else:
+            g.replay()
+        torch.cuda.synchronize()
+        ref = _step(twin, tok, pos, max_len=1300)
+        assert torch.equal(host_out, ref.cpu()), k
+    assert T.tpa_read_device_error() == 0
+    assert torch.equal(cache.seq_lens, twin.seq_lens)
