@@ -123,3 +123,28 @@ def test_merge_lse_long_workload_in_shards():
                              cpu["b_v"][0, :L], f64(q[0])[heads], float(q_pos[0]), default_scale(w.head_dim),
                              w.rope_base)
     assert_rows_close(f64(merged[0])[heads], ref, BF16, "long workload vs oracle")
+
+
+def test_decode_token_sharded_through_a_process_group():
+    """sharded.decode_token_sharded end to end through torch.distributed (a one-rank NCCL
+    group: the all-gather runs, the merge combines one part) equals the plain decode."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device(DEV, 0))
+    try:
+        w = S.WORKLOADS["decode_b8_l8k"].replace(name="sharded_pg", seed=97)
+        cache, x, q, q_pos = build_decode_cache(w, batch=3, length=3000, lengths=[3000, 0, 1700])
+        out, lse = sharded.decode_token_sharded(cache, q, q_pos, max_len=3000)
+        ref, ref_lse = T.tpa_decode_attention_lse(cache, q, q_pos, max_len=3000)
+        assert T.tpa_read_device_error() == 0
+        assert torch.equal(out, ref)
+        assert torch.equal(lse, ref_lse)
+    finally:
+        dist.destroy_process_group()
