@@ -489,7 +489,7 @@ class DecodeStepPlan:
         ``dev_in`` (the device memory the bound inputs live in), the step, and the copy of the
         output into ``host_out`` (pinned).  Each ``replay()`` runs all three with the buffers'
         current contents, for one graph launch per step; like any CUDA graph it replays on the
-        current stream."""
+        current stream.  Building the graph runs one step first, outside the capture."""
         stream = torch.cuda.Stream(device=self._device) if stream is None else stream
         g = torch.cuda.CUDAGraph()
 
