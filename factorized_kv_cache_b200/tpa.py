@@ -437,7 +437,8 @@ class DecodeStepPlan:
     """tpa_decode_step bound to fixed buffers, for a generation loop: the arguments are checked
     and marshalled once, and each call is a single C call with the stored pointers.  The
     buffers' contents may change between calls (new factors, query, positions); the tensors
-    themselves, and the cache's planes, must stay the same objects."""
+    themselves, and the cache's planes, must stay the same objects.  ``out`` may be pinned host
+    memory: the kernels then write the output straight to the host."""
 
     def __init__(self, cache: TpaCache, positions, a_k, b_k, a_v, b_v, out, q=None, a_q=None, b_q=None,
                  scale: float | None = None, max_len: int | None = None, advance: bool = True, num_splits: int = 0,
@@ -450,7 +451,14 @@ class DecodeStepPlan:
         _need(b_k, "b_k", dt, (B, cache.r_k, d), dev)
         _need(a_v, "a_v", dt, (B, cache.r_v, h), dev)
         _need(b_v, "b_v", dt, (B, cache.r_v, d), dev)
-        _need(out, "out", torch.float32, (B, h, d), dev)
+        if out.device.type == "cpu":
+            # pinned host memory is addressable by the kernels: the step writes its output there
+            # directly, with no separate device-to-host copy
+            if not out.is_pinned():
+                raise ValueError("out on the host must be pinned memory")
+            _need(out, "out", torch.float32, (B, h, d))
+        else:
+            _need(out, "out", torch.float32, (B, h, d), dev)
         if q is not None:
             if a_q is not None or b_q is not None:
                 raise ValueError("pass either q or (a_q, b_q)")

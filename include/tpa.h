@@ -241,6 +241,8 @@ tpa_status tpa_merge_lse(int32_t n_parts, int32_t rows, int32_t head_dim, const 
  *   out [batch][heads][head_dim] float32: attention of the query over slots
  *     0 .. L of sequence b, where L = seq_lens[b] on entry and slot L now
  *     holds x_t (B_K stored rotated, exactly as tpa_cache_append stores it);
+ *     device memory, or pinned host memory the device can address (the kernels
+ *     then write the output to the host directly, with no copy to launch);
  *   advance: 1 = seq_lens[b] becomes L + 1 (generation); 0 = seq_lens is left
  *     at L, so the next call overwrites the same slot (a fixed-length cache,
  *     or a token that may be rejected);

@@ -311,3 +311,26 @@ def test_plan_graph_copies_in_steps_and_copies_out():
         assert torch.equal(host_out, ref.cpu()), k
     assert T.tpa_read_device_error() == 0
     assert torch.equal(cache.seq_lens, twin.seq_lens)
+
+
+def test_plan_writes_its_output_to_pinned_host_memory():
+    """DecodeStepPlan with a pinned host ``out``: the kernels write the output to the host
+    directly; it equals the step with a device output."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="step_host_out", seed=83)
+    lengths = [2100, 0, 64, 1]
+    cache, x, _, _ = build_decode_cache(w, batch=4, length=2200, lengths=lengths)
+    twin = T.TpaCache(*(t.clone() for t in (cache.a_k, cache.b_k, cache.a_v, cache.b_v, cache.seq_lens)),
+                      rope_base=cache.rope_base)
+    tok = _token(w, 4, 160)
+    pos = cache.seq_lens.clone()
+    host_out = torch.full((4, w.heads, w.head_dim), float("nan"), dtype=torch.float32).pin_memory()
+    plan = T.DecodeStepPlan(cache, pos, tok["a_k"], tok["b_k"], tok["a_v"], tok["b_v"], host_out, q=tok["q"],
+                            max_len=2200)
+    plan()
+    torch.cuda.synchronize()
+    ref = _step(twin, tok, pos.clone(), max_len=2200)
+    assert T.tpa_read_device_error() == 0
+    assert torch.equal(host_out, ref.cpu())
+    with pytest.raises(ValueError):
+        T.DecodeStepPlan(cache, pos, tok["a_k"], tok["b_k"], tok["a_v"], tok["b_v"],
+                         torch.empty(4, w.heads, w.head_dim), q=tok["q"])   # pageable host memory
