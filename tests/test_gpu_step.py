@@ -270,6 +270,35 @@ def test_step_and_lse_at_maximum_batch():
         assert_rows_close(f64(o2[b]), o, BF16, f"max-batch lse decode b={b}")
 
 
+@pytest.mark.parametrize("rank", [1, 2])
+def test_step_advance_over_many_merge_waves(rank):
+    """256 sequences whose lengths sit on tile edges, advanced by the step.  The merge grid runs
+    in several waves, and the head-0 CTAs of the first wave advance every length (each by a
+    whole new tile) before later waves start: every merge CTA must still use the partition and
+    the lengths the split kernel used, and merge exactly the partials it wrote."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="step_waves", r_k=rank, r_v=rank, seed=140 + rank)
+    g = np.random.default_rng(140 + rank)
+    lengths = g.choice([128, 256, 384], size=256)
+    lengths[::37] = 0
+    cache, x, _, _ = build_decode_cache(w, batch=256, length=400, lengths=lengths.tolist(), nan_tail=False)
+    before = [t.clone() for t in (cache.a_k, cache.b_k, cache.a_v, cache.b_v, cache.seq_lens)]
+    tok = _token(w, 256, 141 + rank)
+    pos = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    out = _step(cache, tok, pos, max_len=400)
+    assert T.tpa_read_device_error() == 0
+    assert torch.equal(cache.seq_lens.cpu(), torch.tensor(lengths, dtype=torch.int32) + 1)
+    _same_as_append(cache, before, tok, pos, lengths.tolist())
+    sample = sorted(set(g.choice(256, 24, replace=False).tolist()) | {0, 1, 254, 255})
+    cpu = readback(T.TpaCache(*before, rope_base=cache.rope_base), sample)
+    for n, b in enumerate(sample):
+        L = int(lengths[b])
+        ref, _ = O.decode_step(cpu["a_k"][n, :L], cpu["b_k"][n, :L], cpu["a_v"][n, :L], cpu["b_v"][n, :L],
+                               f64(tok["a_k"][b]), f64(tok["b_k"][b]), f64(tok["a_v"][b]), f64(tok["b_v"][b]),
+                               float(pos[b]), default_scale(w.head_dim), w.rope_base, q=f64(tok["q"][b]),
+                               storage="bf16")
+        assert_rows_close(f64(out[b]), ref, BF16, f"many-wave step R={rank} b={b}")
+
+
 def test_plan_graph_copies_in_steps_and_copies_out():
     """DecodeStepPlan.graph(): each replay copies the host inputs in, steps (advancing the
     lengths) and copies the output back; the same as the plain calls on a twin cache."""
