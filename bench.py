@@ -373,20 +373,22 @@ def run_ours_decode(args, w, rank, world, dev):
     e2e_steps = max(1, min(K, 2000))
 
     if fused:
-        # a generation loop binds its buffers once (T.DecodeStepPlan) and calls it every step; the
-        # output goes to pinned host memory, which the kernels write directly (the device-to-host
+        # a generation loop binds its buffers once (T.DecodeStepPlan) and calls it every step: the
+        # plan copies the packed inputs from the pinned host buffer, then runs the step, whose
+        # output goes to pinned host memory that the kernels write directly (the device-to-host
         # transfer of the result, with no copy to launch)
         v = views
         qkw = {"a_q": v["a_q"], "b_q": v["b_q"]} if rq > 0 else {"q": v["q"]}
         plans = [T.DecodeStepPlan(caches[c], v["q_pos"], v["a_k"], v["b_k"], v["a_v"], v["b_v"], host_out, **qkw,
-                                  max_len=cap, advance=False, kernel=kernel, workspace_buf=ws) for c in range(copies)]
+                                  max_len=cap, advance=False, kernel=kernel, workspace_buf=ws,
+                                  stage=(host_in, dev_in)) for c in range(copies)]
 
     def e2e_step(c):
-        with torch.cuda.stream(stream):
-            dev_in.copy_(host_in, non_blocking=True)
-            if fused:
-                plans[c](stream)
-            else:
+        if fused:
+            plans[c](stream)
+        else:
+            with torch.cuda.stream(stream):
+                dev_in.copy_(host_in, non_blocking=True)
                 step(c, views)
                 host_out.copy_(out, non_blocking=True)
         stream.synchronize()

@@ -444,6 +444,14 @@ tpa_status tpa_merge_lse(int32_t n_parts, int32_t rows, int32_t head_dim, const 
   return TPA_OK;
 }
 
+tpa_status tpa_stage_async(void* dst, const void* src, size_t bytes, void* stream) {
+  if (bytes == 0) return TPA_OK;
+  if (!dst || !src) return fail(TPA_ERR_NULL, "dst or src is NULL");
+  const cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "input copy");
+  return TPA_OK;
+}
+
 tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, const void* a_k, const void* b_k,
                            const void* a_v, const void* b_v, int32_t r_q, const void* a_q, const void* q, float scale,
                            float* out, int32_t max_len, int32_t advance, int32_t num_splits, int32_t kernel,

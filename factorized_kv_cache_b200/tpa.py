@@ -88,6 +88,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_merge_lse": (ctypes.c_int, [I32, I32, I32, P, P, P, P, P]),
         "tpa_decode_step": (ctypes.c_int, [C, P, P, P, P, P, I32, P, P, ctypes.c_float, P, I32, I32, I32, I32, P,
                                             ctypes.c_size_t, P]),
+        "tpa_stage_async": (ctypes.c_int, [P, P, ctypes.c_size_t, P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
@@ -433,16 +434,38 @@ def tpa_merge_lse(parts_out, parts_lse, out=None, lse_out=None, stream=None):
     return out, lse_out
 
 
+def tpa_stage_async(dst: torch.Tensor, src: torch.Tensor, stream=None):
+    """Copy ``src`` (pinned host memory) into ``dst`` (device memory, at least as many bytes)
+    on ``stream`` (default: the current stream of ``dst``'s device), asynchronously."""
+    nbytes = _stage_bytes(dst, src)
+    _check(load_library().tpa_stage_async(_ptr(dst), _ptr(src), nbytes, _stream(stream, dst.device)))
+
+
+def _stage_bytes(dst: torch.Tensor, src: torch.Tensor) -> int:
+    if src.device.type != "cpu" or not src.is_pinned():
+        raise ValueError("src must be pinned host memory")
+    if dst.device.type != "cuda":
+        raise ValueError("dst must be device memory")
+    if not src.is_contiguous() or not dst.is_contiguous():
+        raise ValueError("src and dst must be contiguous")
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < nbytes:
+        raise ValueError(f"dst holds fewer than the {nbytes} bytes of src")
+    return nbytes
+
+
 class DecodeStepPlan:
     """tpa_decode_step bound to fixed buffers, for a generation loop: the arguments are checked
     and marshalled once, and each call is a single C call with the stored pointers.  The
     buffers' contents may change between calls (new factors, query, positions); the tensors
     themselves, and the cache's planes, must stay the same objects.  ``out`` may be pinned host
-    memory: the kernels then write the output straight to the host."""
+    memory: the kernels then write the output straight to the host.  ``stage=(host_in,
+    dev_in)``: each call first copies ``host_in`` (pinned) into ``dev_in`` (the device memory
+    the bound inputs live in) on the same stream, for a loop whose inputs come from the host."""
 
     def __init__(self, cache: TpaCache, positions, a_k, b_k, a_v, b_v, out, q=None, a_q=None, b_q=None,
                  scale: float | None = None, max_len: int | None = None, advance: bool = True, num_splits: int = 0,
-                 kernel: int = TPA_KERNEL_AUTO, workspace_buf=None):
+                 kernel: int = TPA_KERNEL_AUTO, workspace_buf=None, stage=None):
         lib = load_library()
         B, h, d = cache.batch, cache.heads, cache.head_dim
         dev, dt = cache.a_k.device, cache.dtype
@@ -487,9 +510,20 @@ class DecodeStepPlan:
         self._args = (ctypes.byref(self._struct), _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v), _ptr(b_v), r_q,
                       _ptr(qa), _ptr(qb), float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits, kernel,
                       _ptr(workspace_buf), nbytes)
+        self._stage = None
+        if stage is not None:
+            host_in, dev_in = stage
+            if dev_in.device != dev:
+                raise ValueError(f"stage: dev_in is on {dev_in.device}, expected {dev}")
+            self._stage = (_ptr(dev_in), _ptr(host_in), _stage_bytes(dev_in, host_in))
+            self._stage_fn = lib.tpa_stage_async
+            self._keep += (host_in, dev_in)
 
     def __call__(self, stream=None):
-        _check(self._fn(*self._args, _stream(stream, self._device)))
+        s = _stream(stream, self._device)
+        if self._stage is not None:
+            _check(self._stage_fn(*self._stage, s))
+        _check(self._fn(*self._args, s))
         return self.out
 
     def graph(self, host_in=None, dev_in=None, host_out=None, stream=None):

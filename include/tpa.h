@@ -265,6 +265,21 @@ tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, con
                            int32_t kernel, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Copies a step's inputs, packed in one buffer, from host memory to device
+ * memory on `stream`: one asynchronous copy, ordered before whatever the
+ * caller launches next on that stream (tpa_decode_step).  This is a
+ * deployment convenience for bindings with no CUDA runtime of their own; the
+ * pages define no such call.
+ *   dst: device memory; src: host memory, pinned (page-locked) for the copy to
+ *   be asynchronous (pageable memory is copied through a driver staging buffer,
+ *   and the call may then return only once the copy is done); bytes == 0 is a
+ *   no-op.  The caller owns both buffers and must not change src until the
+ *   copy has run.
+ * Errors: NULL (dst or src NULL with bytes > 0), CUDA (the copy was not enqueued).
+ */
+tpa_status tpa_stage_async(void* dst, const void* src, size_t bytes, void* stream);
+
+/*
  * tpa_decode_attention for callers that cannot allocate device memory (no
  * counterpart on the page; this is a deployment convenience).  Same
  * arguments and result as tpa_decode_attention minus the workspace: the

@@ -3,6 +3,7 @@ reject bad arguments before touching the GPU (no GPU needed)."""
 import ctypes
 
 import pytest
+import torch
 
 from factorized_kv_cache_b200 import tpa as T
 
@@ -144,6 +145,15 @@ def test_lse_decode_and_merge_reject_bad_arguments():
     assert merge(o=None) == 1
     assert merge(po=P + 8) == 6
     assert merge(lo=P + 2) == 6
+
+
+def test_stage_rejects_bad_arguments():
+    lib = T.load_library()
+    assert lib.tpa_stage_async(None, None, 0, None) == 0          # nothing to copy
+    assert lib.tpa_stage_async(None, 0x90000, 16, None) == 1
+    assert lib.tpa_stage_async(0x90000, None, 16, None) == 1
+    with pytest.raises(ValueError):
+        T.tpa_stage_async(torch.empty(4), torch.empty(4))          # src is not pinned
 
 
 def test_append_rejects_bad_arguments():

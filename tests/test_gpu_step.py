@@ -363,3 +363,40 @@ def test_plan_writes_its_output_to_pinned_host_memory():
     with pytest.raises(ValueError):
         T.DecodeStepPlan(cache, pos, tok["a_k"], tok["b_k"], tok["a_v"], tok["b_v"],
                          torch.empty(4, w.heads, w.head_dim), q=tok["q"])   # pageable host memory
+
+
+def test_plan_stages_its_inputs_from_pinned_host_memory():
+    """DecodeStepPlan with ``stage=(host_in, dev_in)``: every call copies the packed inputs from
+    pinned host memory before the step, so new host contents reach the kernels; each step equals
+    the step on device inputs."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="step_staged", seed=84)
+    lengths = [900, 0, 128, 5]
+    cache, x, _, _ = build_decode_cache(w, batch=4, length=1000, lengths=lengths)
+    twin = T.TpaCache(*(t.clone() for t in (cache.a_k, cache.b_k, cache.a_v, cache.b_v, cache.seq_lens)),
+                      rope_base=cache.rope_base)
+    names = ("q_pos", "a_k", "b_k", "a_v", "b_v", "q")
+    first = dict(_token(w, 4, 170), q_pos=cache.seq_lens.clone())
+    layout, off = [], 0
+    for n in names:
+        nb = first[n].numel() * first[n].element_size()
+        layout.append((n, off, nb))
+        off += (nb + 255) // 256 * 256
+    host_in = torch.zeros(off, dtype=torch.uint8).pin_memory()
+    dev_in = torch.zeros(off, dtype=torch.uint8, device=DEV)
+    views = {n: dev_in[o:o + nb].view(first[n].dtype).view(first[n].shape) for n, o, nb in layout}
+    out = torch.empty(4, w.heads, w.head_dim, dtype=torch.float32, device=DEV)
+    plan = T.DecodeStepPlan(cache, views["q_pos"], views["a_k"], views["b_k"], views["a_v"], views["b_v"], out,
+                            q=views["q"], max_len=1000, stage=(host_in, dev_in))
+    for k in range(3):
+        tok = dict(_token(w, 4, 170 + k), q_pos=twin.seq_lens.clone())
+        for n, o, nb in layout:
+            host_in[o:o + nb].copy_(tok[n].cpu().contiguous().view(-1).view(torch.uint8))
+        got = plan().clone()
+        ref = _step(twin, tok, tok["q_pos"], max_len=1000)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), k
+        assert torch.equal(cache.seq_lens, twin.seq_lens), k
+    assert T.tpa_read_device_error() == 0
+    with pytest.raises(ValueError):
+        T.DecodeStepPlan(cache, views["q_pos"], views["a_k"], views["b_k"], views["a_v"], views["b_v"], out,
+                         q=views["q"], stage=(torch.zeros(off, dtype=torch.uint8), dev_in))   # pageable host memory
