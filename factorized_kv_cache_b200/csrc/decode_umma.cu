@@ -369,9 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!*s_abort) atomicOr(p.err, kErrTimeout);
         *s_abort = 1;
       }
-      // every MMA issued by this thread completes before TMEM can be released
+      // every MMA issued by this thread completes before TMEM can be released; TMEM is released
+      // after the time limit all the same, with the error recorded
       ptx::umma_commit(fin);
-      ptx::mbar_wait_bounded(fin, 0);
+      if (!ptx::mbar_wait_bounded(fin, 0)) atomicOr(p.err, kErrTimeout);
     } else if (blockIdx.x == 0 && p.ws_len) {
       record_lengths(lane - 1, 31);  // the other lanes of the MMA warp are idle
     }
