@@ -274,7 +274,7 @@ namespace {
 tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, int32_t r_q, const int32_t* q_pos,
                        float scale, float* out, int32_t max_len, int32_t num_splits, int32_t kernel, void* workspace,
                        size_t workspace_bytes, void* stream, const DecodeStepArgs* step = nullptr,
-                       float* lse = nullptr) {
+                       float* lse = nullptr, TensorDecodeArgs* bind = nullptr) {
   tpa_status s = check_cache(cache);
   if (s != TPA_OK) return s;
   if (!q || !q_pos || !out) return fail(TPA_ERR_NULL, "q, q_pos or out is NULL");
@@ -357,10 +357,15 @@ tpa_status decode_impl(const tpa_cache* cache, const void* q, const void* a_q, i
     a.variant = variant;
     a.step = step;
     a.lse = lse;
+    if (bind) {  // a step plan: checked and prepared, launched later
+      *bind = a;
+      return TPA_OK;
+    }
     e = launch_tensor_decode(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
     return TPA_OK;
   }
+  if (bind) return fail(TPA_ERR_UNSUPPORTED, "a step plan needs the tcgen05 kernel");
   const SplitPlan plan = plan_splits(cache, max_len, num_splits, sms);
   DecodeWs ws = carve_decode_ws(workspace, cache->batch, cache->heads, cache->head_dim, plan.splits);
   if (ws.bytes > 0) {
@@ -449,6 +454,79 @@ tpa_status tpa_stage_async(void* dst, const void* src, size_t bytes, void* strea
   if (!dst || !src) return fail(TPA_ERR_NULL, "dst or src is NULL");
   const cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "input copy");
+  return TPA_OK;
+}
+
+namespace {
+
+constexpr uint32_t kStepPlanMagic = 0x54504153u;
+
+// What a tpa_step_plan holds: the checked launch arguments of one decode step.
+struct StepPlan {
+  uint32_t magic;  // kStepPlanMagic once initialised
+  int device;
+  DecodeStepArgs step;
+  TensorDecodeArgs args;  // args.step is pointed at `step` at each run (the plan may be copied)
+  void* stage_dst;
+  const void* stage_src;
+  size_t stage_bytes;
+};
+static_assert(sizeof(StepPlan) <= sizeof(tpa_step_plan), "tpa_step_plan is too small");
+static_assert(alignof(StepPlan) <= alignof(tpa_step_plan), "tpa_step_plan is under-aligned");
+
+}  // namespace
+
+tpa_status tpa_step_plan_init(tpa_step_plan* plan, const tpa_cache* cache, const int32_t* positions,
+                              const void* a_k, const void* b_k, const void* a_v, const void* b_v, int32_t r_q,
+                              const void* a_q, const void* q, float scale, float* out, int32_t max_len,
+                              int32_t advance, int32_t num_splits, int32_t kernel, void* workspace,
+                              size_t workspace_bytes, void* stage_dst, const void* stage_src, size_t stage_bytes) {
+  if (!plan) return fail(TPA_ERR_NULL, "plan is NULL");
+  memset(plan, 0, sizeof(*plan));
+  StepPlan* sp = reinterpret_cast<StepPlan*>(plan);
+  if (r_q < 0) return fail(TPA_ERR_SHAPE, "r_q = %d < 0", r_q);
+  if (stage_bytes > 0 && (!stage_dst || !stage_src)) return fail(TPA_ERR_NULL, "stage_dst or stage_src is NULL");
+  sp->step.a_k = a_k;
+  sp->step.b_k = b_k;
+  sp->step.a_v = a_v;
+  sp->step.b_v = b_v;
+  sp->step.advance = advance;
+  const tpa_status s = decode_impl(cache, q, r_q > 0 ? a_q : nullptr, r_q, positions, scale, out, max_len,
+                                   num_splits, kernel, workspace, workspace_bytes, nullptr, &sp->step, nullptr,
+                                   &sp->args);
+  if (s != TPA_OK) {
+    memset(plan, 0, sizeof(*plan));
+    return s;
+  }
+  const cudaError_t e = cudaGetDevice(&sp->device);
+  if (e != cudaSuccess) {
+    memset(plan, 0, sizeof(*plan));
+    return cuda_fail(e, "device query");
+  }
+  sp->stage_dst = stage_bytes > 0 ? stage_dst : nullptr;
+  sp->stage_src = stage_bytes > 0 ? stage_src : nullptr;
+  sp->stage_bytes = stage_bytes;
+  sp->magic = kStepPlanMagic;
+  return TPA_OK;
+}
+
+tpa_status tpa_step_plan_run(const tpa_step_plan* plan, void* stream) {
+  if (!plan) return fail(TPA_ERR_NULL, "plan is NULL");
+  const StepPlan* sp = reinterpret_cast<const StepPlan*>(plan);
+  if (sp->magic != kStepPlanMagic) return fail(TPA_ERR_SHAPE, "the plan is not initialised");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  if (dev != sp->device) return fail(TPA_ERR_UNSUPPORTED, "the plan is for device %d, device %d is current", sp->device, dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (sp->stage_bytes > 0) {
+    e = cudaMemcpyAsync(sp->stage_dst, sp->stage_src, sp->stage_bytes, cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "input copy");
+  }
+  TensorDecodeArgs a = sp->args;
+  a.step = &sp->step;
+  e = launch_tensor_decode(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "tensor decode launch");
   return TPA_OK;
 }
 

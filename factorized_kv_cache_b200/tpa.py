@@ -59,6 +59,11 @@ class tpa_cache(ctypes.Structure):
     ]
 
 
+class tpa_step_plan(ctypes.Structure):
+    """Caller-owned storage of a bound decode step (contents private to libtpa)."""
+    _fields_ = [("opaque", ctypes.c_uint64 * 256)]
+
+
 _lib = None
 
 
@@ -89,6 +94,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_decode_step": (ctypes.c_int, [C, P, P, P, P, P, I32, P, P, ctypes.c_float, P, I32, I32, I32, I32, P,
                                             ctypes.c_size_t, P]),
         "tpa_stage_async": (ctypes.c_int, [P, P, ctypes.c_size_t, P]),
+        "tpa_step_plan_init": (ctypes.c_int, [ctypes.POINTER(tpa_step_plan), C, P, P, P, P, P, I32, P, P,
+                                               ctypes.c_float, P, I32, I32, I32, I32, P, ctypes.c_size_t, P, P,
+                                               ctypes.c_size_t]),
+        "tpa_step_plan_run": (ctypes.c_int, [ctypes.POINTER(tpa_step_plan), P]),
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
@@ -455,13 +464,14 @@ def _stage_bytes(dst: torch.Tensor, src: torch.Tensor) -> int:
 
 
 class DecodeStepPlan:
-    """tpa_decode_step bound to fixed buffers, for a generation loop: the arguments are checked
-    and marshalled once, and each call is a single C call with the stored pointers.  The
-    buffers' contents may change between calls (new factors, query, positions); the tensors
-    themselves, and the cache's planes, must stay the same objects.  ``out`` may be pinned host
-    memory: the kernels then write the output straight to the host.  ``stage=(host_in,
-    dev_in)``: each call first copies ``host_in`` (pinned) into ``dev_in`` (the device memory
-    the bound inputs live in) on the same stream, for a loop whose inputs come from the host."""
+    """tpa_decode_step bound to fixed buffers, for a generation loop (tpa_step_plan_init): the
+    arguments are checked and marshalled once, and each call is one C call, tpa_step_plan_run,
+    with the plan and the stream.  The buffers' contents may change between calls (new factors,
+    query, positions); the tensors themselves, and the cache's planes, must stay the same
+    objects.  ``out`` may be pinned host memory: the kernels then write the output straight to
+    the host.  ``stage=(host_in, dev_in)``: each call first copies ``host_in`` (pinned) into
+    ``dev_in`` (the device memory the bound inputs live in) on the same stream, in the same C
+    call, for a loop whose inputs come from the host."""
 
     def __init__(self, cache: TpaCache, positions, a_k, b_k, a_v, b_v, out, q=None, a_q=None, b_q=None,
                  scale: float | None = None, max_len: int | None = None, advance: bool = True, num_splits: int = 0,
@@ -506,24 +516,24 @@ class DecodeStepPlan:
         self.out = out
         self._keep = (cache, positions, a_k, b_k, a_v, b_v, qa, qb, out, workspace_buf)
         self._device = dev
-        self._fn = lib.tpa_decode_step
-        self._args = (ctypes.byref(self._struct), _ptr(positions), _ptr(a_k), _ptr(b_k), _ptr(a_v), _ptr(b_v), r_q,
-                      _ptr(qa), _ptr(qb), float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits, kernel,
-                      _ptr(workspace_buf), nbytes)
-        self._stage = None
+        staged = (None, None, 0)
         if stage is not None:
             host_in, dev_in = stage
             if dev_in.device != dev:
                 raise ValueError(f"stage: dev_in is on {dev_in.device}, expected {dev}")
-            self._stage = (_ptr(dev_in), _ptr(host_in), _stage_bytes(dev_in, host_in))
-            self._stage_fn = lib.tpa_stage_async
+            staged = (_ptr(dev_in), _ptr(host_in), _stage_bytes(dev_in, host_in))
             self._keep += (host_in, dev_in)
+        self._plan = tpa_step_plan()
+        with torch.cuda.device(dev):
+            _check(lib.tpa_step_plan_init(ctypes.byref(self._plan), ctypes.byref(self._struct), _ptr(positions),
+                                          _ptr(a_k), _ptr(b_k), _ptr(a_v), _ptr(b_v), r_q, _ptr(qa), _ptr(qb),
+                                          float(scale), _ptr(out), max_len, 1 if advance else 0, num_splits, kernel,
+                                          _ptr(workspace_buf), nbytes, *staged))
+        self._plan_ref = ctypes.byref(self._plan)
+        self._run = lib.tpa_step_plan_run
 
     def __call__(self, stream=None):
-        s = _stream(stream, self._device)
-        if self._stage is not None:
-            _check(self._stage_fn(*self._stage, s))
-        _check(self._fn(*self._args, s))
+        _check(self._run(self._plan_ref, _stream(stream, self._device)))
         return self.out
 
     def graph(self, host_in=None, dev_in=None, host_out=None, stream=None):

@@ -280,6 +280,47 @@ tpa_status tpa_decode_step(const tpa_cache* cache, const int32_t* positions, con
 tpa_status tpa_stage_async(void* dst, const void* src, size_t bytes, void* stream);
 
 /*
+ * A decode step bound once, for a generation loop: tpa_step_plan_init checks
+ * and stores the arguments of tpa_decode_step (plus an optional input copy),
+ * and each tpa_step_plan_run then launches the step with no argument
+ * marshalling or checking.  A deployment convenience with no counterpart on
+ * the pages; the step computed is exactly tpa_decode_step's.
+ * The plan is caller-owned storage whose contents are private to libtpa; it
+ * holds no resources (nothing to release) and may be copied.
+ */
+typedef struct tpa_step_plan {
+  uint64_t opaque[256];
+} tpa_step_plan;
+
+/*
+ * Fills `plan` for tpa_decode_step with these arguments (same meaning, layout
+ * and checks as tpa_decode_step; the stream is given to each run instead).
+ * stage_bytes > 0: every run first copies stage_bytes from stage_src (pinned
+ * host memory) to stage_dst (device memory) on the run's stream, as
+ * tpa_stage_async does, so a loop whose inputs come from the host packs them
+ * into stage_src and the copy lands where the bound inputs live.
+ * The buffers must stay allocated, and the cache's planes and seq_lens in
+ * place, while the plan is used; their contents may change between runs.
+ * Runs must use the device that was current at init.  On error the plan is
+ * left unusable (a run returns TPA_ERR_SHAPE).
+ * Errors: those of tpa_decode_step; NULL (plan, or stage_dst / stage_src with
+ * stage_bytes > 0); CUDA (device query).
+ */
+tpa_status tpa_step_plan_init(tpa_step_plan* plan, const tpa_cache* cache, const int32_t* positions,
+                              const void* a_k, const void* b_k, const void* a_v, const void* b_v, int32_t r_q,
+                              const void* a_q, const void* q, float scale, float* out, int32_t max_len,
+                              int32_t advance, int32_t num_splits, int32_t kernel, void* workspace,
+                              size_t workspace_bytes, void* stage_dst, const void* stage_src, size_t stage_bytes);
+
+/*
+ * One step of an initialised plan on `stream`: the input copy if the plan has
+ * one, then the step's two launches, as tpa_decode_step.
+ * Errors: NULL (plan), SHAPE (plan not initialised), UNSUPPORTED (another
+ * device is current), CUDA (a copy or launch failed).
+ */
+tpa_status tpa_step_plan_run(const tpa_step_plan* plan, void* stream);
+
+/*
  * tpa_decode_attention for callers that cannot allocate device memory (no
  * counterpart on the page; this is a deployment convenience).  Same
  * arguments and result as tpa_decode_attention minus the workspace: the

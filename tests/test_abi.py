@@ -156,6 +156,30 @@ def test_stage_rejects_bad_arguments():
         T.tpa_stage_async(torch.empty(4), torch.empty(4))          # src is not pinned
 
 
+def test_step_plan_rejects_bad_arguments():
+    lib = T.load_library()
+    P = 0x90000
+
+    def init(plan, c=None, rq=0, ak=P, stage=(None, None, 0), kernel=0):
+        c = _fake_cache() if c is None else c
+        return lib.tpa_step_plan_init(plan, ctypes.byref(c), 0x70000, ak, P, P, P, rq, None, 0x60000, 0.1, 0x80000,
+                                      64, 1, 0, kernel, None, 0, *stage)
+
+    plan = T.tpa_step_plan()
+    assert lib.tpa_step_plan_run(None, None) == 1
+    assert lib.tpa_step_plan_run(ctypes.byref(plan), None) == 2        # never initialised
+    assert init(None) == 1
+    assert init(ctypes.byref(plan), rq=-1) == 2
+    assert init(ctypes.byref(plan), ak=None) == 1
+    assert init(ctypes.byref(plan), ak=P + 4) == 6
+    assert init(ctypes.byref(plan), stage=(None, 0xA0000, 64)) == 1
+    assert init(ctypes.byref(plan), stage=(0xA0000, None, 64)) == 1
+    assert init(ctypes.byref(plan), c=_fake_cache(dtype=T.TPA_F32)) == 3
+    assert init(ctypes.byref(plan), kernel=T.TPA_KERNEL_SIMT) == 3
+    assert lib.tpa_step_plan_run(ctypes.byref(plan), None) == 2        # a failed init leaves it unusable
+    assert ctypes.sizeof(T.tpa_step_plan) == 2048
+
+
 def test_append_rejects_bad_arguments():
     lib = T.load_library()
     c = _fake_cache()
