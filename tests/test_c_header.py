@@ -1,5 +1,6 @@
 """include/tpa.h is a C header: a C99 translation unit that includes it and takes the address
-of every declared entry point compiles with gcc -Wall -Werror and links against libtpa.so."""
+of every declared entry point compiles with gcc -Wall -Werror and links against libtpa.so, and
+its host-side checks answer a C caller (no GPU needed)."""
 import os
 import shutil
 import subprocess
@@ -23,6 +24,9 @@ int main(void) {{
 {body}
   tpa_cache c = {{0}};
   c.batch = 1;
+  tpa_step_plan plan = {{{{0}}}};
+  /* a plan that was never initialised is refused without touching the device */
+  if (tpa_step_plan_run(NULL, NULL) != TPA_ERR_NULL || tpa_step_plan_run(&plan, NULL) != TPA_ERR_SHAPE) return 2;
   printf("%zu %d\\n", tpa_factor_elements_per_token(32, 128, 1, 1), (int)(fns[0] != 0) + c.batch);
   return 0;
 }}
