@@ -277,6 +277,35 @@ def pin_brute_force_decode(O):
                 assert abs(o[i, k] - ref) <= 1e-12 * (1 + abs(ref)), (seed, i, k, o[i, k], ref)
 
 
+def pin_brute_force_from_unrotated(O):
+    """End-to-end decode from unrotated factors by scalar loops: each cached key row rotated
+    at its own token's position (not the query's), rounded to the storage dtype when one is
+    given (round_to_storage is itself pinned against PyTorch's conversion), the query rotated
+    at its position, then softmax over the cached tokens with math.fsum."""
+    cases = [(3, 2, 4, 2, 1, None), (4, 2, 6, 1, 2, "bf16"), (2, 1, 4, 2, 2, "f32"), (5, 3, 8, 2, 2, "bf16")]
+    for seed, (L, h, d, rk, rv, storage) in enumerate(cases):
+        c = _rand_case(140 + seed, L, h, d, rk, rv)
+        pos = [float(5 * s + 2) for s in range(L)]
+        qpos, scale, base = 31.0, 0.9, 100.0
+        o = O.decode_attention_from_unrotated(c["a_k"], c["b_k"], c["a_v"], c["b_v"], np.array(pos), c["q"], qpos,
+                                              scale, base, storage=storage)
+        rows = [[O.round_to_storage(np.array(_brute_rot(list(c["b_k"][s, r]), pos[s], base)), storage).tolist()
+                 for r in range(rk)] for s in range(L)]
+        for i in range(h):
+            qr = _brute_rot(list(c["q"][i]), qpos, base)
+            z = []
+            for s in range(L):
+                key = [math.fsum(c["a_k"][s, r, i] * rows[s][r][k] for r in range(rk)) / rk for k in range(d)]
+                z.append(scale * math.fsum(qr[k] * key[k] for k in range(d)))
+            m = max(z)
+            w = [math.exp(x - m) for x in z]
+            tot = math.fsum(w)
+            for k in range(d):
+                ref = math.fsum(w[s] / tot * math.fsum(c["a_v"][s, r, i] * c["b_v"][s, r, k] for r in range(rv)) / rv
+                                for s in range(L))
+                assert abs(o[i, k] - ref) <= 1e-12 * (1 + abs(ref)), (seed, storage, i, k, o[i, k], ref)
+
+
 def pin_brute_force_prefill(O):
     """Causal prefill with a previous chunk (P > 0) by scalar loops on tiny inputs."""
     g = np.random.default_rng(21)
@@ -567,6 +596,7 @@ ALL_PINS = [
     pin_general_sdpa,
     pin_prefill_causal_sdpa,
     pin_brute_force_decode,
+    pin_brute_force_from_unrotated,
     pin_brute_force_prefill,
     pin_prefill_first_row,
     pin_factored_query_rank_one,

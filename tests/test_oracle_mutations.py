@@ -127,6 +127,22 @@ def _lse_log2(a_k, b_k_rot, a_v, b_v, q, q_pos, scale, base, block=8192):   # ba
     return o, lse / np.log(2.0)
 
 
+_from_unrot = O.decode_attention_from_unrotated
+
+
+def _unrot_keys_at_query_position(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, storage=None):
+    return _from_unrot(a_k, b_k, a_v, b_v, np.full(np.shape(positions), q_pos, dtype=np.float64), q, q_pos, scale,
+                       base, storage)
+
+
+def _unrot_storage_ignored(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, storage=None):
+    return _from_unrot(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, None)
+
+
+def _unrot_keys_left_unrotated(a_k, b_k, a_v, b_v, positions, q, q_pos, scale, base, storage=None):
+    return O.decode_attention(a_k, O.round_to_storage(b_k, storage), a_v, b_v, q, q_pos, scale, base)
+
+
 def _round_truncate(x, storage):               # truncation instead of round-to-nearest-even
     if storage != "bf16":
         return _round(x, storage)
@@ -164,6 +180,9 @@ MUTANTS = {
     "merge_unnormalised": ("merge_lse", _merge_unnormalised),
     "merge_plain_mean": ("merge_lse", _merge_plain_mean),
     "lse_log2": ("decode_attention_lse", _lse_log2),
+    "unrotated_keys_at_query_position": ("decode_attention_from_unrotated", _unrot_keys_at_query_position),
+    "unrotated_storage_ignored": ("decode_attention_from_unrotated", _unrot_storage_ignored),
+    "unrotated_keys_left_unrotated": ("decode_attention_from_unrotated", _unrot_keys_left_unrotated),
 }
 
 
