@@ -14,6 +14,13 @@ step, so every step attends exactly sum_b L_b tokens.
 One step of the prefill workload writes the prompt's factors and runs the
 causal prefill over them.
 
+The default workload is decode_b32_var32k (B=32, R=2, lengths uniform in
+[16384, 32768]), the largest decode that fits one GPU.  On one GPU the same run
+also times the long-context decode (decode_long_512k, the fused step) and the
+causal prefill (prefill_b4_t4k) and adds them to the line as ``long_context``
+and ``prefill``, each with its own roofline and clock record (``--extras``).
+The CPU oracle baseline runs on rank 0 at N=1 only.
+
 Rank 0 prints one JSON line.  Under torchrun every rank runs its own batch on
 its own GPU (weak scaling, no collective on the data path); the time is the
 maximum over ranks.
@@ -60,6 +67,11 @@ def source_sha(paths):
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+TRAFFIC_SOURCE = ("not measured in this run: dram__bytes_read.sum + dram__bytes_write.sum of one launch of the "
+                  "dominant kernel from a committed ncu capture (profiles/ncu_traffic.json), reported only while "
+                  "the hash of the kernel's sources matches the captured one (null otherwise)")
 
 
 def ncu_traffic(workload: str, kernel_sources):
@@ -201,7 +213,7 @@ def decode_host_inputs(w, rank):
     return S.decode_inputs(rank_workload(w, rank))
 
 
-def run_ours_decode(args, w, rank, world, dev):
+def run_ours_decode(args, w, rank, world, dev, with_e2e=True):
     import torch
     import torch.distributed as dist
     from factorized_kv_cache_b200 import synthetic as S
@@ -354,6 +366,18 @@ def run_ours_decode(args, w, rank, world, dev):
     if T.tpa_read_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
 
+    e2e = run_decode_e2e(args, K, W, B, w, inputs, fused, rq, caches, copies, cap, kernel, ws, out, step, stream,
+                         world, dev, tokens_per_step) if with_e2e else None
+    return _decode_result(args, w, world, K, W, B, lengths, tokens_per_step, per_tok, fused, query_bytes, rq,
+                          kernel, splits, copies, cache_bytes, elapsed_ms, decode_ms, n_calls, clk, e2e), x, lengths
+
+
+def run_decode_e2e(args, K, W, B, w, inputs, fused, rq, caches, copies, cap, kernel, ws, out, step, stream, world,
+                   dev, tokens_per_step):
+    """The decode step end to end through the public API with host buffers."""
+    import torch
+    import torch.distributed as dist
+    from factorized_kv_cache_b200 import tpa as T
     # e2e through the public API with host buffers: every step copies its inputs from one pinned
     # host buffer (one H2D copy) and reads the output back (one D2H copy), then synchronises
     layout, off = [], 0
@@ -402,7 +426,13 @@ def run_ours_decode(args, w, rank, world, dev):
         e2e_step(k % copies)
     e2e_s = time.perf_counter() - t0
     e2e_s = max_over_ranks(e2e_s, world, dev)
+    return {"value": world * tokens_per_step * e2e_steps / e2e_s, "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
+
+def _decode_result(args, w, world, K, W, B, lengths, tokens_per_step, per_tok, fused, query_bytes, rq, kernel,
+                   splits, copies, cache_bytes, elapsed_ms, decode_ms, n_calls, clk, e2e):
+    from factorized_kv_cache_b200 import tpa as T
     launches_per_step = 2 if fused else 1 + 1 + (1 if splits > 1 else 0)
     # factor bytes of every attended token (cached, or the step's own read from its inputs), the
     # step's token stored (fused), the query and the fp32 output
@@ -452,19 +482,19 @@ def run_ours_decode(args, w, rank, world, dev):
         "roofline": {
             "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "traffic": ncu_traffic(w.name, kernel_src) if kernel_src else None,
-            "peak_kind": kind, "kernel": ("fused step call" if fused else "decode attention call") +
-                                          " (split kernel + merge), timed right after the K "
-                                          "timed steps on the same stream: graphs of back-to-back decode calls "
-                                          "over the same cache copies, CUDA events around each graph",
+            "traffic_source": TRAFFIC_SOURCE, "peak_kind": kind,
+            "kernel": ("fused step call" if fused else "decode attention call") +
+                      " (split kernel + merge), timed right after the K timed steps on the same stream: graphs of "
+                      "back-to-back decode calls over the same cache copies, CUDA events around each graph",
             "calls_per_graph": n_calls,
             "algorithmic_bytes_per_launch": bytes_per_decode, "mean_launch_us": mean_decode_s * 1e6,
         },
-        "e2e": {"value": world * tokens_per_step * e2e_steps / e2e_s, "unit": "tokens/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": K * launches_per_step,
         "clocks": clk,
     }
-    return res, x, lengths
+    if e2e is not None:
+        res["e2e"] = e2e
+    return res
 
 
 def run_ours_decode_sharded(args, w, rank, world, dev):
@@ -863,7 +893,12 @@ def run_ours_prefill(args, w, rank, world, dev):
     e2e_s = max_over_ranks(time.perf_counter() - t0, world, dev)
 
     pairs = B * Tn * (Tn + 1) // 2
-    flops = pairs * w.heads * 2 * w.head_dim * (w.r_k + w.r_v)   # score + value contractions, per (query, key) pair
+    # algorithmic flops per causal (query, key) pair, counted with the scores formed on the rank
+    # factors (B_Q . B_K^T, R_Q R_K dot products of d_h shared by all heads) and the value
+    # contraction per head (R_V rank-one updates of d_h); the dense per-head count (a d_h dot
+    # product per head and rank of the key, plus the same value term) is reported beside it
+    flops = pairs * (2 * w.r_q * w.r_k * w.head_dim + 2 * w.heads * w.r_v * w.head_dim)
+    flops_dense = pairs * w.heads * 2 * w.head_dim * (w.r_k + w.r_v)
     mean_s = statistics.mean(pre_ms) / 1e3
     peaks, kind = measured_peaks()
     achieved = flops / mean_s / 1e12
@@ -882,8 +917,13 @@ def run_ours_prefill(args, w, rank, world, dev):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
                      "traffic": ncu_traffic(w.name, src), "peak_kind": kind + " (bf16 burst)",
-                     "kernel": "prefill attention call (query build + causal attention)",
-                     "algorithmic_flops_per_launch": flops, "mean_launch_us": mean_s * 1e6},
+                     "kernel": "prefill attention call",
+                     "algorithmic_flops_per_launch": flops,
+                     "flops_count": "rank-factor scores (2 R_Q R_K d_h per pair) + per-head values (2 h R_V d_h "
+                                    "per pair), causal pairs only",
+                     "dense_equivalent_flops_per_launch": flops_dense,
+                     "dense_equivalent_tflops": flops_dense / mean_s / 1e12,
+                     "mean_launch_us": mean_s * 1e6},
         "e2e": {"value": world * B * Tn * e2e_steps / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": K * 3,
@@ -903,13 +943,46 @@ def add_prefill_cpu_baseline(res, x, w, target_s):
                                      f"{workers} spawned processes"}
 
 
+DEFAULT_WORKLOAD = "decode_b32_var32k"   # the largest single-GPU decode workload
+
+
+def add_extras(args, res, dev):
+    """Two more workloads timed in the same run on one GPU, each with its own roofline and clock
+    record: the long-context decode (one sequence of 524288 tokens, the fused step) and the
+    causal prefill (its own metric: query tokens/s and tensor TFLOP/s)."""
+    import gc
+    import torch
+    from factorized_kv_cache_b200 import synthetic as S
+    gc.collect()
+    torch.cuda.empty_cache()
+    keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "roofline", "e2e", "gpu_launches",
+            "clocks")
+    wl = S.WORKLOADS["decode_long_512k"]
+    r_long, x, _ = run_ours_decode(args, wl, 0, 1, dev)
+    del x
+    res["long_context"] = dict({"metric": METRIC}, **{k: r_long[k] for k in keep if k in r_long})
+    gc.collect()
+    torch.cuda.empty_cache()
+    wp = S.WORKLOADS["prefill_b4_t4k"]
+    pargs = argparse.Namespace(**vars(args))
+    pargs.steps = max(3, min(args.steps, 10))
+    r_pre, x = run_ours_prefill(pargs, wp, 0, 1, dev)
+    del x
+    if args.cpu_seconds > 0:
+        add_prefill_cpu_baseline(r_pre, None, wp, min(args.cpu_seconds, 8.0))
+    res["prefill"] = dict({"metric": PREFILL_METRIC}, **{k: r_pre[k] for k in keep + ("cpu_baseline",)
+                                                         if k in r_pre})
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode_b8_l8k",
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     choices=["decode_tiny_f32", "decode_b8_l8k", "decode_b32_var32k", "prefill_b4_t4k",
                              "decode_long_512k"])
     ap.add_argument("--kernel", choices=["auto", "simt", "tensor", "tensor_sync"], default="auto")
@@ -920,6 +993,9 @@ def main():
     ap.add_argument("--shard-tokens", action="store_true",
                     help="decode workloads: split every sequence's token range across the ranks (strong scaling)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample length (0: skip)")
+    ap.add_argument("--extras", choices=["auto", "on", "off"], default="auto",
+                    help="one GPU: also time the long-context decode and the causal prefill in the same run "
+                         "(auto: with the default workload)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling smaller cases)")
     ap.add_argument("--seq-len", type=int, default=0, help="override the workload's length / prompt tokens")
     args = ap.parse_args()
@@ -954,16 +1030,21 @@ def main():
     try:
         if isinstance(w, S.PrefillWorkload):
             res, x = run_ours_prefill(args, w, rank, world, dev)
-            if rank == 0 and args.cpu_seconds > 0:
+            if rank == 0 and world == 1 and args.cpu_seconds > 0:
                 add_prefill_cpu_baseline(res, x, w, args.cpu_seconds)
         elif args.shard_tokens:
             res, x, lengths = run_ours_decode_sharded(args, w, rank, world, dev)
-            if rank == 0 and args.cpu_seconds > 0:
+            if rank == 0 and world == 1 and args.cpu_seconds > 0:
                 add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
         else:
             res, x, lengths = run_ours_decode(args, w, rank, world, dev)
-            if rank == 0 and args.cpu_seconds > 0:
+            if rank == 0 and world == 1 and args.cpu_seconds > 0:
                 add_cpu_baseline(res, x, w, lengths, args.cpu_seconds)
+            del x
+            extras = args.extras == "on" or (args.extras == "auto" and args.workload == DEFAULT_WORKLOAD and
+                                             args.batch == 0 and args.seq_len == 0)
+            if extras and world == 1:
+                add_extras(args, res, dev)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
