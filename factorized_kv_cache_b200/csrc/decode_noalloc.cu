@@ -14,7 +14,8 @@
 // sees a host-side stand-in under the array's name, so the device address is
 // looked up with cudaGetSymbolAddress, once per device, on the first call
 // made with that device current; that first call on each device should
-// therefore come before any stream capture.  All calls on a device share the
+// therefore come before any stream capture (a lookup that fails is not kept,
+// and the next call tries again).  All calls on a device share the
 // one array, which keeps whatever the previous call left in it: the decode
 // kernels write every partial before the merge reads it, so nothing has to
 // start at zero, but two calls that overlap on the GPU (different streams,
@@ -34,22 +35,24 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxNoAllocDevices = 64;
-std::once_flag g_scratch_once[kMaxNoAllocDevices];
-void* g_scratch_ptr[kMaxNoAllocDevices];
-cudaError_t g_scratch_status[kMaxNoAllocDevices];
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxNoAllocDevices];  // non-null once a lookup on that device has succeeded
 
-// Device address of the scratch array on the current device.
+// Device address of the scratch array on the current device.  Only a successful lookup is
+// kept: a failed one (made during a stream capture, or a transient error) is tried again on
+// the next call.
 cudaError_t scratch_address(void** ptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxNoAllocDevices) return cudaErrorInvalidDevice;
-  std::call_once(g_scratch_once[dev], [dev]() {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    g_scratch_status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
     g_scratch_ptr[dev] = p;
-  });
-  if (g_scratch_status[dev] != cudaSuccess) return g_scratch_status[dev];
+  }
   *ptr = g_scratch_ptr[dev];
   return cudaSuccess;
 }

@@ -503,6 +503,21 @@ tpa_status tpa_step_plan_init(tpa_step_plan* plan, const tpa_cache* cache, const
     memset(plan, 0, sizeof(*plan));
     return cuda_fail(e, "device query");
   }
+  if (stage_bytes > 0) {
+    // the bound copy runs every step without further checks: its ends must be device memory of
+    // this device and page-locked host memory
+    cudaPointerAttributes ad, as;
+    const bool dst_ok = cudaPointerGetAttributes(&ad, stage_dst) == cudaSuccess &&
+                        (ad.type == cudaMemoryTypeDevice || ad.type == cudaMemoryTypeManaged) &&
+                        ad.device == sp->device;
+    const bool src_ok = cudaPointerGetAttributes(&as, stage_src) == cudaSuccess && as.type == cudaMemoryTypeHost;
+    cudaGetLastError();  // a failed attribute query leaves no error behind
+    if (!dst_ok || !src_ok) {
+      memset(plan, 0, sizeof(*plan));
+      return fail(TPA_ERR_UNSUPPORTED, "%s", !dst_ok ? "stage_dst is not device memory of the current device"
+                                                     : "stage_src is not page-locked host memory");
+    }
+  }
   sp->stage_dst = stage_bytes > 0 ? stage_dst : nullptr;
   sp->stage_src = stage_bytes > 0 ? stage_src : nullptr;
   sp->stage_bytes = stage_bytes;

@@ -304,7 +304,10 @@ typedef struct tpa_step_plan {
  * Runs must use the device that was current at init.  On error the plan is
  * left unusable (a run returns TPA_ERR_SHAPE).
  * Errors: those of tpa_decode_step; NULL (plan, or stage_dst / stage_src with
- * stage_bytes > 0); CUDA (device query).
+ * stage_bytes > 0); UNSUPPORTED (stage_bytes > 0 and stage_dst is not device
+ * memory of the current device, or stage_src is not page-locked host memory:
+ * both are checked here, once, since runs copy without checks); CUDA (device
+ * query).
  */
 tpa_status tpa_step_plan_init(tpa_step_plan* plan, const tpa_cache* cache, const int32_t* positions,
                               const void* a_k, const void* b_k, const void* a_v, const void* b_v, int32_t r_q,
@@ -328,12 +331,15 @@ tpa_status tpa_step_plan_run(const tpa_step_plan* plan, void* stream);
  * on every GPU that loads the library until the process exits.  Nothing is
  * allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - num_splits == 0: the default split count, lowered if needed until the
- *     partials fit in the 16 MiB array (one split needs no scratch at all).
+ *     partials fit in the 16 MiB array (the CUDA-core kernel with one split
+ *     needs no scratch; the tcgen05 kernel's partials, at its fixed grid of
+ *     one CTA per SM, take about 5 MB at the largest batch and always fit).
  *   - num_splits > 0 whose partials exceed 16 MiB: TPA_ERR_WORKSPACE, nothing
  *     launched, and tpa_last_error_message() says how much was needed.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  A lookup that fails returns TPA_ERR_CUDA
+ *     and is not remembered: the next call tries again.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents (no call depends on them); calls that overlap on the
  *     GPU race on the array: order them on one stream or with events.
