@@ -1,51 +1,64 @@
 // Causal prefill on the 5th-generation tensor cores (tcgen05, TMEM
-// accumulators, TMA), bf16, h = 32, d_h = 128, R_K = R_V = R in {1, 2}, R_Q <= 8.
+// accumulators, TMA), bf16 cache, h = 32, d_h = 128, R_K = R_V = R in {1, 2},
+// R_Q <= 8.
 //
 // What it computes (Tensor Product Attention Is All You Need, sections
-// 解决思路 for Q_t = (1/R_Q) A_Q^T B_Q, 关键设计 for the K/V factors,
-// RoPE 兼容性 for RoPE on the B factors, FlashTPA for attention on factors):
-// for query t of a chunk (cache slot P + t) and head i,
+// 解决思路 for Q_t = (1/R_Q) A_Q^T B_Q, 关键设计 / 张量积分解 for the K/V
+// factors, RoPE 兼容性 for RoPE on the B factors, FlashTPA for attention on
+// the factors): for query t of a chunk (cache slot P + t) and head i,
 //   q_{t,i}     = (1/R_Q) sum_j A_Q[t, j, i] RoPE(B_Q[t, j], pos_t)
 //   S[t, (s,r)] = q_{t,i} . B~_K[s, r]                       (tensor cores)
 //   z[t, s]     = scale/R_K sum_r A_K[s, r, i] S[t, (s, r)],  s <= P + t
 //   W[t, (s,r)] = softmax_s(z)[t, s] A_V[s, r, i] / R_V
 //   O[t, i, :]  = sum_(s,r) W[t, (s,r)] B_V[s, r, :]         (tensor cores)
-// The dense per-head query is the only thing expanded: it is built once per
-// chunk in fp32 by prefill_q_kernel and split by the softmax threads into
-// bf16 high and low parts in TMEM.  Keys and values stay factorized: the
-// score MMA contracts the query with B_K rows, and the value MMA contracts
-// the softmax weights with B_V rows.  Putting the head factors on the query
-// side of the MMA (a dense Q tile per head) costs 2 h d_h R_K tensor flops
-// per (query, key) pair and little CUDA-core work; contracting B_Q with B_K
-// first would save tensor flops but needs ~h R_Q R_K CUDA-core FMAs per pair
-// to apply A_Q and A_K, which is slower on this machine.
+// Keys and values stay factorized: the score MMA contracts the query with B_K
+// rows, and the value MMA contracts the softmax weights with B_V rows.  Putting
+// the head factors on the query side of the MMA (a dense query tile per head)
+// costs 2 h d_h R_K tensor flops per (query, key) pair and little CUDA-core
+// work; contracting B_Q with B_K first would save tensor flops but needs
+// ~h R_Q R_K CUDA-core FMAs per pair to apply A_Q and A_K, on the path that
+// already bounds this kernel (the softmax).
+//
+// Operands are fp16.  A pre-pass (prefill_prep_kernel, launched just before)
+// writes to the workspace (i) fp16 copies of the B_K and B_V rows of every
+// sequence's cached tokens, exact for bf16 values in fp16's normal range
+// (bf16's 8 significant bits fit in fp16's 11; magnitudes above 65504 are not
+// supported by this path and become infinite), and (ii) the chunk's B_Q rank
+// rows rotated at their positions, rounded to fp16.  The dense per-head query
+// is formed in this kernel from (ii) and A_Q, in fp32, and rounded once to
+// fp16 in TMEM; it is never written to global memory.  With the softmax
+// weights also rounded once to fp16 (11 significant bits: ~4e-4 relative each
+// on the prefill workload, against ~3.5e-3 for a bf16 rounding) one MMA per
+// contraction suffices where bf16 needed a high + low pair.
 //
 // CTA = (sequence, head, tile of 128 queries); heavy (late) query tiles are
 // dispatched first.  Both MMAs take their A operand from TMEM, so shared
 // memory only feeds their B operands (a 128-row B_K or B_V tile per 16 of K).
-// Roles (352 threads): warp 0 issues TMA loads of 128-row tiles {B_K, B_V,
-// the 8-head slices of A_K and A_V holding the head} into a 3-stage ring;
-// warp 1 allocates all 512 TMEM columns and one of its threads issues the
-// MMAs; warps 2-9 run the softmax, two threads per query row (TMEM lane):
-// warps 2-5 take the first 64 cache rows of a tile, warps 6-9 the last 64;
-// warp 10 stages A_K and A_V of the head as fp32 (scale folded in) and zeroes
-// B_V rows past the sequence end, which may hold NaN.
+// Roles (352 threads): warp 0 issues TMA loads of 128-row tiles {B_K, B_V (the
+// fp16 copies), the 8-head slices of A_K and A_V holding the head} into a
+// 3-stage ring; warp 1 allocates all 512 TMEM columns and one of its threads
+// issues the MMAs; warps 2-9 form the queries, then run the softmax, two
+// threads per query row (TMEM lane): warps 2-5 take the first 64 cache rows
+// of a tile, warps 6-9 the last 64; warp 10 stages A_K and A_V of the head as
+// fp32 (scales folded in) and zeroes B_V rows past the sequence end, which
+// may hold NaN.
 // TMEM: S double-buffered in columns [128 b, +128) and overwritten in place by
-// W as bf16 hi (first 64 columns) and lo (next 64), O in [256, 384), the
-// query hi in [384, 448) and lo in [448, 512).  Per key tile j:
-//   S = (Q_hi + Q_lo) B_K^T  (M = 128 queries, N = 128 rows, K = 128), into
-//       the buffer that tile j - 1 does not use, so it overlaps the softmax
-//       of tile j - 1;
+// W (fp16, two cache rows per column, the first 64 columns), O in [256, 384),
+// the query (fp16) in [384, 448).  Per key tile j:
+//   S = Q B_K^T  (M = 128 queries, N = 128 rows, K = 128), into the buffer
+//       that tile j - 1 does not use, so it overlaps the softmax of tile j - 1;
 //   softmax: A_K weighting, causal mask, online softmax with a lazily
-//       rescaled maximum (only when it grows by more than 2^8; the two
-//       threads of a row share their maxima through shared memory), W = p A_V;
-//   O += W_hi B_V + W_lo B_V  (B_V MN-major).
-// Both the query and W are split into two bf16 parts, which keeps them to
-// ~16 bits: one bf16 rounding of either costs ~3.5e-3 relative error on the
-// prefill workload, above its 2e-3 budget.  Every wait is bounded (2 s);
-// a timeout sets the error word and an abort flag, and TMEM is released
-// only after the MMA thread's last commit.
+//       rescaled maximum (only when it grows by more than 2^4; the two threads
+//       of a row share their maxima through shared memory), W = p A_V / R_V
+//       with p = 2^(z - m - 2): the keys near the maximum get p in [1/4, 4],
+//       so their weights stay in fp16's normal range for |A_V| / R_V from
+//       2.4e-4 to 16376 (the row sum takes the same factor, which cancels in
+//       O / l);
+//   O += W B_V  (B_V MN-major).
+// Every wait is bounded (2 s); a timeout sets the error word and an abort
+// flag, and TMEM is released only after the MMA thread's last commit.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include <mutex>
@@ -87,10 +100,13 @@ static_assert(kStageBytes % 1024 == 0 && kBBox % 1024 == 0, "swizzle atoms stay 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256, kColQ = 384;
 constexpr unsigned kErrTimeout = 0x8u;
+constexpr float kLazy = 4.f;  // rescale only when a row maximum grows by more than 2^4
+constexpr float kShift = 2.f;  // p = 2^(z - m - kShift): at most 2^(kLazy - kShift) = 4
+constexpr int kMaxRq = 8;
 
-// kind::f16 instruction descriptors, D fp32, A (TMEM) and B bf16, M = 128, N = 128;
+// kind::f16 instruction descriptors, D fp32, A (TMEM) and B fp16, M = 128, N = 128;
 // the value MMA's B (the B_V tile) is MN-major.
-constexpr uint32_t kIdescScore = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescScore = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescValue = kIdescScore | (1u << 16);
 
 struct PrefillTcParams {
@@ -98,10 +114,79 @@ struct PrefillTcParams {
   int batch, capacity, n_tokens, n_qtiles;
   float zs;       // scale * log2(e) / R_K
   float inv_rv;   // 1 / R_V
-  const float* q;  // [B][T][32][128] fp32 rotated queries
+  int r_q;
+  float inv_rq;                // 1 / R_Q
+  const __nv_bfloat16* a_q;    // [B][T][R_Q][32]
+  const __half* bq_rot;        // [B][T][R_Q][128] rank rows rotated at their positions (the pre-pass)
   float* out;      // [B][T][32][128]
   unsigned int* err;
 };
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_f16(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
+struct PrepParams {
+  const int32_t* seq_lens;
+  int batch, capacity, r, n_tokens, r_q;
+  const __nv_bfloat16* b_k;   // the cache planes
+  const __nv_bfloat16* b_v;
+  const __nv_bfloat16* b_q;   // [B][T][R_Q][128], unrotated
+  const int32_t* q_pos;       // [B][T]
+  __half* wk;                 // fp16 copies [B][cap][R][128]
+  __half* wv;
+  __half* wq;                 // [B][T][R_Q][128] rotated
+  RopeTable rope;
+};
+
+// The pre-pass.  blockIdx.z = 0, 1: fp16 copies of the B_K, B_V rows of every sequence's
+// cached tokens (slots below seq_lens[b]), blockIdx.y striding over the sequences; z = 2: the
+// chunk's B_Q rank rows rotated at their positions (one thread per (query, pair): the pair's
+// cos and sin are formed once for all ranks), rounded to fp16.
+__global__ void __launch_bounds__(256) prefill_prep_kernel(const __grid_constant__ PrepParams p) {
+  ptx::pdl_launch_dependents();  // the attention grid may start its set-up
+  if (blockIdx.z < 2) {
+    for (int b = blockIdx.y; b < p.batch; b += gridDim.y) {
+      const int len = min(max(p.seq_lens[b], 0), p.capacity);
+      const size_t base = static_cast<size_t>(b) * p.capacity * p.r * kD;
+      const uint4* src = reinterpret_cast<const uint4*>((blockIdx.z == 0 ? p.b_k : p.b_v) + base);
+      uint4* dst = reinterpret_cast<uint4*>((blockIdx.z == 0 ? p.wk : p.wv) + base);
+      const size_t nvec = static_cast<size_t>(len) * p.r * kD / 8;
+      for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
+           v += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const uint4 x = src[v];
+        uint4 y;
+        y.x = pack_f16(ptx::bf16_lo(x.x), ptx::bf16_hi(x.x));
+        y.y = pack_f16(ptx::bf16_lo(x.y), ptx::bf16_hi(x.y));
+        y.z = pack_f16(ptx::bf16_lo(x.z), ptx::bf16_hi(x.z));
+        y.w = pack_f16(ptx::bf16_lo(x.w), ptx::bf16_hi(x.w));
+        dst[v] = y;
+      }
+    }
+    return;
+  }
+  const size_t n = static_cast<size_t>(p.batch) * p.n_tokens * (kD / 2);
+  const size_t stride = static_cast<size_t>(gridDim.x) * gridDim.y * blockDim.x;
+  for (size_t e = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; e < n;
+       e += stride) {
+    const size_t qrow = e / (kD / 2);  // b * T + t
+    const int pr = static_cast<int>(e % (kD / 2));
+    float c, sn;
+    rope_cos_sin(p.q_pos[qrow], p.rope.theta[pr], &c, &sn);
+    for (int j = 0; j < p.r_q; ++j) {
+      const size_t off = (qrow * p.r_q + j) * kD / 2 + pr;  // in pairs
+      const uint32_t w = reinterpret_cast<const uint32_t*>(p.b_q)[off];
+      float x = ptx::bf16_lo(w), y = ptx::bf16_hi(w);
+      rope_pair(x, y, c, sn);
+      reinterpret_cast<uint32_t*>(p.wq)[off] = pack_f16(x, y);
+    }
+  }
+}
 
 template <int R>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -179,6 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_bv);
       ptx::prefetch_tmap(&tm_ak);
       ptx::prefetch_tmap(&tm_av);
+      ptx::pdl_wait();  // the fp16 copies of B_K and B_V
       int issued = 0;
       bool ok = true;
       for (int j = 0; j < nk; ++j) {
@@ -216,13 +302,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto score = [&](int j) {
         const uint32_t sb = sbase + kOffStages + (j % kStages) * kStageBytes;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {  // query hi, then query lo
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {         // K = 128 features in steps of 16
-            const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBBox + (k & 3) * 32, 16, 1024);
-            ptx::umma_ts(tbase + 128u * (j & 1), tbase + kColQ + half * 64 + k * 8, db, kIdescScore,
-                         (half > 0 || k > 0) ? 1u : 0u);
-          }
+        for (int k = 0; k < 8; ++k) {  // K = 128 features in steps of 16
+          const uint64_t db = ptx::umma_desc_sw128(sb + (k >> 2) * kBBox + (k & 3) * 32, 16, 1024);
+          ptx::umma_ts(tbase + 128u * (j & 1), tbase + kColQ + k * 8, db, kIdescScore, k > 0 ? 1u : 0u);
         }
         ptx::umma_commit(sfull(j & 1));
       };
@@ -248,13 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t bv = sbase + kOffStages + (j % kStages) * kStageBytes + kBBytes;
         const uint32_t ts = tbase + 128u * (j & 1);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {    // W hi, then W lo
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {        // K = 128 cache rows in steps of 16
-            const uint64_t db = ptx::umma_desc_sw128(bv + kk * 2048, kBBox, 1024);
-            ptx::umma_ts(tbase + kColO, ts + half * 64 + kk * 8, db, kIdescValue,
-                         (j > 0 || half > 0 || kk > 0) ? 1u : 0u);
-          }
+        for (int kk = 0; kk < 8; ++kk) {  // K = 128 cache rows in steps of 16
+          const uint64_t db = ptx::umma_desc_sw128(bv + kk * 2048, kBBox, 1024);
+          ptx::umma_ts(tbase + kColO, ts + kk * 8, db, kIdescValue, (j > 0 || kk > 0) ? 1u : 0u);
         }
         ptx::umma_commit(odone);
         ptx::umma_commit(empty(j % kStages));
@@ -323,23 +401,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;          // query row within the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const int tq = q0 + row;                   // query index in the chunk
-    const int qslot = P + tq;                  // its cache slot: keys s <= qslot
+    const int qslot = min(P + tq, len - 1);    // its cache slot: keys s <= qslot (a padding row: the cached ones)
     const uint32_t pair_bar = 1 + quad;        // named barrier of warps (quad, half 0) and (quad, half 1)
-    // stage features [64 hf, +64) of this thread's query row as bf16 hi + lo in TMEM
+    // features [64 hf, +64) of this thread's query row, q = (1/R_Q) sum_j A_Q[t, j, head] B~_Q[t, j]
+    // from the rotated rank rows of the pre-pass (read after the wait on it), formed in fp32 and
+    // rounded once to fp16 in TMEM
     {
-      const float* qr = p.q + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD + 64 * hf;
-      uint32_t hi[32], lo[32];
+      const size_t qrow = static_cast<size_t>(b) * p.n_tokens + tq;
+      const bool real = tq < p.n_tokens;
+      float aq[kMaxRq];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (tq < p.n_tokens) v = *reinterpret_cast<const float4*>(qr + 4 * c);
-        hi[2 * c] = ptx::pack_bf16(v.x, v.y);
-        hi[2 * c + 1] = ptx::pack_bf16(v.z, v.w);
-        lo[2 * c] = ptx::pack_bf16(v.x - ptx::bf16_lo(hi[2 * c]), v.y - ptx::bf16_hi(hi[2 * c]));
-        lo[2 * c + 1] = ptx::pack_bf16(v.z - ptx::bf16_lo(hi[2 * c + 1]), v.w - ptx::bf16_hi(hi[2 * c + 1]));
+      for (int j = 0; j < kMaxRq; ++j)
+        aq[j] = (real && j < p.r_q) ? __bfloat162float(p.a_q[(qrow * p.r_q + j) * kH + head]) * p.inv_rq : 0.f;
+      ptx::pdl_wait();  // the rotated rank rows
+      float acc[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < kMaxRq; ++j) {
+        if (real && j < p.r_q) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.bq_rot + (qrow * p.r_q + j) * kD + 64 * hf);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 v = src[c];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 f = unpack_f16(w[k]);
+              acc[8 * c + 2 * k] = fmaf(aq[j], f.x, acc[8 * c + 2 * k]);
+              acc[8 * c + 2 * k + 1] = fmaf(aq[j], f.y, acc[8 * c + 2 * k + 1]);
+            }
+          }
+        }
       }
-      ptx::tmem_st32(tbase + lane_off + kColQ + 32 * hf, hi);
-      ptx::tmem_st32(tbase + lane_off + kColQ + 64 + 32 * hf, lo);
+      uint32_t qh[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) qh[k] = pack_f16(acc[2 * k], acc[2 * k + 1]);
+      ptx::tmem_st32(tbase + lane_off + kColQ + 32 * hf, qh);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -403,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mx = fmaxf(mx, mxbuf[(1 - hf) * kQ + row]);
       // ---- online softmax with a lazily rescaled maximum; both threads of a row take the same
       // decision, and the warp-wide TMEM rescale of O runs when any row of the warp needs it
-      const bool grow = mx > m + 8.f || (m == -INFINITY && mx != -INFINITY);
+      const bool grow = mx > m + kLazy || (m == -INFINITY && mx != -INFINITY);
       const float alpha = !grow ? 1.f : (m == -INFINITY ? 0.f : ptx::ex2(m - mx));
       if (grow) {
         l *= alpha;
@@ -430,8 +528,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           *s_abort = 1;
         }
       }
-      // ---- W = p A_V / R_V as bf16 hi + lo, two cache rows per TMEM column, over S
-      uint32_t whi[32], wlo[32];
+      // ---- W = p A_V / R_V as fp16, two cache rows per TMEM column, over S; p = 2^(z - m - 2) <= 4
+      // (every z <= m + 4 here): the weights near the maximum keep fp16's full precision
+      const float mref = m + kShift;
+      uint32_t wh[32];
 #pragma unroll
       for (int e4 = 0; e4 < 16; ++e4) {
         const float4 a4 = reinterpret_cast<const float4*>(av)[e4];
@@ -440,19 +540,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int u = 0; u < 4; u += R) {
           const int s = (4 * e4 + u) / R;
-          const float pz = ptx::ex2(z[s] - m);  // 0 for masked keys (z = -inf, m finite)
+          const float pz = ptx::ex2(z[s] - mref);  // 0 for masked keys (z = -inf, m finite)
           l += pz;
 #pragma unroll
           for (int r = 0; r < R; ++r) w[u + r] = pz * a[u + r];
         }
-        whi[2 * e4] = ptx::pack_bf16(w[0], w[1]);
-        whi[2 * e4 + 1] = ptx::pack_bf16(w[2], w[3]);
-        wlo[2 * e4] = ptx::pack_bf16(w[0] - ptx::bf16_lo(whi[2 * e4]), w[1] - ptx::bf16_hi(whi[2 * e4]));
-        wlo[2 * e4 + 1] =
-            ptx::pack_bf16(w[2] - ptx::bf16_lo(whi[2 * e4 + 1]), w[3] - ptx::bf16_hi(whi[2 * e4 + 1]));
+        wh[2 * e4] = pack_f16(w[0], w[1]);
+        wh[2 * e4 + 1] = pack_f16(w[2], w[3]);
       }
-      ptx::tmem_st32(ts + 32 * hf, whi);
-      ptx::tmem_st32(ts + 64 + 32 * hf, wlo);
+      ptx::tmem_st32(ts + 32 * hf, wh);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
@@ -522,54 +618,103 @@ size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 
 bool tensor_prefill_supported(int dtype, int heads, int head_dim, int r_k, int r_v, int r_q) {
   return dtype == TPA_BF16 && heads == kH && head_dim == kD && r_k == r_v && (r_k == 1 || r_k == 2) && r_q >= 1 &&
-         r_q <= 8;
+         r_q <= kMaxRq;
 }
 
-size_t tensor_prefill_workspace_bytes(int batch, int n_tokens, int heads, int head_dim) {
-  return round256(static_cast<size_t>(batch) * heads * n_tokens * head_dim * 4);  // fp32 rotated queries
+namespace {
+
+// The workspace: fp16 copies of B_K and B_V [B][cap][R][128], then the rotated rank rows
+// [B][T][R_Q][128] (fp16), each section 256-byte aligned.
+struct PrefillWorkspace {
+  __half* wk;
+  __half* wv;
+  __half* wq;
+  size_t bytes;
+};
+
+PrefillWorkspace carve_prefill(void* base, int batch, int capacity, int r, int n_tokens, int r_q) {
+  const size_t plane = round256(static_cast<size_t>(batch) * capacity * r * kD * 2);
+  const size_t qb = round256(static_cast<size_t>(batch) * n_tokens * r_q * kD * 2);
+  char* c = static_cast<char*>(base);
+  PrefillWorkspace w;
+  w.wk = reinterpret_cast<__half*>(c);
+  w.wv = reinterpret_cast<__half*>(c ? c + plane : nullptr);
+  w.wq = reinterpret_cast<__half*>(c ? c + 2 * plane : nullptr);
+  w.bytes = 2 * plane + qb;
+  return w;
+}
+
+}  // namespace
+
+size_t tensor_prefill_workspace_bytes(int batch, int capacity, int r, int n_tokens, int r_q) {
+  return carve_prefill(nullptr, batch, capacity, r, n_tokens, r_q).bytes;
 }
 
 cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t stream) {
   const CacheView& cv = a.cache;
   const int T = a.n_tokens;
-  float* qws = static_cast<float*>(a.workspace);
-  PrefillQArgs qa;
-  qa.batch = cv.batch;
-  qa.n_tokens = T;
-  qa.heads = cv.heads;
-  qa.head_dim = cv.head_dim;
-  qa.r_q = a.r_q;
-  qa.dtype = cv.dtype;
-  qa.a_q = a.a_q;
-  qa.b_q = a.b_q;
-  qa.q_pos = a.q_pos;
-  qa.q_out = qws;
-  qa.rope = a.rope;
-  cudaError_t e = launch_prefill_q(qa, stream);
+  const int R = cv.r_k;
+  const PrefillWorkspace ws = carve_prefill(a.workspace, cv.batch, cv.capacity, R, T, a.r_q);
+  PrepParams pp;
+  pp.seq_lens = cv.seq_lens;
+  pp.batch = cv.batch;
+  pp.capacity = cv.capacity;
+  pp.r = R;
+  pp.n_tokens = T;
+  pp.r_q = a.r_q;
+  pp.b_k = static_cast<const __nv_bfloat16*>(cv.b_k);
+  pp.b_v = static_cast<const __nv_bfloat16*>(cv.b_v);
+  pp.b_q = static_cast<const __nv_bfloat16*>(a.b_q);
+  pp.q_pos = a.q_pos;
+  pp.wk = ws.wk;
+  pp.wv = ws.wv;
+  pp.wq = ws.wq;
+  pp.rope = a.rope;
+  // about four CTAs per SM over the three parts
+  const int sms = a.sms > 0 ? a.sms : 148;
+  const int gy = min(cv.batch, 65535);
+  const size_t vec_per_seq = static_cast<size_t>(cv.capacity) * R * kD / 8;
+  size_t gx = (vec_per_seq + 255) / 256;
+  const size_t cap_x = static_cast<size_t>(max(1, 4 * sms / max(1, 3 * gy)));
+  if (gx > cap_x) gx = cap_x;
+  if (gx < 1) gx = 1;
+  prefill_prep_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 3), 256, 0, stream>>>(pp);
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const uint64_t rows_k = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_k;
-  const uint64_t rows_v = static_cast<uint64_t>(cv.batch) * cv.capacity * cv.r_v;
+  const uint64_t rows = static_cast<uint64_t>(cv.batch) * cv.capacity * R;
   CUtensorMap tbk, tbv, tak, tav;
-  if ((e = encode_bf16_2d(&tbk, cv.b_k, kD, rows_k, 64, kRows, 128)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tbv, cv.b_v, kD, rows_v, 64, kRows, 128)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows_k, kASlice, kRows, 0)) != cudaSuccess) return e;
-  if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows_v, kASlice, kRows, 0)) != cudaSuccess) return e;
-  if ((e = set_smem_once(cv.r_k)) != cudaSuccess) return e;
+  // the fp16 copies move as plain 2-byte elements
+  if ((e = encode_bf16_2d(&tbk, ws.wk, kD, rows, 64, kRows, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tbv, ws.wv, kD, rows, 64, kRows, 128)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tak, cv.a_k, kH, rows, kASlice, kRows, 0)) != cudaSuccess) return e;
+  if ((e = encode_bf16_2d(&tav, cv.a_v, kH, rows, kASlice, kRows, 0)) != cudaSuccess) return e;
+  if ((e = set_smem_once(R)) != cudaSuccess) return e;
   PrefillTcParams p;
   p.seq_lens = cv.seq_lens;
   p.batch = cv.batch;
   p.capacity = cv.capacity;
   p.n_tokens = T;
   p.n_qtiles = (T + kQ - 1) / kQ;
-  p.zs = a.scale * kLog2e / static_cast<float>(cv.r_k);
+  p.zs = a.scale * kLog2e / static_cast<float>(R);
   p.inv_rv = 1.f / static_cast<float>(cv.r_v);
-  p.q = qws;
+  p.r_q = a.r_q;
+  p.inv_rq = 1.f / static_cast<float>(a.r_q);
+  p.a_q = static_cast<const __nv_bfloat16*>(a.a_q);
+  p.bq_rot = ws.wq;
   p.out = a.out;
   p.err = a.err;
-  dim3 grid(cv.batch * kH, p.n_qtiles);
-  auto kern = cv.r_k == 1 ? prefill_tc_kernel<1> : prefill_tc_kernel<2>;
-  kern<<<grid, kThreads, kSmemBytes, stream>>>(p, tbk, tbv, tak, tav);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cv.batch * kH, p.n_qtiles);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto kern = R == 1 ? prefill_tc_kernel<1> : prefill_tc_kernel<2>;
+  return cudaLaunchKernelEx(&cfg, kern, p, tbk, tbv, tak, tav);
 }
 
 }  // namespace tpa

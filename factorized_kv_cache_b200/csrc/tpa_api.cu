@@ -564,7 +564,7 @@ size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int3
   if (check_cache(cache) != TPA_OK || n_tokens < 0 || r_q < 1 || r_q > 8) return 0;
   if (kernel != TPA_KERNEL_SIMT &&
       tensor_prefill_supported(cache->dtype, cache->heads, cache->head_dim, cache->r_k, cache->r_v, r_q))
-    return tensor_prefill_workspace_bytes(cache->batch, n_tokens, cache->heads, cache->head_dim);
+    return tensor_prefill_workspace_bytes(cache->batch, cache->capacity, cache->r_k, n_tokens, r_q);
   return round256(static_cast<size_t>(cache->batch) * n_tokens * cache->heads * cache->head_dim * sizeof(float));
 }
 

@@ -51,7 +51,8 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
 
 // ---- causal prefill (bf16, h = 32, d_h = 128, R_K == R_V in {1, 2}, R_Q <= 8)
 bool tensor_prefill_supported(int dtype, int heads, int head_dim, int r_k, int r_v, int r_q);
-size_t tensor_prefill_workspace_bytes(int batch, int n_tokens, int heads, int head_dim);
+// fp16 copies of the cache's B_K and B_V planes and of the chunk's rotated B_Q rank rows
+size_t tensor_prefill_workspace_bytes(int batch, int capacity, int r, int n_tokens, int r_q);
 
 struct TensorPrefillArgs {
   CacheView cache;

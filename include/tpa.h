@@ -349,7 +349,13 @@ tpa_status tpa_decode_attention_noalloc(const tpa_cache* cache, const void* q, c
                                         float scale, float* out, int32_t max_len, int32_t num_splits,
                                         int32_t kernel, void* stream);
 
-/* Workspace bytes tpa_prefill_attention needs. */
+/* Workspace bytes tpa_prefill_attention needs: on the tensor-core path, fp16
+ * copies of the cache's B_K and B_V planes (2 * batch * capacity * r_k *
+ * head_dim * 2 bytes) and the chunk's B_Q rank rows rotated at their
+ * positions (batch * n_tokens * r_q * head_dim * 2 bytes; the dense
+ * per-head queries are formed inside the kernel and never stored); on the
+ * CUDA-core path, the dense rotated fp32 queries (batch * n_tokens * heads *
+ * head_dim * 4 bytes). */
 size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q,
                                   int32_t kernel);
 
@@ -363,6 +369,13 @@ size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int3
  *   query t, head i: q = (1/r_q) sum_j A_Q[t][j][i] RoPE(B_Q[t][j], q_pos[t]);
  *   out [batch][n_tokens][heads][head_dim] float32, device.
  *   workspace: device, >= tpa_prefill_workspace_size(...) bytes, 256-byte aligned.
+ * The tensor-core path (bf16, heads 32, head_dim 128, r_k == r_v <= 2)
+ * multiplies in fp16 with fp32 accumulation: the cache's B_K and B_V rows
+ * are copied to fp16 (exact for magnitudes up to fp16's 65504; larger
+ * values are outside this path and give non-finite outputs), the rotated
+ * B_Q rank rows, the queries formed from them and the softmax weights are
+ * rounded once each to fp16 (about 4e-4 relative each on unit-variance
+ * factors).
  * Errors: NULL, SHAPE (n_tokens < 0 or > capacity), UNSUPPORTED, WORKSPACE,
  * ALIGNMENT, CUDA.  n_tokens > seq_lens[b] sets TPA_DEVERR_PREFILL_LEN and
  * leaves out[b] untouched.

@@ -109,7 +109,9 @@ def test_prefill_workload_full_size(kernel):
 def test_last_prefill_row_equals_factored_decode(tokens, prior):
     """Two kernels, one quantity: the prefill's last query row (slot L - 1, attending slots
     0 .. L - 1) is the decode of a query in TPA form (A_Q, B_Q of that token, at position L - 1)
-    over the same cache."""
+    over the same cache.  The decode keeps ~16 bits of its query and weights (bf16 high + low
+    parts), the tensor-core prefill rounds both once to fp16 (11 bits, ~4e-4 relative each), so
+    the two agree to the prefill's own error, well inside the 2e-3 parity budget."""
     w = S.WORKLOADS["prefill_b4_t4k"]
     cache, x, a_q, b_q, q_pos = _prefill_case(w, 2, tokens, prior)
     out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos)
@@ -117,4 +119,4 @@ def test_last_prefill_row_equals_factored_decode(tokens, prior):
     dec = T.tpa_decode_attention_factored(cache, a_q[:, -1].contiguous(), b_q[:, -1].contiguous(),
                                           q_pos[:, -1].contiguous(), max_len=L)
     assert T.tpa_read_device_error() == 0
-    assert_rows_close(f64(dec), f64(out[:, -1]), 2e-4, "prefill last row vs factored decode")
+    assert_rows_close(f64(dec), f64(out[:, -1]), 1.5e-3, "prefill last row vs factored decode")
