@@ -108,27 +108,48 @@ def test_length_above_max_len_is_reported():
     assert T.tpa_read_device_error() & T.TPA_DEVERR_LEN_RANGE
 
 
+_E2E_REFS = {}
+
+
+def _end_to_end_all_heads(w, x, b, got, kernel):
+    """Sequence b on all heads, end to end: the oracle rotates the unrotated factors itself
+    (RoPE at each token's position, the stored rows rounded to the cache dtype) and attends
+    with its own query RoPE.  The float64 reference is computed once per workload and reused
+    by every kernel."""
+    key = (w.name, b)
+    if key not in _E2E_REFS:
+        L = int(x["lengths"][b])
+        _E2E_REFS[key] = O.decode_attention_from_unrotated(
+            f64(x["a_k"][b, :L]), f64(x["b_k"][b, :L]), f64(x["a_v"][b, :L]), f64(x["b_v"][b, :L]), np.arange(L),
+            f64(x["q"][b]), float(x["q_pos"][b]), default_scale(w.head_dim), w.rope_base, storage=w.dtype)
+    assert_rows_close(f64(got[b]), _E2E_REFS[key], TOL[torch.bfloat16], f"{w.name} end-to-end b={b} kernel={kernel}")
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_b32_var32k_workload_full_size(kernel):
-    """The full R=2 variable-length workload; oracle on 4 sequences x 4 heads."""
+    """The full R=2 variable-length workload; oracle on 4 sequences x 4 heads at cache level,
+    and the longest sequence end to end on all 32 heads."""
     w = S.WORKLOADS["decode_b32_var32k"]
     cache, x, q, q_pos = build_decode_cache(w, nan_tail=False)
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
     L = x["lengths"].numpy()
     picks = [int(np.argmin(L)), int(np.argmax(L)), 7, 19]
     _check(w, cache, x, q, q_pos, out, batches=picks, heads=[0, 11, 22, 31], end_to_end=False)
+    _end_to_end_all_heads(w, x, int(np.argmax(L)), out, kernel)
     assert T.tpa_read_device_error() == 0
 
 
 @pytest.mark.slow
 @pytest.mark.parametrize("kernel", KERNELS)
 def test_long_512k_workload_full_size(kernel):
-    """The long-context workload (B=1, L=524288); oracle on 3 heads."""
+    """The long-context workload (B=1, L=524288); oracle on 3 heads at cache level, and end to
+    end on all 32 heads."""
     w = S.WORKLOADS["decode_long_512k"]
     cache, x, q, q_pos = build_decode_cache(w, nan_tail=False)
     out = T.tpa_decode_attention(cache, q, q_pos, max_len=w.length, kernel=kernel)
     _check(w, cache, x, q, q_pos, out, heads=[0, 17, 31], end_to_end=False)
+    _end_to_end_all_heads(w, x, 0, out, kernel)
     assert T.tpa_read_device_error() == 0
 
 

@@ -1,6 +1,7 @@
 """GPU parity of tpa_decode_step (append the generated token and attend with its
 query, fused) against the oracle's decode_step, and against the two-call path
 (tpa_cache_append, then tpa_decode_attention) for what the cache holds."""
+import ctypes
 import numpy as np
 import pytest
 import torch
@@ -400,3 +401,21 @@ def test_plan_stages_its_inputs_from_pinned_host_memory():
     with pytest.raises(ValueError):
         T.DecodeStepPlan(cache, views["q_pos"], views["a_k"], views["b_k"], views["a_v"], views["b_v"], out,
                          q=views["q"], stage=(torch.zeros(off, dtype=torch.uint8), dev_in))   # pageable host memory
+    # the C entry point checks the copy's ends itself (a C caller has no binding to check them):
+    # pageable host memory as the source, or host memory as the destination, is refused
+    lib = T.load_library()
+    c = cache.struct()
+    pageable = torch.zeros(off, dtype=torch.uint8)
+
+    nws = int(lib.tpa_decode_workspace_size(ctypes.byref(c), 1000, 0, 0))
+    ws = T.workspace(nws, DEV)
+
+    def c_init(dst, src):
+        p = T.tpa_step_plan()
+        return lib.tpa_step_plan_init(ctypes.byref(p), ctypes.byref(c), T._ptr(views["q_pos"]), T._ptr(views["a_k"]),
+                                      T._ptr(views["b_k"]), T._ptr(views["a_v"]), T._ptr(views["b_v"]), 0, None,
+                                      T._ptr(views["q"]), 0.1, T._ptr(out), 1000, 1, 0, 0, T._ptr(ws), nws,
+                                      T._ptr(dst), T._ptr(src), off)
+    assert c_init(dev_in, pageable) == 3      # TPA_ERR_UNSUPPORTED
+    assert c_init(host_in, host_in) == 3
+    assert c_init(dev_in, host_in) == T.TPA_OK
