@@ -523,6 +523,7 @@ struct TcStepParams {
 
 struct TcMergeParams {
   int batch, grid;
+  int setup;               // set-up units before each non-empty sequence's tiles (the split kernel's)
   const int32_t* prefix;
   const float* ws_ml;
   const float* ws_o;
@@ -698,7 +699,9 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     write_lse(nv ? zn : 0.f, nv ? 1.f : 0.f);
     return;
   }
-  const int cs = owner_of(t0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
+  const int setup = p.setup > 0 ? p.prefix[p.batch + 1] : 0;  // the set-up units the split kernel charged
+  const int w0 = t0 + setup;  // the sequence's first tile unit (it is not empty here)
+  const int cs = owner_of(w0, NT, p.grid), ce = owner_of(t1 - 1, NT, p.grid);
   if (cs == ce) {  // finished by the split kernel
     if (nv || lse) {
       const float2 ml = reinterpret_cast<const float2*>(p.whole_ml)[static_cast<size_t>(b) * kH + i];
@@ -723,7 +726,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     const int cc = cs + u;
     if (dense) return (2 * cc + ((u > 0 || cs_first) ? 0 : 1)) * kH + i;
     const int a = dec::first_tile(cc, NT, p.grid), e = dec::first_tile(cc + 1, NT, p.grid);
-    if (!(a < e && a < t1 && e > t0)) return -1;
+    if (!(a < e && a < t1 && e > w0)) return -1;
     return (2 * cc + (a >= t0 ? 0 : 1)) * kH + i;
   };
   float L = 0.f;
@@ -876,12 +879,12 @@ struct TcWorkspace {
   size_t bytes;
 };
 
-// [prefix: B + 1 int32][ml: 2G x 32 x 2 f32][o: 2G x 32 x 128 f32][len: B int32][step ml: B x 32 x 2 f32],
+// [prefix: B + 2 int32 (the tile prefix, then the set-up units charged)][ml: 2G x 32 x 2 f32][o: 2G x 32 x 128 f32][len: B int32][step ml: B x 32 x 2 f32],
 // each section 256-byte aligned.
 TcWorkspace carve(void* base, int batch, int grid) {
   TcWorkspace w;
   const size_t slots = 2 * static_cast<size_t>(grid);
-  const size_t pb = round256((static_cast<size_t>(batch) + 1) * 4);
+  const size_t pb = round256((static_cast<size_t>(batch) + 2) * 4);
   const size_t mlb = round256(slots * kH * 2 * 4);
   const size_t ob = round256(slots * kH * kD * 4);
   const size_t lb = round256(static_cast<size_t>(batch) * 4);
@@ -937,6 +940,9 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   p.whole_ml = (a.step || a.lse) ? ws.step_ml : nullptr;
   p.err = a.err;
   p.rope = a.rope;
+  // a sequence's query stage costs a tcgen05 CTA about one tile of streaming; the warp-level
+  // kernel's partition counts tiles only
+  p.setup = a.variant == kDecodeUmma ? 1 : 0;
   if (a.variant == kDecodeUmma) {
     e = launch_decode_umma(p, cv, stream);
   } else {
@@ -956,6 +962,7 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   TcMergeParams mp;
   mp.batch = cv.batch;
   mp.grid = a.grid;
+  mp.setup = p.setup;
   mp.prefix = ws.prefix;
   mp.ws_ml = ws.ml;
   mp.ws_o = ws.o;

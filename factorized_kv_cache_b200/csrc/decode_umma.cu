@@ -177,6 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (sbase - raw);
   float* s_red = reinterpret_cast<float*>(gbase + kOffRed);
   float* s_cs = reinterpret_cast<float*>(gbase + kOffCs);
+  // a query in TPA form: its raw rank rows [r_q][128] bf16 and A_Q / R_Q [r_q][32] staged in the W
+  // buffers, which are idle whenever a sequence segment starts
+  __nv_bfloat16* s_bqr = reinterpret_cast<__nv_bfloat16*>(gbase + kOffW);
+  float* s_aq = reinterpret_cast<float*>(gbase + kOffW + 8 * kD * 2);
   const uint32_t bar0 = sbase + kOffBar;
   auto kfull = [&](int s) { return bar0 + 8 * s; };
   auto kempty = [&](int s) { return bar0 + 8 * (2 + s); };
@@ -232,11 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (it waits for this grid before it reads anything written here).
   ptx::pdl_launch_dependents();
 
-  dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
+  const int setup = dec::build_prefix<TOK, kThreads>(p, s_pref, s_len, s_tmp);  // ends with __syncthreads
   const int B = p.batch;
   const int NT = s_pref[B];
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
     for (int b = tid; b <= B; b += kThreads) p.ws_prefix[b] = s_pref[b];
+    if (tid == 0) p.ws_prefix[B + 1] = setup;  // for the merge
+  }
   const int c = blockIdx.x;
   const int t_begin = NT == 0 ? 0 : dec::first_tile_fast(c, NT, p.grid, p.inv_grid);
   const int t_end = NT == 0 ? 0 : dec::first_tile_fast(c + 1, NT, p.grid, p.inv_grid);
@@ -256,17 +262,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Load order K0, K1, V0, K2, V1, K3, ...: the score MMA of a tile needs only its K
     // slot, and the softmax reaches for A_V (the V slot) last.
     if (lane == 0) {
-      const int n = t_end - t_begin;
-      int kb_seq = b_first, vb_seq = b_first;  // sequence cursors of the K and V streams
-      auto row_of = [&](int j, int& cur) {
-        const int t = t_begin + j;
-        while (s_pref[cur + 1] <= t) ++cur;
-        return (cur * p.capacity + (t - s_pref[cur]) * TOK) * R;
+      // the CTA's tiles in order: units [t_begin, t_end) without the set-up units
+      int n = 0;
+      for (int b = b_first; b < B && s_pref[b] < t_end; ++b)
+        n += max(0, min(t_end, s_pref[b + 1]) - max(t_begin, dec::first_work(s_pref, b, setup)));
+      // cursors (sequence, unit) of the K and V streams: each call moves one to the next tile
+      // (units past a sequence's set-up units) and returns the tile's first cache row
+      int k_seq = b_first, k_unit = t_begin - 1, v_seq = b_first, v_unit = t_begin - 1;
+      auto next_row = [&](int& cb, int& ct) {
+        ++ct;
+        while (cb < B) {
+          const int w0 = dec::first_work(s_pref, cb, setup);
+          if (ct < w0) ct = w0;
+          if (ct < s_pref[cb + 1]) break;
+          ++cb;
+        }
+        return (cb * p.capacity + (ct - dec::first_work(s_pref, cb, setup)) * TOK) * R;
       };
       auto load_k = [&](int j) -> bool {
         const int s = j & 1;
         if (j >= 2 && !ptx::mbar_wait_bounded(kempty(s), ((j >> 1) & 1) ^ 1)) return false;
-        const int row0 = row_of(j, kb_seq);
+        const int row0 = next_row(k_seq, k_unit);
         const uint32_t kb = sbase + kOffK + s * kSlotBytes;
         ptx::mbar_arrive_expect_tx(kfull(s), kSlotBytes);
         ptx::tma_load_2d(kb, &tm_bk, 0, row0, kfull(s));
@@ -277,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_v = [&](int j) -> bool {
         const int s = j & 1;
         if (j >= 2 && !ptx::mbar_wait_bounded(vempty(s), ((j >> 1) & 1) ^ 1)) return false;
-        const int row0 = row_of(j, vb_seq);
+        const int row0 = next_row(v_seq, v_unit);
         const uint32_t vb = sbase + kOffV + s * kSlotBytes;
         ptx::mbar_arrive_expect_tx(vfull(s), kSlotBytes);
         ptx::tma_load_2d(vb, &tm_bv, 0, row0, vfull(s));
@@ -334,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0, seg = 0, pend = -1;
       bool pend_first = false, ok = true;
       for (int b = b_first; b < B && s_pref[b] < t_end && ok; ++b) {
-        const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
+        const int ta = max(t_begin, dec::first_work(s_pref, b, setup)), tb = min(t_end, s_pref[b + 1]);
         if (ta >= tb) continue;
         for (int t = ta; t < tb; ++t, ++it) {
           if (*s_abort) {
@@ -386,100 +402,85 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool aborted = false;
     for (int b = b_first; b < B && s_pref[b] < t_end; ++b) {
-      const int ta = max(t_begin, s_pref[b]), tb = min(t_end, s_pref[b + 1]);
+      const int w0 = dec::first_work(s_pref, b, setup);
+      const int ta = max(t_begin, w0), tb = min(t_end, s_pref[b + 1]);
       if (ta >= tb) continue;
       const int len_b = s_len[b];
       // ---- rotated query as bf16 hi (rows 0..31) and lo (rows 32..63), K-major, 128-byte swizzle.
       // This thread's 16 features of one head and the position are loaded together, first.  A
-      // factorized query (section 解决思路: q = (1/R_Q) A_Q^T B_Q) is formed here in fp32 from
-      // its rotated rank rows.
+      // factorized query (section 解决思路: q = (1/R_Q) A_Q^T B_Q, RoPE on the B factor) is
+      // combined from its unrotated rank rows in fp32 first and rotated once after, as a dense
+      // query is: RoPE is linear, so RoPE((1/R_Q) sum_j A_Q[j] B_Q[j]) equals
+      // (1/R_Q) sum_j A_Q[j] RoPE(B_Q[j]) (the same rounding count, in another order).
       {
         const int head = wt >> 3, f0 = (wt & 7) * 16;
         uint32_t hi[8], lo[8];
+        float qf[16];
+        uint4 qv[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};  // a dense query, raw until after the barrier
         if (p.r_q == 0) {
           const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
                                                             (static_cast<size_t>(b) * kH + head) * kD + f0);
-          const uint4 qv[2] = {src[0], src[1]};
-          if (wt < kD / 2) {
-            float cs, sn;
-            rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
-            s_cs[2 * wt] = cs;
-            s_cs[2 * wt + 1] = sn;
-          }
-          ptx::named_barrier(1, kSoftmaxThreads);
+          qv[0] = src[0];
+          qv[1] = src[1];
+        } else {
+          // the rank rows are shared by all heads: each is loaded once, by 16 threads, as raw bf16
+          // into the (idle) W buffers, A_Q / R_Q beside them
+          const int jr = wt >> 4, c8 = (wt & 15) * 8;  // rank row, first feature of 8
+          if (jr < p.r_q)
+            reinterpret_cast<uint4*>(s_bqr + jr * kD)[c8 / 8] = *reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.r_q + jr) * kD + c8);
+          const int ja = wt >> 5;                       // A_Q: rank row ja, head (wt & 31)
+          if (ja < p.r_q)
+            s_aq[ja * kH + (wt & 31)] =
+                __bfloat162float(static_cast<const __nv_bfloat16*>(p.a_q)[(static_cast<size_t>(b) * p.r_q + ja) * kH +
+                                                                          (wt & 31)]) * p.inv_rq;
+        }
+        if (wt < kD / 2) {
+          float cs, sn;
+          rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
+          s_cs[2 * wt] = cs;
+          s_cs[2 * wt + 1] = sn;
+        }
+        ptx::named_barrier(1, kSoftmaxThreads);
+        if (p.r_q == 0) {
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
             const uint32_t w[4] = {qv[v].x, qv[v].y, qv[v].z, qv[v].w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              const int e = 4 * v + k;
-              const int jp = f0 / 2 + e;  // RoPE pair (features 2 jp, 2 jp + 1)
-              float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
-              rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
-              hi[e] = ptx::pack_bf16(x, y);
-              lo[e] = ptx::pack_bf16(x - ptx::bf16_lo(hi[e]), y - ptx::bf16_hi(hi[e]));
+              qf[8 * v + 2 * k] = ptx::bf16_lo(w[k]);
+              qf[8 * v + 2 * k + 1] = ptx::bf16_hi(w[k]);
             }
           }
         } else {
-          // The rank rows are shared by all heads: each is loaded and rotated once, by
-          // 16 threads, into fp32 scratch in the (idle) W buffers with A_Q / R_Q beside it.
-          // rows of 128 features, each 16-feature chunk padded by 4 floats so that the eight
-          // chunks one warp reads land in distinct banks
-          constexpr int kChunk = 20, kRowF = 8 * kChunk;
-          float* s_bq = reinterpret_cast<float*>(gbase + kOffW);  // [r_q][8 chunks][20] rotated B_Q
-          float* s_aq = s_bq + 8 * kRowF;                            // [r_q][32] A_Q / R_Q
-          const int jr = wt >> 4, c8 = (wt & 15) * 8;                // rank row, first feature of 8
-          uint4 bv = make_uint4(0, 0, 0, 0);
-          if (jr < p.r_q)
-            bv = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                 (static_cast<size_t>(b) * p.r_q + jr) * kD + c8);
-          const int ja = wt >> 5;                                    // A_Q: rank row ja, head (wt & 31)
-          float av = 0.f;
-          if (ja < p.r_q)
-            av = __bfloat162float(static_cast<const __nv_bfloat16*>(p.a_q)[(static_cast<size_t>(b) * p.r_q + ja) * kH +
-                                                                           (wt & 31)]) * p.inv_rq;
-          if (wt < kD / 2) {
-            float cs, sn;
-            rope_cos_sin(p.q_pos[b], p.rope.theta[wt], &cs, &sn);
-            s_cs[2 * wt] = cs;
-            s_cs[2 * wt + 1] = sn;
-          }
-          ptx::named_barrier(1, kSoftmaxThreads);
-          if (jr < p.r_q) {
-            const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+          // this thread's 16 features of its head: (1/R_Q) sum_j A_Q[j] B_Q[j], unrotated
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int jp = c8 / 2 + k;
-              float x = ptx::bf16_lo(w[k]), y = ptx::bf16_hi(w[k]);
-              rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
-              const int f = c8 + 2 * k;
-              s_bq[jr * kRowF + (f >> 4) * kChunk + (f & 15)] = x;
-              s_bq[jr * kRowF + (f >> 4) * kChunk + (f & 15) + 1] = y;
+          for (int e = 0; e < 16; ++e) qf[e] = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (j < p.r_q) {
+              const float wq = s_aq[j * kH + head];
+              const uint4* src = reinterpret_cast<const uint4*>(s_bqr + j * kD + f0);
+#pragma unroll
+              for (int v = 0; v < 2; ++v) {
+                const uint4 rv = src[v];
+                const uint32_t w[4] = {rv.x, rv.y, rv.z, rv.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  qf[8 * v + 2 * k] = fmaf(wq, ptx::bf16_lo(w[k]), qf[8 * v + 2 * k]);
+                  qf[8 * v + 2 * k + 1] = fmaf(wq, ptx::bf16_hi(w[k]), qf[8 * v + 2 * k + 1]);
+                }
+              }
             }
           }
-          if (ja < p.r_q) s_aq[ja * kH + (wt & 31)] = av;
-          ptx::named_barrier(1, kSoftmaxThreads);
-          float acc[16];
+        }
 #pragma unroll
-          for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-#pragma unroll
-          for (int jq = 0; jq < 8; ++jq) {
-            if (jq >= p.r_q) break;
-            const float wq = s_aq[jq * kH + head];
-#pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-              const float4 v4 = reinterpret_cast<const float4*>(s_bq + jq * kRowF + (f0 >> 4) * kChunk)[e4];
-              acc[4 * e4] = fmaf(wq, v4.x, acc[4 * e4]);
-              acc[4 * e4 + 1] = fmaf(wq, v4.y, acc[4 * e4 + 1]);
-              acc[4 * e4 + 2] = fmaf(wq, v4.z, acc[4 * e4 + 2]);
-              acc[4 * e4 + 3] = fmaf(wq, v4.w, acc[4 * e4 + 3]);
-            }
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            hi[e] = ptx::pack_bf16(acc[2 * e], acc[2 * e + 1]);
-            lo[e] = ptx::pack_bf16(acc[2 * e] - ptx::bf16_lo(hi[e]), acc[2 * e + 1] - ptx::bf16_hi(hi[e]));
-          }
+        for (int e = 0; e < 8; ++e) {
+          const int jp = f0 / 2 + e;  // RoPE pair (features 2 jp, 2 jp + 1)
+          float x = qf[2 * e], y = qf[2 * e + 1];
+          rope_pair(x, y, s_cs[2 * jp], s_cs[2 * jp + 1]);
+          hi[e] = ptx::pack_bf16(x, y);
+          lo[e] = ptx::pack_bf16(x - ptx::bf16_lo(hi[e]), y - ptx::bf16_hi(hi[e]));
         }
         uint8_t* qb = gbase + kOffQ + (f0 >> 6) * kQBox;
 #pragma unroll
@@ -511,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *s_abort = 1;
         }
         ptx::tc_fence_after();
-        const int tok0 = (t - s_pref[b]) * TOK;
+        const int tok0 = (t - w0) * TOK;
         const int valid_rows = min(kRows, (len_b - tok0) * R);
         const bool valid = row < valid_rows;
         // ---- 16 scores of this row: z[i] = (S_hi + S_lo) A_K scale/R_K, log2 units
@@ -655,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tmem_ld16(tbase + lane_off + kColO + 32 + kHalf * hh, o1);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      const bool whole = dec::owner_of(s_pref[b], NT, p.grid) == dec::owner_of(s_pref[b + 1] - 1, NT, p.grid);
+      const bool whole = dec::owner_of(w0, NT, p.grid) == dec::owner_of(s_pref[b + 1] - 1, NT, p.grid);
       const int d = row;
       if (whole) {
         float* op = p.out + (static_cast<size_t>(b) * kH + kHalf * hh) * kD + d;
