@@ -55,6 +55,9 @@
 //       2.4e-4 to 16376 (the row sum takes the same factor, which cancels in
 //       O / l);
 //   O += W B_V  (B_V MN-major).
+// The softmax is the measured bound of this kernel (the tensor pipe idles most of the time), so
+// its per-tile work is trimmed: the second half of a thread's scores is loaded from TMEM while
+// the first half is weighted, and the weights use two-wide fp32 arithmetic.
 // Every wait is bounded (2 s); a timeout sets the error word and an abort
 // flag, and TMEM is released only after the MMA thread's last commit.
 #include <cuda.h>
@@ -121,6 +124,26 @@ struct PrefillTcParams {
   float* out;      // [B][T][32][128]
   unsigned int* err;
 };
+
+// Two-wide fp32 arithmetic: one instruction for both lanes of a pair.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<const uint64_t*>(&a)),
+      "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<const uint64_t*>(&a)),
+      "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(*reinterpret_cast<const uint64_t*>(&a)),
+      "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&d);
+}
 
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
@@ -460,10 +483,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!fail) {
         uint32_t sv[2][32];
         ptx::tmem_ld32(ts + kHalfRows * hf, sv[0]);
-        ptx::tmem_ld32(ts + kHalfRows * hf + 32, sv[1]);
         ptx::tmem_wait_ld();
+        ptx::tmem_ld32(ts + kHalfRows * hf + 32, sv[1]);  // in flight while the first half is used
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
+          if (c2 == 1) ptx::tmem_wait_ld();
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 a4 = reinterpret_cast<const float4*>(ak + 32 * c2)[e4];
@@ -532,22 +556,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (every z <= m + 4 here): the weights near the maximum keep fp16's full precision
       const float mref = m + kShift;
       uint32_t wh[32];
+      float2 l2 = make_float2(0.f, 0.f);  // two running partial sums, added at the end
 #pragma unroll
       for (int e4 = 0; e4 < 16; ++e4) {
         const float4 a4 = reinterpret_cast<const float4*>(av)[e4];
-        const float a[4] = {a4.x, a4.y, a4.z, a4.w};
         float w[4];
-#pragma unroll
-        for (int u = 0; u < 4; u += R) {
-          const int s = (4 * e4 + u) / R;
-          const float pz = ptx::ex2(z[s] - mref);  // 0 for masked keys (z = -inf, m finite)
-          l += pz;
-#pragma unroll
-          for (int r = 0; r < R; ++r) w[u + r] = pz * a[u + r];
+        if (R == 2) {
+          // tokens s0, s1 = rows (4 e4, +1) and (4 e4 + 2, +3): two-wide fp32 ops
+          const int s0 = 2 * e4;
+          const float2 d = sub2(make_float2(z[s0], z[s0 + 1]), make_float2(mref, mref));
+          const float2 pz = make_float2(ptx::ex2(d.x), ptx::ex2(d.y));  // 0 for masked keys
+          l2 = add2(l2, pz);
+          const float2 w01 = mul2(make_float2(pz.x, pz.x), make_float2(a4.x, a4.y));
+          const float2 w23 = mul2(make_float2(pz.y, pz.y), make_float2(a4.z, a4.w));
+          w[0] = w01.x; w[1] = w01.y; w[2] = w23.x; w[3] = w23.y;
+        } else {
+          const float2 d0 = sub2(make_float2(z[4 * e4], z[4 * e4 + 1]), make_float2(mref, mref));
+          const float2 d1 = sub2(make_float2(z[4 * e4 + 2], z[4 * e4 + 3]), make_float2(mref, mref));
+          const float2 p0 = make_float2(ptx::ex2(d0.x), ptx::ex2(d0.y));
+          const float2 p1 = make_float2(ptx::ex2(d1.x), ptx::ex2(d1.y));
+          l2 = add2(l2, add2(p0, p1));
+          const float2 w01 = mul2(p0, make_float2(a4.x, a4.y));
+          const float2 w23 = mul2(p1, make_float2(a4.z, a4.w));
+          w[0] = w01.x; w[1] = w01.y; w[2] = w23.x; w[3] = w23.y;
         }
         wh[2 * e4] = pack_f16(w[0], w[1]);
         wh[2 * e4 + 1] = pack_f16(w[2], w[3]);
       }
+      l += l2.x + l2.y;
       ptx::tmem_st32(ts + 32 * hf, wh);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
