@@ -478,10 +478,11 @@ __global__ void __maxnreg__(168)  // 168 x 32 x 3 warps fit one SM sub-partition
 // (sequence, head).  The touched CTAs of sequence b are cs..ce; when every CTA
 // owns at least one tile (G <= NT) they all touched b, b is the first sequence
 // of each of them but possibly cs, and only cs needs a division.  The (m, l)
-// pairs are reduced across the CTA; the features are then summed by eight
-// partial groups of 32 threads (one float4 column per thread), each thread
-// with kMergeBatch partial loads in flight at once, so even the ~150 partials
-// of a single long sequence take only a few L2 round trips.
+// pairs are reduced across the CTA; the features are then summed by partial
+// groups of 32 threads (one float4 column per thread), each thread with
+// kMergeBatch partial loads in flight at once: 8 groups of 4 for 256 threads,
+// and for a batch of one or two sequences (each split over ~150 CTAs) 32 groups
+// of 5, so that all of a long sequence's partials arrive in one L2 round trip.
 //
 // Decode step (kStep): the token being generated (its factors and its query,
 // section 解决思路: Q_t, K_t, V_t all come from x_t) is appended and attended
@@ -535,11 +536,14 @@ struct TcMergeParams {
 
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr int kMergeThreads = 256;
-constexpr int kMergeGroups = kMergeThreads / 32;
-constexpr int kMergeBatch = 4;
+// Threads of a merge CTA: 256 for most batches; 1024 when a batch of one or two sequences
+// spreads each over ~150 CTAs of the split kernel, so that one pass loads every partial.
+constexpr int kMergeThreadsSmallBatch = 1024;
 constexpr int kMergeMax = 1024;  // partials per pass
 
+// Block-wide max or sum over NT / 32 warps.  The warps' values meet in s_red and every warp
+// reduces them itself, so the result reaches all threads after one barrier past the write.
+template <int NT>
 __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -549,14 +553,26 @@ __device__ __forceinline__ float merge_reduce(float v, bool is_max, float* s_red
   __syncthreads();
   if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
   __syncthreads();
-  v = s_red[0];
+  if constexpr (NT <= 256) {  // a few warps: read their values in turn
+    v = s_red[0];
 #pragma unroll
-  for (int k = 1; k < kMergeThreads / 32; ++k) v = is_max ? fmaxf(v, s_red[k]) : v + s_red[k];
+    for (int k = 1; k < NT / 32; ++k) v = is_max ? fmaxf(v, s_red[k]) : v + s_red[k];
+  } else {  // up to 32 warps: one value per lane, then a shuffle tree
+    const int lane = threadIdx.x & 31;
+    v = lane < NT / 32 ? s_red[lane] : (is_max ? -INFINITY : 0.f);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float w = __shfl_xor_sync(0xffffffffu, v, o);
+      v = is_max ? fmaxf(v, w) : v + w;
+    }
+  }
   return v;
 }
 
-template <bool kStep>
+template <bool kStep, int kMergeThreads>
 __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __grid_constant__ TcMergeParams p) {
+  constexpr int kMergeGroups = kMergeThreads / 32;
+  constexpr int kMergeBatch = kMergeThreads >= 1024 ? 5 : 4;  // 32 x 5 partials in one pass
   // the next decode may start its set-up on SMs this grid frees; it waits for this grid to
   // complete before it touches memory
   ptx::pdl_launch_dependents();
@@ -747,11 +763,11 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     const int my = tid < n ? slot_of(tid) : -1;
     const float2 ml = my >= 0 ? *reinterpret_cast<const float2*>(p.ws_ml + 2 * static_cast<size_t>(my))
                               : make_float2(-INFINITY, 0.f);
-    M = merge_reduce(ml.x, true, s_red);
+    M = merge_reduce<kMergeThreads>(ml.x, true, s_red);
     if (nv) M = fmaxf(M, zn);
     const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
     if (tid < n) s_w[tid] = w;
-    L = merge_reduce(ml.y * w, false, s_red);  // ends with a barrier: s_w visible
+    L = merge_reduce<kMergeThreads>(ml.y * w, false, s_red);  // ends with a barrier: s_w visible
 #pragma unroll
     for (int k = 0; k < kMergeBatch; ++k) {
       const float wk = has[k] ? s_w[grp + kMergeGroups * k] : 0.f;
@@ -766,7 +782,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       const int sl = slot_of(u);
       if (sl >= 0) M = fmaxf(M, p.ws_ml[2 * static_cast<size_t>(sl)]);
     }
-    M = merge_reduce(M, true, s_red);
+    M = merge_reduce<kMergeThreads>(M, true, s_red);
     if (nv) M = fmaxf(M, zn);
     for (int c0 = 0; c0 < n; c0 += kMergeMax) {
       const int cn = min(kMergeMax, n - c0);
@@ -782,7 +798,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
         s_w[u] = w;
         s_slot[u] = sl;
       }
-      L += merge_reduce(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
+      L += merge_reduce<kMergeThreads>(lpart, false, s_red);  // ends with a barrier: s_w, s_slot visible
       for (int u0 = grp; u0 < cn; u0 += kMergeGroups * kMergeBatch) {
         float4 v[kMergeBatch];
         float wv[kMergeBatch];
@@ -817,10 +833,24 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
   }
   s_acc[grp][f4] = acc;
   __syncthreads();
+  if constexpr (kMergeGroups > 8) {  // fold the groups to 8 first, in parallel
+    if (tid < 8 * 32) {
+      float4 r = s_acc[grp][f4];
+#pragma unroll
+      for (int g2 = grp + 8; g2 < kMergeGroups; g2 += 8) {
+        r.x += s_acc[g2][f4].x;
+        r.y += s_acc[g2][f4].y;
+        r.z += s_acc[g2][f4].z;
+        r.w += s_acc[g2][f4].w;
+      }
+      s_acc[grp][f4] = r;
+    }
+    __syncthreads();
+  }
   if (tid < 32) {
     float4 r = s_acc[0][tid];
 #pragma unroll
-    for (int g2 = 1; g2 < kMergeGroups; ++g2) {
+    for (int g2 = 1; g2 < (kMergeGroups < 8 ? kMergeGroups : 8); ++g2) {
       r.x += s_acc[g2][tid].x;
       r.y += s_acc[g2][tid].y;
       r.z += s_acc[g2][tid].z;
@@ -996,15 +1026,20 @@ cudaError_t launch_tensor_decode(const TensorDecodeArgs& a, cudaStream_t stream)
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cv.batch, kH);
-  cfg.blockDim = dim3(kMergeThreads);
+  const bool small_batch = cv.batch <= 2;
+  cfg.blockDim = dim3(small_batch ? kMergeThreadsSmallBatch : 256);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (a.step) return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<true>, mp);
-  return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<false>, mp);
+  if (small_batch) {
+    if (a.step) return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<true, kMergeThreadsSmallBatch>, mp);
+    return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<false, kMergeThreadsSmallBatch>, mp);
+  }
+  if (a.step) return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<true, 256>, mp);
+  return cudaLaunchKernelEx(&cfg, decode_tc_merge_kernel<false, 256>, mp);
 }
 
 }  // namespace tpa

@@ -419,3 +419,36 @@ def test_plan_stages_its_inputs_from_pinned_host_memory():
     assert c_init(dev_in, pageable) == 3      # TPA_ERR_UNSUPPORTED
     assert c_init(host_in, host_in) == 3
     assert c_init(dev_in, host_in) == T.TPA_OK
+
+
+@pytest.mark.parametrize("lengths", [[60000], [40001, 1], [0, 30000]])
+@pytest.mark.parametrize("grid", [0, 300])
+@pytest.mark.parametrize("r_q", [0, 6])
+def test_small_batch_merge(lengths, grid, r_q):
+    """A batch of one or two sequences, each split over many CTAs: the merge then runs 1024
+    threads a CTA and loads every partial in one pass (with 300 CTAs, more partials than one
+    pass holds).  The plain decode with its log-sum-exp and the fused step against the oracle."""
+    w = S.WORKLOADS["decode_b8_l8k"].replace(name="small_batch", seed=91)
+    B, cap = len(lengths), max(lengths) + 2
+    cache, x, q, q_pos = build_decode_cache(w, batch=B, length=cap, lengths=lengths)
+    cpu = readback(cache)
+    scale = default_scale(w.head_dim)
+    if r_q == 0:
+        out, lse = T.tpa_decode_attention_lse(cache, q, q_pos, max_len=cap, num_splits=grid)
+        for b, L in enumerate(lengths):
+            ref, ref_lse = O.decode_attention_lse(cpu["a_k"][b, :L], cpu["b_k"][b, :L], cpu["a_v"][b, :L],
+                                                  cpu["b_v"][b, :L], f64(q[b]), float(q_pos[b]), scale,
+                                                  w.rope_base)
+            if L:
+                assert_rows_close(f64(out[b]), ref, BF16, f"decode b={b}")
+                # an absolute error e in the log-sum-exp is a relative error e in the softmax's sum
+                assert np.abs(f64(lse[b]) - ref_lse).max() <= BF16, f"lse b={b}"
+            else:
+                assert torch.count_nonzero(out[b]) == 0 and torch.isneginf(lse[b]).all()
+    tok = _token(w, B, 92, r_q)
+    pos = cache.seq_lens.clone()
+    got = f64(_step(cache, tok, pos, max_len=cap, num_splits=grid))
+    for b in range(B):
+        ref, _ = _oracle(cpu, lengths, tok, pos.cpu(), w, b)
+        assert_rows_close(got[b], ref, BF16, f"step b={b}")
+    assert T.tpa_read_device_error() == 0
