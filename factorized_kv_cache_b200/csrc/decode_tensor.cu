@@ -583,20 +583,23 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
   const int b = blockIdx.x, i = blockIdx.y, tid = threadIdx.x;
   const int f4 = tid & 31, grp = tid >> 5;  // float4 column, partial group
 
-  // ---- the step's token for head i: score z_t (log2 units) and value V_t (columns 4 f4 ..
-  // 4 f4 + 3), every input load issued before the first is used
+  // ---- the step's token for head i: score z_t (log2 units, warps 0-1) and value V_t (columns
+  // 4 f4 .. 4 f4 + 3, warp kVnWarp), both chains' loads issued at once
+  constexpr int kVnWarp = 2;
+  const bool vn_warp = (tid >> 5) == kVnWarp;
   float zn = 0.f;
   float4 vn = make_float4(0.f, 0.f, 0.f, 0.f);
   uint32_t bkr[2] = {0u, 0u};  // rotated B_K pair 2 tid, 2 tid + 1 of rank rows 0, 1 (bf16 x 2), tid < 64
   uint32_t word = 0u;          // one 4-byte word of the token's A_K | A_V | B_V, head-0 CTA, tid >= 64
+  __shared__ float s_dot[2];
   if constexpr (kStep) {
     const TcStepParams& st = p.st;
     const int R = st.r;
-    float ak[2] = {0.f, 0.f};
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-      if (r < R) ak[r] = __bfloat162float(st.a_k[(static_cast<size_t>(b) * R + r) * kH + i]);
     if (tid < 64) {
+      float ak[2] = {0.f, 0.f};
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+        if (r < R) ak[r] = __bfloat162float(st.a_k[(static_cast<size_t>(b) * R + r) * kH + i]);
       const int pos = st.pos[b];
       __nv_bfloat162 kk[2], qq[8];
       float aq[8];
@@ -648,19 +651,29 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      if ((tid & 31) == 0) s_red[tid >> 5] = dot;
-    }
-    if (tid < 32) {
-      for (int r = 0; r < R; ++r) {
-        const size_t row = static_cast<size_t>(b) * R + r;
-        const float a = __bfloat162float(st.a_v[row * kH + i]) * st.inv_rv;
-        const uint2 raw = reinterpret_cast<const uint2*>(st.b_v + row * kD)[tid];
-        const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-        const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-        vn.x = fmaf(a, __low2float(v01), vn.x);
-        vn.y = fmaf(a, __high2float(v01), vn.y);
-        vn.z = fmaf(a, __low2float(v23), vn.z);
-        vn.w = fmaf(a, __high2float(v23), vn.w);
+      if ((tid & 31) == 0) s_dot[tid >> 5] = dot;
+    } else if (vn_warp) {
+      float av[2] = {0.f, 0.f};
+      uint2 raw[2] = {make_uint2(0u, 0u), make_uint2(0u, 0u)};
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (r < R) {
+          const size_t row = static_cast<size_t>(b) * R + r;
+          av[r] = __bfloat162float(st.a_v[row * kH + i]);
+          raw[r] = reinterpret_cast<const uint2*>(st.b_v + row * kD)[f4];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        if (r < R) {
+          const float a = av[r] * st.inv_rv;
+          const __nv_bfloat162 v01 = *reinterpret_cast<const __nv_bfloat162*>(&raw[r].x);
+          const __nv_bfloat162 v23 = *reinterpret_cast<const __nv_bfloat162*>(&raw[r].y);
+          vn.x = fmaf(a, __low2float(v01), vn.x);
+          vn.y = fmaf(a, __high2float(v01), vn.y);
+          vn.z = fmaf(a, __low2float(v23), vn.z);
+          vn.w = fmaf(a, __high2float(v23), vn.w);
+        }
       }
     }
     if (blockIdx.y == 0 && tid >= 64) {
@@ -671,8 +684,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
         word = reinterpret_cast<const uint32_t*>(st.b_v + static_cast<size_t>(b) * R * kD)[w - 2 * na];
     }
     __syncthreads();
-    zn = (s_red[0] + s_red[1]) * st.zs;
-    __syncthreads();  // s_red is reused by the merge below
+    zn = (s_dot[0] + s_dot[1]) * st.zs;
   }
 
   ptx::pdl_wait();  // the split kernel's partials, outputs and recorded lengths
@@ -711,7 +723,7 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
     if (lse && tid == 0) *lse = l > 0.f ? (m2 + log2f(l)) * kLn2 : -INFINITY;
   };
   if (t1 <= t0) {  // nothing cached: the step's token alone, or zeros
-    if (tid < 32) reinterpret_cast<float4*>(o)[tid] = nv ? vn : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (vn_warp) reinterpret_cast<float4*>(o)[f4] = nv ? vn : make_float4(0.f, 0.f, 0.f, 0.f);
     write_lse(nv ? zn : 0.f, nv ? 1.f : 0.f);
     return;
   }
@@ -724,10 +736,10 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       const float M = nv ? fmaxf(ml.x, zn) : ml.x;
       const float wo = (ml.x == -INFINITY ? 0.f : exp2f(ml.x - M)) * ml.y;
       const float wn = nv ? exp2f(zn - M) : 0.f;
-      if (nv && tid < 32) {
-        const float4 on = reinterpret_cast<const float4*>(o)[tid];
+      if (nv && vn_warp) {
+        const float4 on = reinterpret_cast<const float4*>(o)[f4];
         const float inv = 1.f / (wo + wn);
-        reinterpret_cast<float4*>(o)[tid] = make_float4((on.x * wo + vn.x * wn) * inv, (on.y * wo + vn.y * wn) * inv,
+        reinterpret_cast<float4*>(o)[f4] = make_float4((on.x * wo + vn.x * wn) * inv, (on.y * wo + vn.y * wn) * inv,
                                                         (on.z * wo + vn.z * wn) * inv, (on.w * wo + vn.w * wn) * inv);
       }
       write_lse(M, wo + wn);
@@ -821,10 +833,10 @@ __global__ void __launch_bounds__(kMergeThreads) decode_tc_merge_kernel(const __
       __syncthreads();  // s_w, s_slot are rewritten by the next pass
     }
   }
-  if (nv) {  // the step's token: one more partial (z_t, 1, V_t), added once (group 0 holds V_t)
+  if (nv) {  // the step's token: one more partial (z_t, 1, V_t), added once (warp kVnWarp holds V_t)
     const float wn = exp2f(zn - M);
     L += wn;
-    if (grp == 0) {
+    if (vn_warp) {
       acc.x = fmaf(vn.x, wn, acc.x);
       acc.y = fmaf(vn.y, wn, acc.y);
       acc.z = fmaf(vn.z, wn, acc.z);
