@@ -103,6 +103,9 @@ static_assert(kStageBytes % 1024 == 0 && kBBox % 1024 == 0, "swizzle atoms stay 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256, kColQ = 384;
 constexpr unsigned kErrTimeout = 0x8u;
+constexpr int kOPitch = kD + 4;          // floats per staged output row (528 bytes)
+constexpr uint32_t kEpilogueBar = 5;     // named barrier of the softmax warps (1-4: the row pairs)
+static_assert(kQ * kOPitch * 4 <= kStages * kStageBytes, "the staged output fits in the K/V stages");
 constexpr float kLazy = 4.f;  // rescale only when a row maximum grows by more than 2^4
 constexpr float kShift = 2.f;  // p = 2^(z - m - kShift): at most 2^(kLazy - kShift) = 4
 constexpr int kMaxRq = 8;
@@ -145,6 +148,26 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return *reinterpret_cast<const float2*>(&d);
 }
 
+// max of three (one instruction)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// The maximum of n values as a tree of three-input maxima (depth log3 n instead of n).
+template <int N>
+__device__ __forceinline__ float max_tree(const float* v) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else if constexpr (N == 2) {
+    return fmaxf(v[0], v[1]);
+  } else {
+    constexpr int A = (N + 2) / 3, B = (N - A + 1) / 2;
+    return max3(max_tree<A>(v), max_tree<B>(v + A), max_tree<N - A - B>(v + A + B));
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   const __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -163,14 +186,22 @@ struct PrepParams {
   const int32_t* q_pos;       // [B][T]
   __half* wk;                 // fp16 copies [B][cap][R][128]
   __half* wv;
-  __half* wq;                 // [B][T][R_Q][128] rotated
+  __half* wq;                 // rotated rank rows, interleaved by 32 queries (wq_chunk)
   RopeTable rope;
 };
 
+// The rotated B_Q rank rows in the workspace, in 16-byte chunks of 8 features: chunk c (features
+// 64 hf + 8 c .. + 7) of rank j of query t = 32 blk + r sits at this index, so that the 32 queries
+// a warp of the attention kernel forms (one per lane) read 512 contiguous bytes per load.
+__host__ __device__ __forceinline__ size_t wq_chunk(int b, int n_blk, int blk, int r_q, int j, int hf, int c, int r) {
+  return (((static_cast<size_t>(b) * n_blk + blk) * r_q + j) * 16 + hf * 8 + c) * 32 + r;
+}
+
 // The pre-pass.  blockIdx.z = 0, 1: fp16 copies of the B_K, B_V rows of every sequence's
 // cached tokens (slots below seq_lens[b]), blockIdx.y striding over the sequences; z = 2: the
-// chunk's B_Q rank rows rotated at their positions (one thread per (query, pair): the pair's
-// cos and sin are formed once for all ranks), rounded to fp16.
+// chunk's B_Q rank rows rotated at their positions, rounded to fp16, into the interleaved layout
+// of wq_chunk (one thread per (query, 8 features), queries fastest: the cos and sin of its 4
+// pairs are formed once for all ranks).
 __global__ void __launch_bounds__(256) prefill_prep_kernel(const __grid_constant__ PrepParams p) {
   ptx::pdl_launch_dependents();  // the attention grid may start its set-up
   if (blockIdx.z < 2) {
@@ -193,20 +224,34 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const __grid_constant
     }
     return;
   }
-  const size_t n = static_cast<size_t>(p.batch) * p.n_tokens * (kD / 2);
+  const int n_blk = (p.n_tokens + 31) / 32;
+  const size_t n = static_cast<size_t>(p.batch) * n_blk * 16 * 32;
   const size_t stride = static_cast<size_t>(gridDim.x) * gridDim.y * blockDim.x;
   for (size_t e = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x; e < n;
        e += stride) {
-    const size_t qrow = e / (kD / 2);  // b * T + t
-    const int pr = static_cast<int>(e % (kD / 2));
-    float c, sn;
-    rope_cos_sin(p.q_pos[qrow], p.rope.theta[pr], &c, &sn);
+    const int r = static_cast<int>(e % 32);
+    const int ch = static_cast<int>((e / 32) % 16);  // features 8 ch .. 8 ch + 7: pairs 4 ch .. 4 ch + 3
+    const int blk = static_cast<int>((e / 512) % n_blk);
+    const int b = static_cast<int>(e / (512 * static_cast<size_t>(n_blk)));
+    const int t = 32 * blk + r;
+    if (t >= p.n_tokens) continue;
+    const size_t qrow = static_cast<size_t>(b) * p.n_tokens + t;
+    const int pos = p.q_pos[qrow];
+    float cs[4], sn[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rope_cos_sin(pos, p.rope.theta[4 * ch + k], &cs[k], &sn[k]);
+    uint4* dst = reinterpret_cast<uint4*>(p.wq);
     for (int j = 0; j < p.r_q; ++j) {
-      const size_t off = (qrow * p.r_q + j) * kD / 2 + pr;  // in pairs
-      const uint32_t w = reinterpret_cast<const uint32_t*>(p.b_q)[off];
-      float x = ptx::bf16_lo(w), y = ptx::bf16_hi(w);
-      rope_pair(x, y, c, sn);
-      reinterpret_cast<uint32_t*>(p.wq)[off] = pack_f16(x, y);
+      const uint4 x = reinterpret_cast<const uint4*>(p.b_q + (qrow * p.r_q + j) * kD)[ch];
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t y[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float a = ptx::bf16_lo(w[k]), bb = ptx::bf16_hi(w[k]);
+        rope_pair(a, bb, cs[k], sn[k]);
+        y[k] = pack_f16(a, bb);
+      }
+      dst[wq_chunk(b, n_blk, blk, p.r_q, j, ch >> 3, ch & 7, r)] = make_uint4(y[0], y[1], y[2], y[3]);
     }
   }
 }
@@ -428,7 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t pair_bar = 1 + quad;        // named barrier of warps (quad, half 0) and (quad, half 1)
     // features [64 hf, +64) of this thread's query row, q = (1/R_Q) sum_j A_Q[t, j, head] B~_Q[t, j]
     // from the rotated rank rows of the pre-pass (read after the wait on it), formed in fp32 and
-    // rounded once to fp16 in TMEM
+    // rounded once to fp16 in TMEM.  The rank rows are interleaved by 32 queries (wq_chunk), so
+    // each load of the warp reads 512 contiguous bytes; two ranks' 16 loads are issued at once.
     {
       const size_t qrow = static_cast<size_t>(b) * p.n_tokens + tq;
       const bool real = tq < p.n_tokens;
@@ -437,22 +483,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < kMaxRq; ++j)
         aq[j] = (real && j < p.r_q) ? __bfloat162float(p.a_q[(qrow * p.r_q + j) * kH + head]) * p.inv_rq : 0.f;
       ptx::pdl_wait();  // the rotated rank rows
+      const int n_blk = (p.n_tokens + 31) / 32;
+      const uint4* src = reinterpret_cast<const uint4*>(p.bq_rot) +
+                         wq_chunk(b, n_blk, q0 / 32 + quad, p.r_q, 0, hf, 0, lane);  // rank j, chunk c: + 512 j + 32 c
       float acc[64];
 #pragma unroll
       for (int e = 0; e < 64; ++e) acc[e] = 0.f;
 #pragma unroll
-      for (int j = 0; j < kMaxRq; ++j) {
-        if (real && j < p.r_q) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.bq_rot + (qrow * p.r_q + j) * kD + 64 * hf);
+      for (int j0 = 0; j0 < kMaxRq; j0 += 2) {
+        uint4 v[2][8];
+#pragma unroll
+        for (int jr = 0; jr < 2; ++jr) {
+          const bool use = real && j0 + jr < p.r_q;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[jr][c] = use ? src[512 * (j0 + jr) + 32 * c] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int jr = 0; jr < 2; ++jr) {
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const uint4 v = src[c];
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t w[4] = {v[jr][c].x, v[jr][c].y, v[jr][c].z, v[jr][c].w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const float2 f = unpack_f16(w[k]);
-              acc[8 * c + 2 * k] = fmaf(aq[j], f.x, acc[8 * c + 2 * k]);
-              acc[8 * c + 2 * k + 1] = fmaf(aq[j], f.y, acc[8 * c + 2 * k + 1]);
+              acc[8 * c + 2 * k] = fmaf(aq[j0 + jr], f.x, acc[8 * c + 2 * k]);
+              acc[8 * c + 2 * k + 1] = fmaf(aq[j0 + jr], f.y, acc[8 * c + 2 * k + 1]);
             }
           }
         }
@@ -503,11 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int tok0 = j * TOK + TOKH * hf;  // first token of this thread's rows
         const bool need_mask = j * TOK + TOK - 1 > P + q0;  // the tile reaches past some query's own slot
+        if (need_mask) {
 #pragma unroll
-        for (int s = 0; s < TOKH; ++s) {
-          if (need_mask && tok0 + s > qslot) z[s] = -INFINITY;
-          mx = fmaxf(mx, z[s]);
+          for (int s = 0; s < TOKH; ++s)
+            if (tok0 + s > qslot) z[s] = -INFINITY;
         }
+        mx = max_tree<TOKH>(z);
       }
       // ---- the row maximum over both halves of the tile: exchange with the partner thread.
       // The pair barrier also orders both threads' S loads before either writes W over S, and
@@ -597,23 +653,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::named_barrier(pair_bar, 64);
       l += s_l[(1 - hf) * kQ + row];
     }
+    // O / l goes through shared memory, so that each warp then writes whole 512-byte output rows
+    // (one row of out[b][t][head][:] per instruction) instead of 16 bytes into 32 rows 16 KB
+    // apart.  Once every MMA has completed (fin), the K/V stages are no longer read or written:
+    // rows of kOPitch floats there, padded so that the 32 rows a warp writes at once spread over
+    // the banks.
     const bool o_ready = ok && ptx::mbar_wait_bounded(fin, 0);
-    if (__all_sync(0xffffffffu, o_ready)) {  // the TMEM loads below are warp-wide
+    const bool warp_ready = __all_sync(0xffffffffu, o_ready);  // the TMEM loads below are warp-wide
+    float* s_o = reinterpret_cast<float*>(gbase + kOffStages);
+    if (warp_ready) {
       ptx::tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      float* op = p.out + ((static_cast<size_t>(b) * p.n_tokens + tq) * kH + head) * kD + 64 * hf;
 #pragma unroll
       for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t ov[32];
         ptx::tmem_ld32(tbase + lane_off + kColO + 64 * hf + 32 * c2, ov);
         ptx::tmem_wait_ld();
-        if (tq < p.n_tokens) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            *reinterpret_cast<float4*>(op + 32 * c2 + e) =
-                make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
-                            __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
-          }
+        for (int e = 0; e < 32; e += 4) {
+          *reinterpret_cast<float4*>(s_o + row * kOPitch + 64 * hf + 32 * c2 + e) =
+              make_float4(__uint_as_float(ov[e]) * inv, __uint_as_float(ov[e + 1]) * inv,
+                          __uint_as_float(ov[e + 2]) * inv, __uint_as_float(ov[e + 3]) * inv);
         }
       }
     } else if (ok && lane == 0) {
@@ -621,6 +681,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       *s_abort = 1;
     }
     ptx::tc_fence_before();
+    // every softmax warp reaches this barrier; its OR says whether any of them could not stage O
+    if (!ptx::named_barrier_or(kEpilogueBar, kSoftmaxWarps * 32, !warp_ready)) {
+      const int sw = warp - 2;  // rows 16 sw .. 16 sw + 15
+#pragma unroll 4
+      for (int r = 16 * sw; r < 16 * sw + 16; ++r) {
+        if (q0 + r < p.n_tokens) {
+          const float4 v = reinterpret_cast<const float4*>(s_o + r * kOPitch)[lane];
+          reinterpret_cast<float4*>(p.out + ((static_cast<size_t>(b) * p.n_tokens + q0 + r) * kH + head) * kD)[lane] = v;
+        }
+      }
+    }
   }
   // The TMA and MMA warps ran their loops on lane 0 alone: reconverge them first, so that the
   // CTA barrier counts every thread and TMEM is released only after every role is done.
@@ -660,7 +731,8 @@ bool tensor_prefill_supported(int dtype, int heads, int head_dim, int r_k, int r
 namespace {
 
 // The workspace: fp16 copies of B_K and B_V [B][cap][R][128], then the rotated rank rows
-// [B][T][R_Q][128] (fp16), each section 256-byte aligned.
+// (fp16, B x T rounded up to 32 x R_Q x 128, interleaved as wq_chunk says), each section
+// 256-byte aligned.
 struct PrefillWorkspace {
   __half* wk;
   __half* wv;
@@ -670,7 +742,7 @@ struct PrefillWorkspace {
 
 PrefillWorkspace carve_prefill(void* base, int batch, int capacity, int r, int n_tokens, int r_q) {
   const size_t plane = round256(static_cast<size_t>(batch) * capacity * r * kD * 2);
-  const size_t qb = round256(static_cast<size_t>(batch) * n_tokens * r_q * kD * 2);
+  const size_t qb = round256(static_cast<size_t>(batch) * ((n_tokens + 31) / 32 * 32) * r_q * kD * 2);
   char* c = static_cast<char*>(base);
   PrefillWorkspace w;
   w.wk = reinterpret_cast<__half*>(c);

@@ -352,8 +352,10 @@ tpa_status tpa_decode_attention_noalloc(const tpa_cache* cache, const void* q, c
 /* Workspace bytes tpa_prefill_attention needs: on the tensor-core path, fp16
  * copies of the cache's B_K and B_V planes (2 * batch * capacity * r_k *
  * head_dim * 2 bytes) and the chunk's B_Q rank rows rotated at their
- * positions (batch * n_tokens * r_q * head_dim * 2 bytes; the dense
- * per-head queries are formed inside the kernel and never stored); on the
+ * positions (batch * n_tokens32 * r_q * head_dim * 2 bytes, n_tokens32 =
+ * n_tokens rounded up to a multiple of 32; the dense per-head queries are
+ * formed inside the kernel and never stored), each part rounded up to 256
+ * bytes; on the
  * CUDA-core path, the dense rotated fp32 queries (batch * n_tokens * heads *
  * head_dim * 4 bytes). */
 size_t tpa_prefill_workspace_size(const tpa_cache* cache, int32_t n_tokens, int32_t r_q,

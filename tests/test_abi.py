@@ -222,12 +222,13 @@ def test_workspace_sizes_follow_the_split_plan():
 
 def test_prefill_workspace_sizes():
     """The tensor-core prefill's workspace: fp16 copies of the B_K and B_V planes and the
-    chunk's rotated B_Q rank rows (no dense query); the CUDA-core prefill's: dense fp32 queries."""
+    chunk's rotated B_Q rank rows, the chunk padded to whole 32-query blocks (no dense query); the
+    CUDA-core prefill's: dense fp32 queries."""
     lib = T.load_library()
     r256 = lambda n: (n + 255) // 256 * 256
     for B, cap, r, n, rq in ((4, 4096, 2, 4096, 6), (3, 1000, 1, 77, 1), (1, 64, 2, 5, 8)):
         c = _fake_cache(batch=B, capacity=cap, r_k=r, r_v=r)
-        want = 2 * r256(B * cap * r * 128 * 2) + r256(B * n * rq * 128 * 2)
+        want = 2 * r256(B * cap * r * 128 * 2) + r256(B * ((n + 31) // 32 * 32) * rq * 128 * 2)
         assert lib.tpa_prefill_workspace_size(ctypes.byref(c), n, rq, T.TPA_KERNEL_AUTO) == want
         assert lib.tpa_prefill_workspace_size(ctypes.byref(c), n, rq, T.TPA_KERNEL_SIMT) == r256(B * n * 32 * 128 * 4)
     # the prefill workload: 42 MB instead of the 268 MB of dense fp32 queries
