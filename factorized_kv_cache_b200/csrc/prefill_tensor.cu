@@ -94,8 +94,8 @@ constexpr int kOffA = kOffStages + kStages * kStageBytes;  // fp32 [2 buffers][A
 constexpr int kOffMx = kOffA + 2 * 2 * kRows * 4;          // fp32 [2 buffers][2 halves][128 rows]
 constexpr int kOffL = kOffMx + 2 * 2 * kQ * 4;             // fp32 [2 halves][128 rows]
 constexpr int kOffBar = kOffL + 2 * kQ * 4;
-// full[3], empty[3], sfull[2], wready[2], odone, staged[2], qready, fin
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 1 + 2 + 1 + 1;
+// full[3], empty[3], sfull[2], wready[2], staged[2], qready, fin
+constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 1 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -275,10 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto empty = [&](int s) { return bar0 + 8 * (kStages + s); };
   auto sfull = [&](int b) { return bar0 + 8 * (2 * kStages + b); };
   auto wready = [&](int b) { return bar0 + 8 * (2 * kStages + 2 + b); };
-  const uint32_t odone = bar0 + 8 * (2 * kStages + 4);
-  auto staged = [&](int b) { return bar0 + 8 * (2 * kStages + 5 + b); };
-  const uint32_t qready = bar0 + 8 * (2 * kStages + 7);
-  const uint32_t fin = bar0 + 8 * (2 * kStages + 8);
+  auto staged = [&](int b) { return bar0 + 8 * (2 * kStages + 4 + b); };
+  const uint32_t qready = bar0 + 8 * (2 * kStages + 6);
+  const uint32_t fin = bar0 + 8 * (2 * kStages + 7);
   volatile uint32_t* s_taddr = reinterpret_cast<volatile uint32_t*>(gbase + kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(gbase + kOffMisc + 4);
 
@@ -310,7 +309,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(wready(bf), kSoftmaxWarps);
       ptx::mbar_init(staged(bf), 1);
     }
-    ptx::mbar_init(odone, 1);
     ptx::mbar_init(qready, kSoftmaxWarps);
     ptx::mbar_init(fin, 1);
     *s_abort = 0;
@@ -388,7 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (j + 1 < nk) {
           ok = ptx::mbar_wait_bounded(full((j + 1) % kStages), ((j + 1) / kStages) & 1);
-          if (ok && j > 0) ok = ptx::mbar_wait_bounded(odone, (j - 1) & 1);
+          // the value MMA of tile j-1 has read W(j-1) there: its stage's release says so (the
+          // stager's arrival for that stage came long before)
+          if (ok && j > 0) ok = ptx::mbar_wait_bounded(empty((j - 1) % kStages), ((j - 1) / kStages) & 1);
           if (!ok) break;
           ptx::tc_fence_after();
           score(j + 1);
@@ -402,8 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t db = ptx::umma_desc_sw128(bv + kk * 2048, kBBox, 1024);
           ptx::umma_ts(tbase + kColO, ts + kk * 8, db, kIdescValue, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::umma_commit(odone);
-        ptx::umma_commit(empty(j % kStages));
+        ptx::umma_commit(empty(j % kStages));  // also tells the softmax that O holds tile j
       }
       if (!ok) {
         if (!*s_abort) atomicOr(p.err, kErrTimeout);
@@ -590,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j > 0 && __any_sync(0xffffffffu, grow)) {
         // the value MMA of tile j-1 may still be accumulating into O; a timeout here is
         // acted on at the next pair barrier, which both warps of the pair reach
-        const bool o_prev = ptx::mbar_wait_bounded(odone, (j - 1) & 1);
+        const bool o_prev = ptx::mbar_wait_bounded(empty((j - 1) % kStages), ((j - 1) / kStages) & 1);
         if (__all_sync(0xffffffffu, o_prev)) {
           ptx::tc_fence_after();
 #pragma unroll
