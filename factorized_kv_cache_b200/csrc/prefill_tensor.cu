@@ -211,15 +211,23 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const __grid_constant
       const uint4* src = reinterpret_cast<const uint4*>((blockIdx.z == 0 ? p.b_k : p.b_v) + base);
       uint4* dst = reinterpret_cast<uint4*>((blockIdx.z == 0 ? p.wk : p.wv) + base);
       const size_t nvec = static_cast<size_t>(len) * p.r * kD / 8;
-      for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
-           v += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const uint4 x = src[v];
-        uint4 y;
-        y.x = pack_f16(ptx::bf16_lo(x.x), ptx::bf16_hi(x.x));
-        y.y = pack_f16(ptx::bf16_lo(x.y), ptx::bf16_hi(x.y));
-        y.z = pack_f16(ptx::bf16_lo(x.z), ptx::bf16_hi(x.z));
-        y.w = pack_f16(ptx::bf16_lo(x.w), ptx::bf16_hi(x.w));
-        dst[v] = y;
+      const size_t step = static_cast<size_t>(gridDim.x) * blockDim.x;
+      // four 16-byte vectors per thread in flight, each load of the warp 512 contiguous bytes
+      for (size_t v = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec; v += 4 * step) {
+        uint4 x[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = v + k * step < nvec ? src[v + k * step] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (v + k * step < nvec) {
+            uint4 y;
+            y.x = pack_f16(ptx::bf16_lo(x[k].x), ptx::bf16_hi(x[k].x));
+            y.y = pack_f16(ptx::bf16_lo(x[k].y), ptx::bf16_hi(x[k].y));
+            y.z = pack_f16(ptx::bf16_lo(x[k].z), ptx::bf16_hi(x[k].z));
+            y.w = pack_f16(ptx::bf16_lo(x[k].w), ptx::bf16_hi(x[k].w));
+            dst[v + k * step] = y;
+          }
+        }
       }
     }
     return;
@@ -241,17 +249,23 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const __grid_constant
 #pragma unroll
     for (int k = 0; k < 4; ++k) rope_cos_sin(pos, p.rope.theta[4 * ch + k], &cs[k], &sn[k]);
     uint4* dst = reinterpret_cast<uint4*>(p.wq);
-    for (int j = 0; j < p.r_q; ++j) {
-      const uint4 x = reinterpret_cast<const uint4*>(p.b_q + (qrow * p.r_q + j) * kD)[ch];
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-      uint32_t y[4];
+    uint4 x[kMaxRq];  // every rank's 16 bytes in flight at once
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float a = ptx::bf16_lo(w[k]), bb = ptx::bf16_hi(w[k]);
-        rope_pair(a, bb, cs[k], sn[k]);
-        y[k] = pack_f16(a, bb);
+    for (int j = 0; j < kMaxRq; ++j)
+      x[j] = j < p.r_q ? reinterpret_cast<const uint4*>(p.b_q + (qrow * p.r_q + j) * kD)[ch] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < kMaxRq; ++j) {
+      if (j < p.r_q) {
+        const uint32_t w[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+        uint32_t y[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float a = ptx::bf16_lo(w[k]), bb = ptx::bf16_hi(w[k]);
+          rope_pair(a, bb, cs[k], sn[k]);
+          y[k] = pack_f16(a, bb);
+        }
+        dst[wq_chunk(b, n_blk, blk, p.r_q, j, ch >> 3, ch & 7, r)] = make_uint4(y[0], y[1], y[2], y[3]);
       }
-      dst[wq_chunk(b, n_blk, blk, p.r_q, j, ch >> 3, ch & 7, r)] = make_uint4(y[0], y[1], y[2], y[3]);
     }
   }
 }
@@ -777,12 +791,12 @@ cudaError_t launch_tensor_prefill(const TensorPrefillArgs& a, cudaStream_t strea
   pp.wv = ws.wv;
   pp.wq = ws.wq;
   pp.rope = a.rope;
-  // about four CTAs per SM over the three parts
+  // about eight CTAs of 256 threads per SM over the three parts
   const int sms = a.sms > 0 ? a.sms : 148;
   const int gy = min(cv.batch, 65535);
   const size_t vec_per_seq = static_cast<size_t>(cv.capacity) * R * kD / 8;
-  size_t gx = (vec_per_seq + 255) / 256;
-  const size_t cap_x = static_cast<size_t>(max(1, 4 * sms / max(1, 3 * gy)));
+  size_t gx = (vec_per_seq + 4 * 256 - 1) / (4 * 256);
+  const size_t cap_x = static_cast<size_t>(max(1, 8 * sms / max(1, 3 * gy)));
   if (gx > cap_x) gx = cap_x;
   if (gx < 1) gx = 1;
   prefill_prep_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 3), 256, 0, stream>>>(pp);
