@@ -912,7 +912,8 @@ def run_ours_prefill(args, w, rank, world, dev):
         "config": {"workload": w.name, "batch": B, "seq_len": Tn, "heads": w.heads, "head_dim": w.head_dim,
                    "r_q": w.r_q, "r_k": w.r_k, "r_v": w.r_v, "kernel": args.kernel,
                    "step": "write prompt factors (RoPE on B_K) + causal prefill, CUDA graphs",
-                   "l2": "inputs larger than L2 (the 268 MB fp32 output and 42 MB of fp16 workspace per step)",
+                   "l2": f"inputs larger than L2 (the {out.numel() * 4 / 1e6:.0f} MB fp32 output and "
+                         f"{(ws.numel() if ws is not None else 0) / 1e6:.0f} MB of workspace per step)",
                    "parallelism": f"dp{world} (independent batches, no collective)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"],
