@@ -668,6 +668,17 @@ tpa_status tpa_read_device_error(uint32_t* code_out, void* stream) {
   return TPA_OK;
 }
 
+tpa_status tpa_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 10000000000ull) return fail(TPA_ERR_SHAPE, "limit_ns = %llu outside [1, 1e10]",
+                                                              static_cast<unsigned long long>(limit_ns));
+  unsigned int* err = nullptr;
+  cudaError_t e = device_info(nullptr, &err);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  e = launch_wait_timeout_selftest(limit_ns, err, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return TPA_OK;
+}
+
 const char* tpa_status_string(tpa_status status) {
   switch (status) {
     case TPA_OK: return "TPA_OK";

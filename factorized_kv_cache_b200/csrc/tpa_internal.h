@@ -104,4 +104,7 @@ struct PrefillQArgs {
 };
 cudaError_t launch_prefill_q(const PrefillQArgs& a, cudaStream_t stream);
 
+// one CTA waiting on a shared-memory barrier that nothing completes, for limit_ns
+cudaError_t launch_wait_timeout_selftest(uint64_t limit_ns, unsigned int* err, cudaStream_t stream);
+
 }  // namespace tpa

@@ -25,6 +25,7 @@ TPA_KERNEL_AUTO, TPA_KERNEL_SIMT, TPA_KERNEL_TENSOR, TPA_KERNEL_TENSOR_SYNC = 0,
 TPA_DEVERR_APPEND_OVERFLOW = 0x1
 TPA_DEVERR_LEN_RANGE = 0x2
 TPA_DEVERR_PREFILL_LEN = 0x4
+TPA_DEVERR_TIMEOUT = 0x8
 
 STATUS_NAMES = {
     0: "TPA_OK", 1: "TPA_ERR_NULL", 2: "TPA_ERR_SHAPE", 3: "TPA_ERR_UNSUPPORTED",
@@ -101,6 +102,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tpa_prefill_workspace_size": (ctypes.c_size_t, [C, I32, I32, I32]),
         "tpa_prefill_attention": (ctypes.c_int, [C, I32, I32, P, P, P, ctypes.c_float, P, I32, P, ctypes.c_size_t, P]),
         "tpa_read_device_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), P]),
+        "tpa_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, P]),
         "tpa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "tpa_last_error_message": (ctypes.c_char_p, []),
     }
@@ -613,6 +615,13 @@ def tpa_prefill_attention(cache: TpaCache, a_q, b_q, q_pos, scale: float | None 
     _check(lib.tpa_prefill_attention(ctypes.byref(s), T, r_q, _ptr(a_q), _ptr(b_q), _ptr(q_pos), float(scale),
                                      _ptr(out), kernel, _ptr(workspace_buf), nbytes, _stream(stream, dev)))
     return out
+
+
+def tpa_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test: one CTA waits limit_ns on a barrier nothing completes and
+    records TPA_DEVERR_TIMEOUT (read it with tpa_read_device_error)."""
+    lib = load_library()
+    _check(lib.tpa_selftest_wait_timeout(int(limit_ns), _stream(stream)))
 
 
 def tpa_read_device_error(stream=None) -> int:

@@ -75,6 +75,10 @@ typedef enum tpa_kernel {
 #define TPA_DEVERR_APPEND_OVERFLOW 0x1u /* an append reached a slot >= capacity */
 #define TPA_DEVERR_LEN_RANGE 0x2u       /* seq_lens[b] < 0, > capacity or > max_len */
 #define TPA_DEVERR_PREFILL_LEN 0x4u     /* prefill n_tokens > seq_lens[b] */
+#define TPA_DEVERR_TIMEOUT 0x8u         /* a tensor-core kernel's wait on its own pipeline (a
+                                         * shared-memory barrier another role of the CTA completes)
+                                         * ran past its 2 s limit; the kernel returned early and the
+                                         * call's outputs are not valid */
 
 /*
  * A factorized KV cache of `batch` sequences, `capacity` token slots each.
@@ -390,6 +394,14 @@ tpa_status tpa_prefill_attention(const tpa_cache* cache, int32_t n_tokens, int32
 /* Synchronise `stream`, copy the current device's error word to *code_out and
  * clear it.  Errors: NULL, CUDA. */
 tpa_status tpa_read_device_error(uint32_t* code_out, void* stream);
+
+/* Self-test of the bounded waits: launches one CTA that waits, for at most
+ * limit_ns nanoseconds, on a shared-memory barrier that nothing completes, the
+ * same bounded wait the tensor-core kernels use on their pipelines, and sets
+ * TPA_DEVERR_TIMEOUT when the limit passes.  The timeout path can thus be made
+ * to run without a fault: the kernel returns and the context stays usable.
+ * limit_ns in [1, 10^10].  Errors: SHAPE (limit_ns out of range), CUDA. */
+tpa_status tpa_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Static description of a status code. */
 const char* tpa_status_string(tpa_status status);

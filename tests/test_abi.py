@@ -220,6 +220,13 @@ def test_workspace_sizes_follow_the_split_plan():
     assert lib.tpa_decode_default_splits(ctypes.byref(c), 1 << 19, T.TPA_KERNEL_SIMT) >= 1
 
 
+def test_selftest_rejects_bad_limits():
+    lib = T.load_library()
+    assert lib.tpa_selftest_wait_timeout(0, None) == 2
+    assert lib.tpa_selftest_wait_timeout(10_000_000_001, None) == 2
+    assert lib.tpa_last_error_message().decode() != ""
+
+
 def test_prefill_workspace_sizes():
     """The tensor-core prefill's workspace: fp16 copies of the B_K and B_V planes and the
     chunk's rotated B_Q rank rows, the chunk padded to whole 32-query blocks (no dense query); the
