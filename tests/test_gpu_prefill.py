@@ -120,3 +120,35 @@ def test_last_prefill_row_equals_factored_decode(tokens, prior):
                                           q_pos[:, -1].contiguous(), max_len=L)
     assert T.tpa_read_device_error() == 0
     assert_rows_close(f64(dec), f64(out[:, -1]), 1.5e-3, "prefill last row vs factored decode")
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+def test_prefill_ragged_prior(kernel):
+    """Sequences with different numbers of cached tokens before the chunk (P = seq_lens[b] - T
+    differs per sequence): each query t of sequence b sits at slot P_b + t and attends slots
+    0 .. P_b + t.  The cache is written with explicit slots, so each sequence holds its own count."""
+    w = S.WORKLOADS["prefill_b4_t4k"]
+    priors, tokens = [37, 300, 0], 133
+    B, n = len(priors), max(priors) + tokens
+    x = S.prefill_inputs(w, batch=B, tokens=n)
+    cap = n + 5
+    cache = T.TpaCache.allocate(B, cap, w.heads, w.head_dim, w.r_k, w.r_v, dtype=TORCH_DTYPE[w.dtype],
+                                rope_base=w.rope_base, fill=float("nan"))
+    # sequence b: its first priors[b] + tokens tokens at slots 0.., the rest of the n written rows
+    # to the slots above, which its length excludes
+    slots = torch.empty(B, n, dtype=torch.int32)
+    for b, pr in enumerate(priors):
+        L = pr + tokens
+        slots[b, :L] = torch.arange(L, dtype=torch.int32)
+        slots[b, L:] = torch.arange(L, n, dtype=torch.int32)
+    T.tpa_cache_write_slots(cache, slots.to(DEV), x["positions"].to(DEV), *(x[k].to(DEV) for k in ("a_k", "b_k", "a_v", "b_v")))
+    cache.seq_lens.copy_(torch.tensor([pr + tokens for pr in priors], dtype=torch.int32, device=DEV))
+    a_q = torch.stack([x["a_q"][b, pr:pr + tokens] for b, pr in enumerate(priors)]).contiguous().to(DEV)
+    b_q = torch.stack([x["b_q"][b, pr:pr + tokens] for b, pr in enumerate(priors)]).contiguous().to(DEV)
+    q_pos = torch.stack([x["positions"][b, pr:pr + tokens] for b, pr in enumerate(priors)]).contiguous().to(DEV)
+    out = T.tpa_prefill_attention(cache, a_q, b_q, q_pos, kernel=kernel)
+    assert T.tpa_read_device_error() == 0
+    got = f64(out)
+    for b, pr in enumerate(priors):
+        ref = _oracle(w, cache, x, pr, tokens, b)
+        assert_rows_close(got[b], ref, TOL[cache.dtype], f"prefill ragged b={b}")
