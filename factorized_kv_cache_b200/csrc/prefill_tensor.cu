@@ -16,17 +16,18 @@
 // the head factors on the query side of the MMA (a dense query tile per head)
 // costs 2 h d_h R_K tensor flops per (query, key) pair and little CUDA-core
 // work; contracting B_Q with B_K first would save tensor flops but needs
-// ~h R_Q R_K CUDA-core FMAs per pair to apply A_Q and A_K, on the path that
-// already bounds this kernel (the softmax).
+// ~h R_Q R_K CUDA-core FMAs per pair to apply A_Q and A_K, on the CUDA cores
+// that the softmax already keeps busy.
 //
 // Operands are fp16.  A pre-pass (prefill_prep_kernel, launched just before)
 // writes to the workspace (i) fp16 copies of the B_K and B_V rows of every
 // sequence's cached tokens, exact for bf16 values in fp16's normal range
 // (bf16's 8 significant bits fit in fp16's 11; magnitudes above 65504 are not
 // supported by this path and become infinite), and (ii) the chunk's B_Q rank
-// rows rotated at their positions, rounded to fp16.  The dense per-head query
-// is formed in this kernel from (ii) and A_Q, in fp32, and rounded once to
-// fp16 in TMEM; it is never written to global memory.  With the softmax
+// rows rotated at their positions, rounded to fp16 and interleaved by 32
+// queries (wq_chunk).  The dense per-head query is formed in this kernel from
+// (ii) and A_Q, in fp32, and rounded once to fp16 in TMEM; it is never written
+// to global memory.  With the softmax
 // weights also rounded once to fp16 (11 significant bits: ~4e-4 relative each
 // on the prefill workload, against ~3.5e-3 for a bf16 rounding) one MMA per
 // contraction suffices where bf16 needed a high + low pair.
@@ -55,9 +56,10 @@
 //       2.4e-4 to 16376 (the row sum takes the same factor, which cancels in
 //       O / l);
 //   O += W B_V  (B_V MN-major).
-// The softmax is the measured bound of this kernel (the tensor pipe idles most of the time), so
-// its per-tile work is trimmed: the second half of a thread's scores is loaded from TMEM while
-// the first half is weighted, and the weights use two-wide fp32 arithmetic.
+// The softmax's per-tile work is trimmed: the second half of a thread's scores is loaded from
+// TMEM while the first half is weighted, the row maximum is a tree of three-input maxima, and the
+// weights use two-wide fp32 arithmetic.  At the end O / l goes through shared memory (the K/V
+// stages, idle by then) and each warp writes whole 512-byte output rows.
 // Every wait is bounded (2 s); a timeout sets the error word and an abort
 // flag, and TMEM is released only after the MMA thread's last commit.
 #include <cuda.h>
